@@ -1,0 +1,396 @@
+"""Benchmark of the compressed all-reduce on B200: one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--schedule fused|three_stage]
+
+A step is one pass of the whole path (quantise -> reduce + requantise ->
+decode, all simulated ranks) for every codec of the workload, back to back.
+Default workload: ``large_int3_int4`` (N=2 simulated ranks x 1 GiB BF16 per
+rank, INT3 then INT4), the large-message configuration on which the HBM
+roofline target is defined; its inputs (2 GiB) are far larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Metric: GB/s = (simulated ranks x per-rank BF16 bytes x codecs) / time, plus
+the fraction of measured HBM bandwidth the dominant kernel reaches.  With
+``--gpus G`` (torchrun, one process per GPU) every GPU runs its own
+independent instance of the workload (weak scaling); there is no data-path
+collective -- the N simulated ranks of one instance live in one GPU's HBM.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "quantized all-reduce GB/s (N x input bytes/s) and % of HBM peak on 1 B200"
+TILE = 2048
+CODEC_C = {"bf16": 2.0, "fp8": 2304 / 2048, "int4": 1152 / 2048, "int3": 896 / 2048}
+KERNEL_SOURCES = ("quantized_precision_all_b200/csrc/lpar_kernels.cu", "quantized_precision_all_b200/csrc/lpar_codec.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+REF_TILES_PER_STEP = 256            # reference arm: 0.5 Mi elements per rank per step
+CPU_BASELINE_TILES = 16384          # cpu_baseline: 32 Mi elements (64 MiB) per rank
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy read+write)"
+    return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+# ---- algorithmic bytes per launch (reads + writes the definition requires) ------
+def kernel_names(codec, schedule, N):
+    if codec == "bf16":
+        return ["k_bf16_reduce<N=%d,fused>" % N] if schedule == "fused" else \
+            ["k_bf16_reduce<N=%d>" % N, "k_broadcast"]
+    if schedule == "fused":
+        return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d,fused>" % (codec, N)]
+    return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d>" % (codec, N), "k_decode<%s>" % codec]
+
+
+def algorithmic_bytes(kernel, codec, N, n):
+    c = CODEC_C[codec]
+    if kernel.startswith("k_quantize"):
+        return N * n * (2 + c)                        # read N BF16 messages, write N wires
+    if kernel.startswith("k_reduce") and kernel.endswith("fused>"):
+        return n * (N * c + c + 2 * N)                # read N wires, write gathered wire + N outputs
+    if kernel.startswith("k_reduce"):
+        return n * (N * c + c)
+    if kernel.startswith("k_decode"):
+        return n * (c + 2 * N)
+    if kernel.startswith("k_bf16_reduce") and kernel.endswith("fused>"):
+        return n * (2 * N + 2 + 2 * N)
+    if kernel.startswith("k_bf16_reduce"):
+        return n * (2 * N + 2)
+    if kernel == "k_broadcast":
+        return n * (2 + 2 * N)
+    raise ValueError(kernel)
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if taken on these sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    sha = source_sha()
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            kv = dict(re.findall(r"(\w+)=(\S+)", line))
+            if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("source_sha") == sha:
+                return int(kv["bytes_per_launch"])
+    return None
+
+
+# ---- clocks sampled during the timed region -------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- our arm -------------------------------------------------------------------------
+def run_ours(args, rank, world, device):
+    from quantized_precision_all_b200 import lpar as L
+
+    w = W.WORKLOADS[args.workload]
+    N, n = w.N, w.n
+    xs = W.make_inputs(w, device)
+    outs = [torch.empty_like(x) for x in xs]
+    ws_bytes = max(L.lpar_workspace_bytes(N, n, L.lpar_effective_codec(n, c, w.min_quant_bytes)) for c in w.codecs)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(stage_events=None):
+        for i, codec in enumerate(w.codecs):
+            L.lpar_allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream,
+                             stage_events=None if stage_events is None else stage_events[i])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    # (1) the timed region: K steps, CUDA events on the launching stream
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # (2) per-kernel durations, live: stage events recorded between the kernels
+    ksteps = max(1, min(args.steps, 200))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in w.codecs] for _ in range(ksteps)]
+    for s in range(ksteps):
+        step(evs[s])
+    torch.cuda.synchronize(device)
+    kern = {}
+    for ci, codec in enumerate(w.codecs):
+        eff = L.lpar_effective_codec(n, codec, w.min_quant_bytes)
+        names = kernel_names(eff, args.schedule, N)
+        bounds = [(0, 1), (1, 2), (2, 3)] if eff != "bf16" else [(1, 2), (2, 3)]
+        for name, (a, b) in zip(names, bounds):
+            tot = sum(evs[s][ci][a].elapsed_time(evs[s][ci][b]) for s in range(ksteps))
+            d = kern.setdefault(name, {"codec": eff, "ms_total": 0.0, "launches": 0})
+            d["ms_total"] += tot
+            d["launches"] += ksteps
+    for name, d in kern.items():
+        d["ms_per_launch"] = d["ms_total"] / d["launches"]
+        d["algorithmic_bytes"] = algorithmic_bytes(name, d["codec"], N, n)
+        d["achieved_gbs"] = d["algorithmic_bytes"] / (d["ms_per_launch"] * 1e-3) / 1e9
+    launches_per_step = sum(len(kernel_names(L.lpar_effective_codec(n, c, w.min_quant_bytes), args.schedule, N))
+                            for c in w.codecs)
+
+    # (3) end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 5))
+        h_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(N)]
+        for h, x in zip(h_in, xs):
+            h.copy_(x)
+        h_out = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(N)]
+
+        def e2e_step():
+            for x, h in zip(xs, h_in):
+                x.copy_(h, non_blocking=True)
+            for codec in w.codecs:
+                L.lpar_allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
+                for h, o in zip(h_out, outs):
+                    h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        bytes_e2e = world * N * 2 * n * len(w.codecs) * e2e_steps
+        e2e = {"value": bytes_e2e / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": N * 2 * n, "d2h_bytes_per_step": N * 2 * n * len(w.codecs),
+               "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
+               "api": "lpar_allreduce with pinned host buffers copied in and out on the same stream"}
+        del h_in, h_out
+
+    # (4) the oracle on the host cores, rank 0 at N=1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, xs)
+
+    return {"ms": ms_max, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
+            "e2e": e2e, "cpu": cpu, "w": w}
+
+
+def cpu_baseline(w, xs_dev, tiles=CPU_BASELINE_TILES):
+    from oracle import oracle as O
+    tiles = min(tiles, w.n // TILE)
+    xs = [x[:tiles * TILE].view(torch.int16).cpu().numpy().view("uint16") for x in xs_dev]
+    t0 = time.perf_counter()
+    for codec in w.codecs:
+        O.allreduce(xs, codec, w.min_quant_bytes)
+    dt = time.perf_counter() - t0
+    value = w.N * 2 * tiles * TILE * len(w.codecs) / dt / 1e9
+    return {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d tiles (%d MiB BF16) of each of the %d ranks, codecs %s, %.1f s single-threaded"
+                      % (tiles, tiles * TILE * 2 >> 20, w.N, "+".join(w.codecs), dt)}
+
+
+# ---- reference arm: the oracle as it stands, on the host --------------------------
+def run_reference(args):
+    from oracle import oracle as O
+    w = W.WORKLOADS[args.workload]
+    tiles = min(REF_TILES_PER_STEP, w.n // TILE)
+    xs = [x.view(torch.int16).numpy().view("uint16") for x in W.make_inputs(w, "cpu", n=tiles * TILE)]
+
+    def step():
+        for codec in w.codecs:
+            O.allreduce(xs, codec, w.min_quant_bytes)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = w.N * 2 * tiles * TILE * len(w.codecs) * args.steps / dt / 1e9
+    sample = "%d tiles (%d KiB BF16) per rank per step of workload %s, codecs %s" % (
+        tiles, tiles * TILE * 2 >> 10, w.name, "+".join(w.codecs))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(w, args),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n,
+            "message_bytes_per_rank": 2 * w.n, "codecs": list(w.codecs), "schedule": args.schedule,
+            "distribution": w.note, "min_quant_bytes": w.min_quant_bytes,
+            "l2": "inputs %d MiB > 126 MB L2: no flush between steps" % (w.N * 2 * w.n >> 20)
+            if w.N * 2 * w.n > 126e6 else "inputs fit in L2",
+            "parallelism": "one independent instance per GPU"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_int3_int4", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--schedule", default="fused", choices=["fused", "three_stage"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res = run_ours(args, rank, world, device)
+    w = res["w"]
+    if rank == 0:
+        peak, peak_src = measured_peaks()
+        step_bytes = w.N * 2 * w.n * len(w.codecs)
+        ms_per_step = res["ms"] / args.steps
+        value = world * step_bytes * args.steps / (res["ms"] * 1e-3) / 1e9
+        kern = res["kern"]
+        dom = max(kern, key=lambda k: kern[k]["ms_total"])
+        total_ms = sum(d["ms_total"] for d in kern.values())
+        alg_step = sum(d["algorithmic_bytes"] * d["launches"] for d in kern.values()) / (
+            max(d["launches"] for d in kern.values()))
+        d = kern[dom]
+        traffic = traffic_for(dom, w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(w, args),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": d["achieved_gbs"], "peak": peak,
+                         "unit": "GB/s", "frac": d["achieved_gbs"] / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": d["algorithmic_bytes"],
+                         "ms_per_launch": d["ms_per_launch"], "share_of_step": d["ms_total"] / total_ms,
+                         "peak_source": peak_src},
+            "step_hbm_fraction": alg_step / (ms_per_step * 1e-3) / 1e9 / peak,
+            "kernels": {k: {"ms_per_launch": v["ms_per_launch"], "achieved_gbs": v["achieved_gbs"],
+                            "frac": v["achieved_gbs"] / peak, "share": v["ms_total"] / total_ms,
+                            "algorithmic_bytes": v["algorithmic_bytes"]} for k, v in kern.items()},
+            "gpu_launches": res["launches_per_step"] * args.steps,
+            "clocks": res["clocks"],
+            "e2e": res["e2e"],
+            "cpu_baseline": res["cpu"],
+            "source_sha": source_sha(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

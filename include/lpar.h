@@ -1,0 +1,157 @@
+/*
+ * lpar.h -- C ABI of the B200 (sm_100a) compressed all-reduce library.
+ *
+ * The library implements the two-shot low-precision all-reduce that these
+ * pages describe, with N "ranks" whose buffers all sit in one GPU's HBM:
+ *
+ *   stage 1  quantise   every rank's BF16 message into a wire of tiles
+ *   stage 2  reduce     per tile: dequantise the N wires, sum in FP32 in
+ *                       ascending rank order, requantise with the same codec
+ *                       (reduce-scatter receiver + all-gather producer)
+ *   stage 3  decode     the gathered wire back to BF16, once per rank
+ *
+ * Sources, by page title and section:
+ *  - "QuickReduce INT3 Quantization and Benchmarking on MI355": Summary (a
+ *    transmitted tile is 1152 B with INT4 and 896 B with INT3), Method
+ *    (block-level FP16 scale, symmetric codes, INT3 split into a low-2-bit
+ *    plane "q2w" and a high-1-bit plane "q1w"), In practice (1 MB activation
+ *    threshold for INT3).
+ *  - "RCCLX: Innovating GPU communications on AMD platforms": Low-Precision
+ *    Collectives (FP8 on the wire, computation in FP32), Direct Data Access
+ *    (tree all-reduce = reduce-scatter followed by all-gather).
+ *  - "FP8 Formats for Deep Learning", abstract (E4M3: no infinities, one NaN
+ *    pattern, so 448 is the largest finite value).
+ *
+ * Formats (readings where the pages are silent are marked "reading"):
+ *  - A tile is 2048 consecutive elements made of 64 blocks of 32 (reading,
+ *    the only split consistent with the printed tile sizes and FP16 scales).
+ *  - INT4 tile (1152 B): 1024 B of 4-bit codes (element i in byte i/2, low
+ *    nibble for even i), then 64 little-endian binary16 scales.
+ *  - INT3 tile (896 B): q2w plane (512 B, element i's code & 3 at bits
+ *    2*(i%4) of byte i/4), q1w plane (256 B, element i's code >> 2 at bit i%8
+ *    of byte i/8), then 64 little-endian binary16 scales.
+ *  - INT codes: s = f16_rne(fl32(absmax / qmax)) saturating at 65504,
+ *    q = clamp(RNE(x / s), -qmax, qmax) of the exact quotient, stored as
+ *    offset binary q + 2^(b-1); qmax = 7 (INT4) or 3 (INT3); s = 0 gives q = 0.
+ *  - FP8 tile (2304 B): 2048 E4M3 codes, then 64 little-endian binary32 scales
+ *    s = fl32(absmax / 448); a block with s < 2^-126 is stored as s = 0 and
+ *    codes 0; otherwise code = e4m3_rne_satfinite(fl32(x * fl32(1 / s))).
+ *  - BF16 "tile" (4096 B): the BF16 values themselves (no compression).
+ *  - Dequantised value: (float)q * s for INT (exact), fl32(e4m3(code) * s) for
+ *    FP8.  Final output: bf16_rne of the dequantised gathered value.
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers on the current CUDA device; the
+ *    pointer ARRAYS (inputs, out, wires) are HOST arrays of N device pointers.
+ *  - n is the number of BF16 elements per rank and must be a multiple of
+ *    LPAR_TILE_ELEMS; n == 0 is a valid no-op.  N must be in [1, LPAR_MAX_RANKS].
+ *  - Every data pointer must be 16-byte aligned.
+ *  - The caller owns all memory.  The library allocates nothing, frees
+ *    nothing, never synchronises and keeps no pointer after a call returns.
+ *    Work is enqueued on `stream` asynchronously; buffers must stay valid
+ *    until the stream has passed the call.
+ *  - Argument errors are detected before anything is launched and return a
+ *    status other than LPAR_OK.  A failed launch returns LPAR_ERR_CUDA.
+ *    Faults during execution surface at the caller's next synchronisation.
+ *    No call aborts, exits or throws.
+ */
+#ifndef LPAR_H
+#define LPAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LPAR_TILE_ELEMS 2048
+#define LPAR_BLOCK_ELEMS 32
+#define LPAR_MAX_RANKS 8
+
+typedef enum {
+    LPAR_CODEC_BF16 = 0,      /* uncompressed passthrough, 4096 B per tile */
+    LPAR_CODEC_FP8_E4M3 = 1,  /* E4M3 codes + binary32 scale per 32 elements, 2304 B per tile */
+    LPAR_CODEC_INT4 = 2,      /* 4-bit codes + binary16 scale per 32 elements, 1152 B per tile */
+    LPAR_CODEC_INT3 = 3       /* q2w + q1w planes + binary16 scale per 32, 896 B per tile */
+} lpar_codec_t;
+
+typedef enum {
+    LPAR_OK = 0,
+    LPAR_ERR_INVALID_ARG = 1,          /* null pointer, N or n out of range, bad tile range */
+    LPAR_ERR_MISALIGNED = 2,           /* a data pointer is not 16-byte aligned */
+    LPAR_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes < lpar_workspace_bytes(...) */
+    LPAR_ERR_UNSUPPORTED = 4,          /* unknown codec or schedule */
+    LPAR_ERR_CUDA = 5                  /* a CUDA launch or device query failed */
+} lpar_status_t;
+
+typedef enum {
+    LPAR_SCHEDULE_FUSED = 0,       /* quantise; reduce + requantise + decode in one kernel */
+    LPAR_SCHEDULE_THREE_STAGE = 1  /* quantise; reduce + requantise; decode (three kernels) */
+} lpar_schedule_t;
+
+typedef struct {
+    /* A quantising codec runs only when the per-rank message (2*n bytes) is at
+     * least this many bytes; smaller messages take the BF16 passthrough.
+     * 0 = always quantise.  The INT3 page recommends 1 MB (1 << 20). */
+    size_t min_quant_bytes;
+    lpar_schedule_t schedule;      /* 0 (LPAR_SCHEDULE_FUSED) is the default */
+    /* Optional tracing: events recorded on `stream` at the stage boundaries --
+     * [0] before stage 1, [1] after stage 1, [2] after stage 2 (after the
+     * fused reduce+decode in the fused schedule), [3] after stage 3 (three-
+     * stage schedule only).  NULL entries are skipped.  The BF16 passthrough
+     * has no stage 1: [0] and [1] are recorded back to back. */
+    cudaEvent_t stage_events[4];
+} lpar_options_t;
+
+/* Bytes of one 2048-element tile: 4096 (BF16), 2304 (FP8), 1152 (INT4), 896
+ * (INT3); 0 for an unknown codec. */
+size_t lpar_tile_bytes(lpar_codec_t codec);
+
+/* Bytes of the wire of an n-element message: (n / 2048) * lpar_tile_bytes(codec). */
+size_t lpar_wire_bytes(lpar_codec_t codec, size_t n);
+
+/* Workspace lpar_allreduce needs when it runs `codec`: N stage-1 wires plus one
+ * gathered wire for a quantising codec, one gathered wire (2n bytes) for BF16;
+ * 0 for N outside [1, LPAR_MAX_RANKS] or an unknown codec.  With a threshold
+ * set, size it for lpar_effective_codec(n, codec, opts). */
+size_t lpar_workspace_bytes(int N, size_t n, lpar_codec_t codec);
+
+/* Stage 1 for one rank: in_bf16 (n BF16 values) -> wire
+ * (lpar_wire_bytes(codec, n) bytes).  For BF16 the wire is a copy. */
+lpar_status_t lpar_quantize(const void *in_bf16, size_t n, lpar_codec_t codec,
+                            void *wire, cudaStream_t stream);
+
+/* Stage 2 for the tiles [tile_begin, tile_begin + tile_count) of N full
+ * wires: wires[r] is the base of rank r's wire; tile t of every wire is
+ * dequantised, summed in FP32 in ascending rank order starting from +0.0f,
+ * requantised, and written as tile t of wire_out (the base of the gathered
+ * wire).  wire_out must not overlap any wires[r]. */
+lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_begin, size_t tile_count,
+                          lpar_codec_t codec, void *wire_out, cudaStream_t stream);
+
+/* Stage 3: wire (n elements' worth) -> out_bf16 (n BF16 values, RNE). */
+lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec,
+                          void *out_bf16, cudaStream_t stream);
+
+/* The whole all-reduce of N ranks' BF16 messages of n elements: inputs[r] ->
+ * every out[r] receives the same BF16 result.  out[r] may equal inputs[r]
+ * (in place); out buffers must not overlap each other or the workspace.
+ * workspace: device memory of at least lpar_workspace_bytes(N, n, effective
+ * codec) bytes, 16-byte aligned, contents ignored and overwritten.
+ * opts may be NULL (always quantise, fused schedule). */
+lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                             void *const *out, void *workspace, size_t workspace_bytes,
+                             const lpar_options_t *opts, cudaStream_t stream);
+
+/* The codec lpar_allreduce runs for these arguments after the threshold. */
+lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts);
+
+/* A static, human-readable name of a status code. */
+const char *lpar_status_string(lpar_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LPAR_H */

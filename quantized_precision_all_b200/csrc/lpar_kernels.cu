@@ -1,0 +1,528 @@
+// lpar_kernels.cu -- sm_100a kernels of the compressed all-reduce and the C ABI.
+//
+// Stages (two-shot all-reduce, "RCCLX: Innovating GPU communications on AMD
+// platforms", Direct Data Access: reduce-scatter then all-gather; FP32
+// compute per its Low-Precision Collectives section; tile formats per
+// "QuickReduce INT3 Quantization and Benchmarking on MI355", Summary/Method):
+//   K1  k_quantize      BF16 -> wire, all N ranks in one launch (grid.y = rank)
+//   K2  k_reduce<.., false>  N wires -> FP32 sum in rank order -> requantised
+//                        gathered wire
+//   K23 k_reduce<.., true>   K2 plus the decode of the gathered block straight
+//                        from registers into every rank's BF16 output
+//   K3  k_decode        gathered wire -> BF16 into every rank's output
+// The BF16 passthrough uses k_bf16_reduce (FP32 sum, one BF16 rounding) and
+// k_broadcast (plain copies).
+//
+// Work decomposition: a CTA of 256 threads owns 4 consecutive tiles; thread t
+// owns block (t mod 64) of tile (t / 64), i.e. 32 consecutive elements.  Codes
+// and scales of one warp's 32 blocks are contiguous in a tile, so packed
+// loads/stores are coalesced as they are.  The BF16 side (64 B per thread) is
+// staged through shared memory with an XOR swizzle so both the coalesced
+// global access and the per-thread 64-B access are bank-conflict free.
+#include "lpar.h"
+#include "lpar_codec.cuh"
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lpar {
+
+constexpr int kThreads = 256;
+constexpr int kTilesPerCta = kThreads / kBlocksPerTile;     // 4
+constexpr int kStageBytes = kThreads * 64;                  // 16 KiB of BF16 per CTA
+constexpr int kMaxRanks = LPAR_MAX_RANKS;
+
+struct InPtrs { const uint8_t *p[kMaxRanks]; };
+struct OutPtrs { uint8_t *p[kMaxRanks]; };
+
+// Byte offset of 16-B piece j (0..3) of thread t's 64-B block in the stage.
+__device__ __forceinline__ int swz(int t, int j) { return 64 * t + 16 * (j ^ ((t >> 1) & 3)); }
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Packed block <-> tile bytes.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_block(const uint8_t *tile, int b, Packed<kINT4> &p) {
+    const uint4 c = *reinterpret_cast<const uint4 *>(tile + 16 * b);
+    p.w[0] = c.x; p.w[1] = c.y; p.w[2] = c.z; p.w[3] = c.w;
+    p.scale = *reinterpret_cast<const uint16_t *>(tile + Layout<kINT4>::kScaleOff + 2 * b);
+}
+__device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<kINT4> &p) {
+    *reinterpret_cast<uint4 *>(tile + 16 * b) = make_uint4(p.w[0], p.w[1], p.w[2], p.w[3]);
+    *reinterpret_cast<uint16_t *>(tile + Layout<kINT4>::kScaleOff + 2 * b) = p.scale;
+}
+__device__ __forceinline__ void load_block(const uint8_t *tile, int b, Packed<kINT3> &p) {
+    const uint2 c = *reinterpret_cast<const uint2 *>(tile + 8 * b);
+    p.q2w[0] = c.x; p.q2w[1] = c.y;
+    p.q1w = *reinterpret_cast<const uint32_t *>(tile + Layout<kINT3>::kQ1wOff + 4 * b);
+    p.scale = *reinterpret_cast<const uint16_t *>(tile + Layout<kINT3>::kScaleOff + 2 * b);
+}
+__device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<kINT3> &p) {
+    *reinterpret_cast<uint2 *>(tile + 8 * b) = make_uint2(p.q2w[0], p.q2w[1]);
+    *reinterpret_cast<uint32_t *>(tile + Layout<kINT3>::kQ1wOff + 4 * b) = p.q1w;
+    *reinterpret_cast<uint16_t *>(tile + Layout<kINT3>::kScaleOff + 2 * b) = p.scale;
+}
+// FP8 codes: two 16-B accesses (the ABI guarantees 16-B alignment only).
+__device__ __forceinline__ void load_block(const uint8_t *tile, int b, Packed<kFP8> &p) {
+    const uint4 c0 = *reinterpret_cast<const uint4 *>(tile + 32 * b);
+    const uint4 c1 = *reinterpret_cast<const uint4 *>(tile + 32 * b + 16);
+    p.w[0] = c0.x; p.w[1] = c0.y; p.w[2] = c0.z; p.w[3] = c0.w;
+    p.w[4] = c1.x; p.w[5] = c1.y; p.w[6] = c1.z; p.w[7] = c1.w;
+    p.scale = *reinterpret_cast<const float *>(tile + Layout<kFP8>::kScaleOff + 4 * b);
+}
+__device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<kFP8> &p) {
+    *reinterpret_cast<uint4 *>(tile + 32 * b) = make_uint4(p.w[0], p.w[1], p.w[2], p.w[3]);
+    *reinterpret_cast<uint4 *>(tile + 32 * b + 16) = make_uint4(p.w[4], p.w[5], p.w[6], p.w[7]);
+    *reinterpret_cast<float *>(tile + Layout<kFP8>::kScaleOff + 4 * b) = p.scale;
+}
+
+template <int C, bool WANT_V>
+__device__ __forceinline__ void encode(const float (&x)[32], float a, Packed<C> &p, uint32_t (&o)[16]) {
+    if constexpr (C == kINT4) encode_int4<WANT_V>(x, a, p, o);
+    else if constexpr (C == kINT3) encode_int3<WANT_V>(x, a, p, o);
+    else encode_fp8<WANT_V>(x, a, p, o);
+}
+
+// Pointer r of a parameter array, selected without dynamic indexing (which
+// would copy the whole array to local memory).
+template <class P>
+__device__ __forceinline__ auto pick(const P &a, int r) -> decltype(a.p[0]) {
+    auto q = a.p[0];
+#pragma unroll
+    for (int i = 1; i < kMaxRanks; ++i) q = (r == i) ? a.p[i] : q;
+    return q;
+}
+
+template <int C>
+__device__ __forceinline__ void accumulate(const Packed<C> &p, float (&acc)[32]) {
+    if constexpr (C == kINT4) accumulate_int4(p, acc);
+    else if constexpr (C == kINT3) accumulate_int3(p, acc);
+    else accumulate_fp8(p, acc);
+}
+
+template <int C>
+__device__ __forceinline__ void decode(const Packed<C> &p, uint32_t (&o)[16]) {
+    if constexpr (C == kINT4) decode_int4(p, o);
+    else if constexpr (C == kINT3) decode_int3(p, o);
+    else decode_fp8(p, o);
+}
+
+// Thread t's 64-B BF16 block <-> the swizzled stage.
+__device__ __forceinline__ void stage_read(const uint8_t *stage, int t, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(stage + swz(t, j));
+        w[4 * j] = q.x; w[4 * j + 1] = q.y; w[4 * j + 2] = q.z; w[4 * j + 3] = q.w;
+    }
+}
+__device__ __forceinline__ void stage_write(uint8_t *stage, int t, const uint32_t (&w)[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4 *>(stage + swz(t, j)) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
+// Coalesced copy of the staged BF16 chunk (ntiles tiles) to N outputs.
+__device__ __forceinline__ void stage_to_outputs(const uint8_t *stage, const OutPtrs &out, int N,
+                                                 size_t byte0, int ntiles) {
+    const int t = threadIdx.x;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int g = t + kThreads * k;                 // 16-B piece index in the chunk
+        if (g < ntiles * 256) {
+            const uint4 d = *reinterpret_cast<const uint4 *>(stage + swz(g >> 2, g & 3));
+#pragma unroll
+            for (int r = 0; r < kMaxRanks; ++r)
+                if (r < N) *reinterpret_cast<uint4 *>(out.p[r] + byte0 + 16 * (size_t)g) = d;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K1: stage 1 for every rank.  grid = (ceil(tiles / 4), N).
+// ---------------------------------------------------------------------------
+template <int C>
+__global__ void __launch_bounds__(kThreads) k_quantize(InPtrs in, OutPtrs wire, size_t tiles) {
+    __shared__ __align__(128) uint8_t stage[kStageBytes];
+    const int r = blockIdx.y;
+    const int t = threadIdx.x;
+    const size_t tile0 = (size_t)blockIdx.x * kTilesPerCta;
+    const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+    const uint8_t *src = pick(in, r) + tile0 * (kTileElems * 2);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int g = t + kThreads * k;
+        if (g < ntiles * 256) cp_async16(stage + swz(g >> 2, g & 3), src + 16 * (size_t)g);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    if (t >= ntiles * kBlocksPerTile) return;
+
+    uint32_t w[16];
+    stage_read(stage, t, w);
+    float x[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(w[k]); x[2 * k + 1] = bf16hi(w[k]); }
+    const float a = absmax_bf16x32(w);
+    Packed<C> p;
+    uint32_t unused[16];
+    encode<C, false>(x, a, p, unused);
+    store_block(pick(wire, r) + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
+}
+
+// ---------------------------------------------------------------------------
+// K2 / K23: tiles [tile_begin, tile_end) of N wires -> gathered wire (and,
+// when FUSED, the decoded BF16 result into every out[r]).
+// ---------------------------------------------------------------------------
+template <int C, int N, bool FUSED>
+__global__ void __launch_bounds__(kThreads) k_reduce(InPtrs wires, uint8_t *gather, OutPtrs out,
+                                                     size_t tile_begin, size_t tile_end) {
+    __shared__ __align__(128) uint8_t stage[FUSED ? kStageBytes : 16];
+    const int t = threadIdx.x;
+    const size_t tile0 = tile_begin + (size_t)blockIdx.x * kTilesPerCta;
+    const int ntiles = (int)min((size_t)kTilesPerCta, tile_end - tile0);
+    if (t < ntiles * kBlocksPerTile) {
+        const size_t tile = tile0 + t / kBlocksPerTile;
+        const int b = t % kBlocksPerTile;
+        Packed<C> p[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) load_block(wires.p[r] + tile * Layout<C>::kTileBytes, b, p[r]);
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.0f;     // +0.0f, then ranks in ascending order
+#pragma unroll
+        for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
+        const float a = absmax_f32x32(acc);
+        Packed<C> g;
+        uint32_t o[16];
+        encode<C, FUSED>(acc, a, g, o);
+        store_block(gather + tile * Layout<C>::kTileBytes, b, g);
+        if (FUSED) stage_write(stage, t, o);
+    }
+    if (FUSED) {
+        __syncthreads();
+        stage_to_outputs(stage, out, N, tile0 * (kTileElems * 2), ntiles);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K3: gathered wire -> BF16 in every out[r].  grid = ceil(tiles / 4).
+// ---------------------------------------------------------------------------
+template <int C>
+__global__ void __launch_bounds__(kThreads) k_decode(const uint8_t *wire, OutPtrs out, int N, size_t tiles) {
+    __shared__ __align__(128) uint8_t stage[kStageBytes];
+    const int t = threadIdx.x;
+    const size_t tile0 = (size_t)blockIdx.x * kTilesPerCta;
+    const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+    if (t < ntiles * kBlocksPerTile) {
+        Packed<C> p;
+        load_block(wire + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
+        uint32_t o[16];
+        decode<C>(p, o);
+        stage_write(stage, t, o);
+    }
+    __syncthreads();
+    stage_to_outputs(stage, out, N, tile0 * (kTileElems * 2), ntiles);
+}
+
+// ---------------------------------------------------------------------------
+// BF16 passthrough: 8 elements (16 B) per thread, all accesses coalesced.
+// ---------------------------------------------------------------------------
+template <int N, bool FUSED>
+__global__ void __launch_bounds__(kThreads) k_bf16_reduce(InPtrs in, uint8_t *gather, OutPtrs out,
+                                                          size_t v_begin, size_t v_end) {
+    const size_t i = v_begin + (size_t)blockIdx.x * kThreads + threadIdx.x;   // 16-B vector index
+    if (i >= v_end) return;
+    uint4 x[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) x[r] = *reinterpret_cast<const uint4 *>(in.p[r] + 16 * i);
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+        const uint32_t w[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc[2 * k] = __fadd_rn(acc[2 * k], bf16lo(w[k]));
+            acc[2 * k + 1] = __fadd_rn(acc[2 * k + 1], bf16hi(w[k]));
+        }
+    }
+    const uint4 o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    *reinterpret_cast<uint4 *>(gather + 16 * i) = o;
+    if (FUSED) {
+#pragma unroll
+        for (int r = 0; r < N; ++r) *reinterpret_cast<uint4 *>(out.p[r] + 16 * i) = o;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) k_broadcast(const uint8_t *src, OutPtrs dst, int N, size_t nvec) {
+    const size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= nvec) return;
+    const uint4 d = *reinterpret_cast<const uint4 *>(src + 16 * i);
+#pragma unroll
+    for (int r = 0; r < kMaxRanks; ++r)
+        if (r < N) *reinterpret_cast<uint4 *>(dst.p[r] + 16 * i) = d;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (no validation here; the C ABI validates first).
+// ---------------------------------------------------------------------------
+static inline unsigned grid_for_tiles(size_t tiles) { return (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta); }
+
+static void launch_quantize(int codec, const InPtrs &in, const OutPtrs &wire, int N, size_t tiles, cudaStream_t st) {
+    const dim3 grid(grid_for_tiles(tiles), N);
+    switch (codec) {
+    case kINT4: k_quantize<kINT4><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
+    case kINT3: k_quantize<kINT3><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
+    case kFP8: k_quantize<kFP8><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
+    default: break;
+    }
+}
+
+template <int C, bool FUSED>
+static void launch_reduce_c(const InPtrs &w, int N, uint8_t *g, const OutPtrs &o, size_t t0, size_t t1, cudaStream_t st) {
+    const unsigned grid = grid_for_tiles(t1 - t0);
+    switch (N) {
+    case 1: k_reduce<C, 1, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 2: k_reduce<C, 2, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 3: k_reduce<C, 3, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 4: k_reduce<C, 4, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 5: k_reduce<C, 5, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 6: k_reduce<C, 6, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 7: k_reduce<C, 7, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    case 8: k_reduce<C, 8, FUSED><<<grid, kThreads, 0, st>>>(w, g, o, t0, t1); break;
+    default: break;
+    }
+}
+
+template <bool FUSED>
+static void launch_reduce(int codec, const InPtrs &w, int N, uint8_t *g, const OutPtrs &o, size_t t0, size_t t1,
+                          cudaStream_t st) {
+    switch (codec) {
+    case kINT4: launch_reduce_c<kINT4, FUSED>(w, N, g, o, t0, t1, st); break;
+    case kINT3: launch_reduce_c<kINT3, FUSED>(w, N, g, o, t0, t1, st); break;
+    case kFP8: launch_reduce_c<kFP8, FUSED>(w, N, g, o, t0, t1, st); break;
+    default: break;
+    }
+}
+
+template <bool FUSED>
+static void launch_bf16_reduce(const InPtrs &in, int N, uint8_t *g, const OutPtrs &o, size_t v0, size_t v1,
+                               cudaStream_t st) {
+    const unsigned grid = (unsigned)((v1 - v0 + kThreads - 1) / kThreads);
+    switch (N) {
+    case 1: k_bf16_reduce<1, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 2: k_bf16_reduce<2, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 3: k_bf16_reduce<3, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 4: k_bf16_reduce<4, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 5: k_bf16_reduce<5, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 6: k_bf16_reduce<6, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 7: k_bf16_reduce<7, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    case 8: k_bf16_reduce<8, FUSED><<<grid, kThreads, 0, st>>>(in, g, o, v0, v1); break;
+    default: break;
+    }
+}
+
+static void launch_decode(int codec, const uint8_t *wire, const OutPtrs &o, int N, size_t tiles, cudaStream_t st) {
+    const unsigned grid = grid_for_tiles(tiles);
+    switch (codec) {
+    case kINT4: k_decode<kINT4><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
+    case kINT3: k_decode<kINT3><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
+    case kFP8: k_decode<kFP8><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
+    default: break;
+    }
+}
+
+static void launch_broadcast(const uint8_t *src, const OutPtrs &o, int N, size_t bytes, cudaStream_t st) {
+    const size_t nvec = bytes / 16;
+    const unsigned grid = (unsigned)((nvec + kThreads - 1) / kThreads);
+    k_broadcast<<<grid, kThreads, 0, st>>>(src, o, N, nvec);
+}
+
+// ---------------------------------------------------------------------------
+// Validation helpers.
+// ---------------------------------------------------------------------------
+static inline bool codec_ok(int c) { return c >= LPAR_CODEC_BF16 && c <= LPAR_CODEC_INT3; }
+static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static inline lpar_status_t launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LPAR_OK : LPAR_ERR_CUDA;
+}
+
+}  // namespace lpar
+
+using namespace lpar;
+
+#define LPAR_API extern "C" __attribute__((visibility("default")))
+
+LPAR_API size_t lpar_tile_bytes(lpar_codec_t codec) {
+    switch (codec) {
+    case LPAR_CODEC_BF16: return Layout<kBF16>::kTileBytes;
+    case LPAR_CODEC_FP8_E4M3: return Layout<kFP8>::kTileBytes;
+    case LPAR_CODEC_INT4: return Layout<kINT4>::kTileBytes;
+    case LPAR_CODEC_INT3: return Layout<kINT3>::kTileBytes;
+    default: return 0;
+    }
+}
+
+LPAR_API size_t lpar_wire_bytes(lpar_codec_t codec, size_t n) { return (n / kTileElems) * lpar_tile_bytes(codec); }
+
+LPAR_API size_t lpar_workspace_bytes(int N, size_t n, lpar_codec_t codec) {
+    if (N < 1 || N > kMaxRanks || !codec_ok(codec)) return 0;
+    if (codec == LPAR_CODEC_BF16) return lpar_wire_bytes(LPAR_CODEC_BF16, n);
+    return (size_t)(N + 1) * lpar_wire_bytes(codec, n);
+}
+
+LPAR_API lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts) {
+    const size_t thr = opts ? opts->min_quant_bytes : 0;
+    if (codec != LPAR_CODEC_BF16 && 2 * n < thr) return LPAR_CODEC_BF16;
+    return codec;
+}
+
+LPAR_API const char *lpar_status_string(lpar_status_t s) {
+    switch (s) {
+    case LPAR_OK: return "ok";
+    case LPAR_ERR_INVALID_ARG: return "invalid argument";
+    case LPAR_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case LPAR_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case LPAR_ERR_UNSUPPORTED: return "unsupported codec or schedule";
+    case LPAR_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+    }
+}
+
+LPAR_API lpar_status_t lpar_quantize(const void *in_bf16, size_t n, lpar_codec_t codec, void *wire,
+                                     cudaStream_t stream) {
+    if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
+    if (n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (n == 0) return LPAR_OK;
+    if (!in_bf16 || !wire) return LPAR_ERR_INVALID_ARG;
+    if (!aligned16(in_bf16) || !aligned16(wire)) return LPAR_ERR_MISALIGNED;
+    const size_t tiles = n / kTileElems;
+    OutPtrs w{};
+    w.p[0] = static_cast<uint8_t *>(wire);
+    if (codec == LPAR_CODEC_BF16) {
+        launch_broadcast(static_cast<const uint8_t *>(in_bf16), w, 1, 2 * n, stream);
+    } else {
+        InPtrs in{};
+        in.p[0] = static_cast<const uint8_t *>(in_bf16);
+        launch_quantize(codec, in, w, 1, tiles, stream);
+    }
+    return launch_status();
+}
+
+LPAR_API lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_begin, size_t tile_count,
+                                   lpar_codec_t codec, void *wire_out, cudaStream_t stream) {
+    if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
+    if (N < 1 || N > kMaxRanks || !wires) return LPAR_ERR_INVALID_ARG;
+    if (tile_begin + tile_count < tile_begin) return LPAR_ERR_INVALID_ARG;
+    if (tile_count == 0) return LPAR_OK;
+    if (!wire_out) return LPAR_ERR_INVALID_ARG;
+    InPtrs w{};
+    for (int r = 0; r < N; ++r) {
+        if (!wires[r]) return LPAR_ERR_INVALID_ARG;
+        if (!aligned16(wires[r])) return LPAR_ERR_MISALIGNED;
+        w.p[r] = static_cast<const uint8_t *>(wires[r]);
+    }
+    if (!aligned16(wire_out)) return LPAR_ERR_MISALIGNED;
+    OutPtrs none{};
+    uint8_t *g = static_cast<uint8_t *>(wire_out);
+    if (codec == LPAR_CODEC_BF16) {
+        const size_t v_per_tile = (size_t)kTileElems * 2 / 16;
+        launch_bf16_reduce<false>(w, N, g, none, tile_begin * v_per_tile, (tile_begin + tile_count) * v_per_tile,
+                                  stream);
+    } else {
+        launch_reduce<false>(codec, w, N, g, none, tile_begin, tile_begin + tile_count, stream);
+    }
+    return launch_status();
+}
+
+LPAR_API lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec, void *out_bf16,
+                                   cudaStream_t stream) {
+    if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
+    if (n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (n == 0) return LPAR_OK;
+    if (!wire || !out_bf16) return LPAR_ERR_INVALID_ARG;
+    if (!aligned16(wire) || !aligned16(out_bf16)) return LPAR_ERR_MISALIGNED;
+    OutPtrs o{};
+    o.p[0] = static_cast<uint8_t *>(out_bf16);
+    if (codec == LPAR_CODEC_BF16) launch_broadcast(static_cast<const uint8_t *>(wire), o, 1, 2 * n, stream);
+    else launch_decode(codec, static_cast<const uint8_t *>(wire), o, 1, n / kTileElems, stream);
+    return launch_status();
+}
+
+LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                                      void *const *out, void *workspace, size_t workspace_bytes,
+                                      const lpar_options_t *opts, cudaStream_t stream) {
+    if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
+    const int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_FUSED;
+    if (schedule != LPAR_SCHEDULE_FUSED && schedule != LPAR_SCHEDULE_THREE_STAGE) return LPAR_ERR_UNSUPPORTED;
+    if (N < 1 || N > kMaxRanks || n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (n == 0) return LPAR_OK;
+    if (!inputs || !out || !workspace) return LPAR_ERR_INVALID_ARG;
+    InPtrs in{};
+    OutPtrs o{};
+    for (int r = 0; r < N; ++r) {
+        if (!inputs[r] || !out[r]) return LPAR_ERR_INVALID_ARG;
+        if (!aligned16(inputs[r]) || !aligned16(out[r])) return LPAR_ERR_MISALIGNED;
+        in.p[r] = static_cast<const uint8_t *>(inputs[r]);
+        o.p[r] = static_cast<uint8_t *>(out[r]);
+    }
+    if (!aligned16(workspace)) return LPAR_ERR_MISALIGNED;
+    const lpar_codec_t eff = lpar_effective_codec(n, codec, opts);
+    if (workspace_bytes < lpar_workspace_bytes(N, n, eff)) return LPAR_ERR_WORKSPACE_TOO_SMALL;
+    const size_t tiles = n / kTileElems;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const bool fused = schedule == LPAR_SCHEDULE_FUSED;
+    auto mark = [&](int i) {
+        if (opts && opts->stage_events[i]) cudaEventRecord(opts->stage_events[i], stream);
+    };
+
+    if (eff == LPAR_CODEC_BF16) {
+        // the wire of every rank is its input; the gathered wire is the workspace
+        const size_t nvec = 2 * n / 16;
+        mark(0);
+        mark(1);
+        if (fused) {
+            launch_bf16_reduce<true>(in, N, ws, o, 0, nvec, stream);
+            mark(2);
+        } else {
+            launch_bf16_reduce<false>(in, N, ws, o, 0, nvec, stream);
+            if (cudaGetLastError() != cudaSuccess) return LPAR_ERR_CUDA;
+            mark(2);
+            launch_broadcast(ws, o, N, 2 * n, stream);
+            mark(3);
+        }
+        return launch_status();
+    }
+
+    const size_t wb = lpar_wire_bytes(eff, n);
+    OutPtrs wires{};
+    InPtrs wires_in{};
+    for (int r = 0; r < N; ++r) {
+        wires.p[r] = ws + (size_t)r * wb;
+        wires_in.p[r] = ws + (size_t)r * wb;
+    }
+    uint8_t *gather = ws + (size_t)N * wb;
+    mark(0);
+    launch_quantize(eff, in, wires, N, tiles, stream);
+    if (cudaGetLastError() != cudaSuccess) return LPAR_ERR_CUDA;
+    mark(1);
+    if (fused) {
+        launch_reduce<true>(eff, wires_in, N, gather, o, 0, tiles, stream);
+        mark(2);
+    } else {
+        launch_reduce<false>(eff, wires_in, N, gather, o, 0, tiles, stream);
+        if (cudaGetLastError() != cudaSuccess) return LPAR_ERR_CUDA;
+        mark(2);
+        launch_decode(eff, gather, o, N, tiles, stream);
+        mark(3);
+    }
+    return launch_status();
+}

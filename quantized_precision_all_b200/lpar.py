@@ -1,0 +1,179 @@
+"""Python binding of the C ABI in ``include/lpar.h`` (argument marshalling only).
+
+Every function has the C name and forwards to ``liblpar.so``; all arithmetic
+runs in the library's CUDA kernels.  Device buffers may be given as CUDA
+``torch.Tensor`` objects (contiguous) or as raw integer device addresses;
+pointer arrays are Python sequences.  ``stream`` defaults to PyTorch's current
+stream on the current device.
+
+A call that returns a status other than LPAR_OK raises :class:`LparError`.
+If the library has not been built, importing it raises ``OSError`` -- there is
+no fallback implementation.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblpar.so")
+
+LPAR_CODEC_BF16, LPAR_CODEC_FP8_E4M3, LPAR_CODEC_INT4, LPAR_CODEC_INT3 = 0, 1, 2, 3
+CODECS = {"bf16": LPAR_CODEC_BF16, "fp8": LPAR_CODEC_FP8_E4M3, "int4": LPAR_CODEC_INT4, "int3": LPAR_CODEC_INT3}
+CODEC_NAMES = {v: k for k, v in CODECS.items()}
+LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE = 0, 1
+SCHEDULES = {"fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE}
+STATUS = {0: "LPAR_OK", 1: "LPAR_ERR_INVALID_ARG", 2: "LPAR_ERR_MISALIGNED",
+          3: "LPAR_ERR_WORKSPACE_TOO_SMALL", 4: "LPAR_ERR_UNSUPPORTED", 5: "LPAR_ERR_CUDA"}
+TILE_ELEMS = 2048
+MAX_RANKS = 8
+
+EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
+           "lpar_decode", "lpar_allreduce", "lpar_effective_codec", "lpar_status_string")
+
+
+class LparError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_lib.lpar_status_string(status).decode()})")
+
+
+class lpar_options_t(ctypes.Structure):
+    _fields_ = [("min_quant_bytes", ctypes.c_size_t), ("schedule", ctypes.c_int),
+                ("stage_events", ctypes.c_void_p * 4)]
+
+
+def _load():
+    L = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    vpp = ctypes.POINTER(ctypes.c_void_p)
+    sigs = {
+        "lpar_tile_bytes": (sz, [i32]),
+        "lpar_wire_bytes": (sz, [i32, sz]),
+        "lpar_workspace_bytes": (sz, [i32, sz, i32]),
+        "lpar_quantize": (i32, [vp, sz, i32, vp, vp]),
+        "lpar_reduce": (i32, [vpp, i32, sz, sz, i32, vp, vp]),
+        "lpar_decode": (i32, [vp, sz, i32, vp, vp]),
+        "lpar_allreduce": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_effective_codec": (i32, [sz, i32, ctypes.POINTER(lpar_options_t)]),
+        "lpar_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes library (for symbol checks)."""
+    return _lib
+
+
+# ---- marshalling helpers ------------------------------------------------------
+def _codec(c):
+    return CODECS[c] if isinstance(c, str) else int(c)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("lpar: tensors must live on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError("lpar: tensors must be contiguous")
+    return x.data_ptr()
+
+
+def _ptr_array(xs):
+    if xs is None:
+        return None
+    arr = (ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _options(min_quant_bytes=0, schedule="fused", stage_events=None):
+    sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    opts = lpar_options_t(min_quant_bytes, sched)
+    for i, ev in enumerate(stage_events or ()):
+        if ev is not None:
+            opts.stage_events[i] = ev if isinstance(ev, int) else ev.cuda_event
+    return opts
+
+
+def _check(status, where):
+    if status != 0:
+        raise LparError(status, where)
+
+
+# ---- the C ABI ------------------------------------------------------------------
+def lpar_tile_bytes(codec):
+    return _lib.lpar_tile_bytes(_codec(codec))
+
+
+def lpar_wire_bytes(codec, n):
+    return _lib.lpar_wire_bytes(_codec(codec), n)
+
+
+def lpar_workspace_bytes(N, n, codec):
+    return _lib.lpar_workspace_bytes(N, n, _codec(codec))
+
+
+def lpar_effective_codec(n, codec, min_quant_bytes=0):
+    opts = _options(min_quant_bytes)
+    return CODEC_NAMES[_lib.lpar_effective_codec(n, _codec(codec), ctypes.byref(opts))]
+
+
+def lpar_quantize(in_bf16, n, codec, wire, stream=None):
+    _check(_lib.lpar_quantize(_ptr(in_bf16), n, _codec(codec), _ptr(wire), _stream(stream)), "lpar_quantize")
+
+
+def lpar_reduce(wires, tile_begin, tile_count, codec, wire_out, stream=None):
+    arr = _ptr_array(wires)
+    _check(_lib.lpar_reduce(arr[0] if arr else None, len(wires) if wires is not None else 0, tile_begin,
+                            tile_count, _codec(codec), _ptr(wire_out), _stream(stream)), "lpar_reduce")
+
+
+def lpar_decode(wire, n, codec, out_bf16, stream=None):
+    _check(_lib.lpar_decode(_ptr(wire), n, _codec(codec), _ptr(out_bf16), _stream(stream)), "lpar_decode")
+
+
+def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_bytes=0, schedule="fused",
+                   stream=None, N=None, stage_events=None):
+    ins = _ptr_array(inputs)
+    outs = _ptr_array(out)
+    N = len(inputs) if N is None else N
+    opts = _options(min_quant_bytes, schedule, stage_events)
+    _check(_lib.lpar_allreduce(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+                               _ptr(workspace), workspace_bytes, ctypes.byref(opts), _stream(stream)),
+           "lpar_allreduce")
+
+
+def lpar_status_string(status):
+    return _lib.lpar_status_string(status).decode()
+
+
+# ---- convenience: allocate with torch, then call the C ABI -----------------------
+def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedule="fused", stream=None):
+    """All-reduce a list of N equal-size BF16 CUDA tensors; returns the N outputs."""
+    import torch
+    n = inputs[0].numel()
+    if out is None:
+        out = [torch.empty_like(x) for x in inputs]
+    need = lpar_workspace_bytes(len(inputs), n, lpar_effective_codec(n, codec, min_quant_bytes))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=inputs[0].device)
+    lpar_allreduce(inputs, n, codec, out, workspace, workspace.numel(), min_quant_bytes, schedule, stream)
+    return out

@@ -1,0 +1,146 @@
+"""The C-ABI library on the host: it loads without a GPU, exports every symbol
+the header declares, reports the page-fixed sizes, and rejects bad arguments
+before launching anything (no GPU is touched by any call here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lpar.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_precision_all_b200 import build
+    build.build()
+    from quantized_precision_all_b200 import lpar
+    return lpar
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\w[\w\s\*]*?\b(lpar_\w+)\s*\(", text, re.M)))
+
+
+def test_header_is_valid_c():
+    subprocess.run(["gcc", "-std=c11", "-fsyntax-only", "-Wall", "-Werror", "-x", "c",
+                    "-I", "/usr/local/cuda/include", HEADER], check=True)
+
+
+def test_library_exports_every_declared_symbol(L):
+    decl = declared_functions()
+    assert decl, "no declarations parsed"
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (lpar_\w+)", out))
+    assert set(decl) <= exported, set(decl) - exported
+    assert set(L.EXPORTS) == set(decl)
+    for name in decl:
+        assert hasattr(L.library(), name)
+
+
+def test_tile_and_wire_sizes(L):
+    assert L.lpar_tile_bytes("int4") == 1152
+    assert L.lpar_tile_bytes("int3") == 896
+    assert L.lpar_tile_bytes("fp8") == 2304
+    assert L.lpar_tile_bytes("bf16") == 4096
+    assert L.lpar_tile_bytes(7) == 0
+    assert L.lpar_wire_bytes("int3", 2048 * 3) == 3 * 896
+    assert L.lpar_wire_bytes("int4", 2048 * 5 + 100) == 5 * 1152
+    n = 512 * 1024 * 1024
+    assert L.lpar_wire_bytes("int3", n) == 234881024 and L.lpar_wire_bytes("int4", n) == 301989888
+
+
+def test_workspace_bytes(L):
+    n = 2048 * 10
+    assert L.lpar_workspace_bytes(2, n, "int4") == 3 * 10 * 1152
+    assert L.lpar_workspace_bytes(8, n, "fp8") == 9 * 10 * 2304
+    assert L.lpar_workspace_bytes(2, n, "int3") == 3 * 10 * 896
+    assert L.lpar_workspace_bytes(4, n, "bf16") == 2 * n
+    assert L.lpar_workspace_bytes(0, n, "int4") == 0
+    assert L.lpar_workspace_bytes(9, n, "int4") == 0
+
+
+def test_effective_codec_threshold(L):
+    thr = 1 << 20
+    assert L.lpar_effective_codec(thr // 2, "int3", thr) == "int3"          # 1 MiB message: >= threshold
+    assert L.lpar_effective_codec(thr // 2 - 2048, "int3", thr) == "bf16"
+    assert L.lpar_effective_codec(2048, "fp8", 0) == "fp8"
+    assert L.lpar_effective_codec(2048, "bf16", thr) == "bf16"
+
+
+# Fake, never-dereferenced device addresses: every call below must fail in
+# validation before any launch.
+A = 0x7F0000000000          # 16-byte aligned
+M = A + 8                   # misaligned
+
+
+def status_of(fn, *args, **kw):
+    from quantized_precision_all_b200.lpar import LparError
+    try:
+        fn(*args, **kw)
+    except LparError as e:
+        return e.status
+    return 0
+
+
+def test_argument_errors_quantize(L):
+    st = 0
+    assert status_of(L.lpar_quantize, A, 2048, 9, A, st) == 4            # unknown codec
+    assert status_of(L.lpar_quantize, A, 2047, "int4", A, st) == 1       # n not a tile multiple
+    assert status_of(L.lpar_quantize, 0, 2048, "int4", A, st) == 1       # null input
+    assert status_of(L.lpar_quantize, A, 2048, "int4", 0, st) == 1       # null wire
+    assert status_of(L.lpar_quantize, M, 2048, "int4", A, st) == 2       # misaligned
+    assert status_of(L.lpar_quantize, A, 2048, "int3", M, st) == 2
+    assert status_of(L.lpar_quantize, 0, 0, "int4", 0, st) == 0          # empty message: no-op
+
+
+def test_argument_errors_reduce_decode(L):
+    st = 0
+    assert status_of(L.lpar_reduce, [A] * 9, 0, 1, "int4", A, st) == 1   # N > 8
+    assert status_of(L.lpar_reduce, [A, 0], 0, 1, "int4", A, st) == 1    # null wire
+    assert status_of(L.lpar_reduce, [A, M], 0, 1, "int4", A, st) == 2
+    assert status_of(L.lpar_reduce, [A, A], 0, 1, "int4", M, st) == 2
+    assert status_of(L.lpar_reduce, [A, A], 0, 1, 5, A, st) == 4
+    assert status_of(L.lpar_reduce, [A, A], 2 ** 64 - 1, 2, "int4", A, st) == 1   # range overflow
+    assert status_of(L.lpar_reduce, [A, A], 3, 0, "int4", A, st) == 0    # empty range: no-op
+    assert status_of(L.lpar_decode, A, 100, "int4", A, st) == 1
+    assert status_of(L.lpar_decode, A, 2048, "fp8", M, st) == 2
+    assert status_of(L.lpar_decode, 0, 2048, "fp8", A, st) == 1
+
+
+def test_argument_errors_allreduce(L):
+    st = 0
+    n = 2048 * 4
+    ws = L.lpar_workspace_bytes(2, n, "int4")
+    ok = dict(min_quant_bytes=0, schedule="fused", stream=st)
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws - 16, **ok) == 3
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, M], A, ws, **ok) == 2
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], M, ws, **ok) == 2
+    assert status_of(L.lpar_allreduce, [A, 0], n, "int4", [A, A], A, ws, **ok) == 1
+    assert status_of(L.lpar_allreduce, [A, A], n + 1, "int4", [A, A], A, ws, **ok) == 1
+    assert status_of(L.lpar_allreduce, [A] * 9, n, "int4", [A] * 9, A, 10 ** 9, **ok) == 1
+    assert status_of(L.lpar_allreduce, [A, A], n, 11, [A, A], A, ws, **ok) == 4
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws, min_quant_bytes=0, schedule=7,
+                     stream=st) == 4
+    assert status_of(L.lpar_allreduce, [A, A], 0, "int4", [A, A], A, 0, **ok) == 0
+    # raw C call with null arrays
+    lib = L.library()
+    opts = L.lpar_options_t(0, 0)
+    assert lib.lpar_allreduce(None, 2, n, 2, None, A, ws, ctypes.byref(opts), None) == 1
+    assert lib.lpar_allreduce(None, 2, n, 2, None, A, ws, None, None) == 1
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.lpar_status_string(s)
+    assert "unknown" in L.lpar_status_string(99)
+
+
+def test_python_binding_rejects_host_tensors(L):
+    import torch
+    x = torch.zeros(2048, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        L.lpar_quantize(x, 2048, "int4", x)

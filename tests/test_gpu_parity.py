@@ -1,0 +1,400 @@
+"""CUDA path vs the CPU oracle, element by element (needs a B200).
+
+Every comparison is bit-exact: wires (codes + scales) byte for byte and BF16
+outputs bit for bit -- the path is deterministic and follows the same
+definitions, so the 1-ulp BF16 allowance is not needed.  Inputs are seeded and
+synthetic; expected values come only from the oracle.  Every device buffer the
+library writes has 4 KiB guard bands on both sides, checked after each call.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096
+CANARY = 0xA5
+CODECS = ("int4", "int3", "fp8", "bf16")
+QCODECS = ("int4", "int3", "fp8")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_precision_all_b200 import build
+    build.build()
+    from quantized_precision_all_b200 import lpar
+    return lpar
+
+
+class Guarded:
+    """A device byte buffer with canary bands on both sides."""
+
+    def __init__(self, nbytes, fill=CANARY):
+        self.nbytes = nbytes
+        self.buf = torch.full((nbytes + 2 * GUARD,), fill, dtype=torch.uint8, device="cuda")
+        self.buf[:GUARD] = CANARY
+        self.buf[GUARD + nbytes:] = CANARY
+
+    @property
+    def t(self):
+        return self.buf[GUARD:GUARD + self.nbytes]
+
+    def ptr(self):
+        return self.t.data_ptr()
+
+    def host(self):
+        return self.t.cpu().numpy()
+
+    def check(self):
+        assert torch.all(self.buf[:GUARD] == CANARY), "front guard overwritten"
+        assert torch.all(self.buf[GUARD + self.nbytes:] == CANARY), "back guard overwritten"
+
+
+def to_device(bits_u16):
+    g = Guarded(bits_u16.size * 2)
+    g.t.copy_(torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.uint8)))
+    return g
+
+
+def host_u16(g):
+    return g.host().view(np.uint16)
+
+
+def f16_value(bits):
+    return float(np.array([bits], np.uint16).view(np.float16)[0])
+
+
+# ---------------------------------------------------------------------------
+# Adversarial BF16 inputs (seeded): block kinds cycle through random normal at
+# random scales, all-zero, single outliers, exact ties of the INT grids,
+# saturating magnitudes, tiny magnitudes (subnormal scales), negative zeros.
+# ---------------------------------------------------------------------------
+def bf16(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def adversarial_bf16(n, seed):
+    rng = np.random.default_rng(seed)
+    nb = n // 32
+    x = np.zeros((nb, 32), np.float32)
+    kinds = rng.integers(0, 9, nb)
+    for b in range(nb):
+        k = kinds[b]
+        if k == 0:
+            x[b] = rng.standard_normal(32) * 10.0 ** rng.uniform(-4, 4)
+        elif k == 1:
+            pass                                                     # all zero
+        elif k == 2:
+            x[b] = rng.standard_normal(32) * 0.01
+            x[b, rng.integers(32)] = rng.choice([-1, 1]) * 10.0 ** rng.uniform(0, 6)
+        elif k in (3, 4):
+            # on-grid block with ties: s = m * 2^e with a 3-bit m keeps (k + 1/2) s in BF16
+            qmax = 7 if k == 3 else 3
+            s = rng.choice([1.0, 1.25, 1.5, 1.75]) * 2.0 ** rng.integers(-12, 12)
+            q = rng.integers(-qmax, qmax, 32) + rng.choice([0.0, 0.5], 32)
+            q[rng.integers(32)] = qmax * rng.choice([-1, 1])
+            x[b] = q * s
+        elif k == 5:
+            x[b] = rng.standard_normal(32) * 10.0 ** rng.uniform(5, 37)  # saturating scales
+        elif k == 6:
+            x[b] = rng.standard_normal(32) * 10.0 ** rng.uniform(-39, -4)  # subnormal / zero scales
+        elif k == 7:
+            x[b] = -0.0
+            x[b, rng.integers(32)] = rng.standard_normal()
+        else:
+            # FP8 ties and saturation: E4M3 grid points and midpoints at a power-of-two scale
+            e = rng.integers(-20, 20)
+            grid = np.array([0.0, 0.5, 1, 1.5, 2, 2.25, 2.5, 3, 17, 18, 19, 240, 416, 432, 440, 448], np.float32)
+            x[b] = rng.choice(grid, 32) * rng.choice([-1, 1], 32) * 2.0 ** e
+            x[b, rng.integers(32)] = 448 * 2.0 ** e
+    bits = bf16(x.reshape(-1))
+    neg0 = (kinds == 7).repeat(32) & (x.reshape(-1) == 0)
+    bits[neg0] = 0x8000
+    return bits
+
+
+def random_bf16(n, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(n, generator=g) * scale).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# Stage 1
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("tiles", [1, 3, 5, 37])
+def test_quantize_matches_oracle(L, codec, tiles):
+    n = tiles * 2048
+    x = adversarial_bf16(n, seed=1000 + tiles)
+    dx = to_device(x)
+    wire = Guarded(L.lpar_wire_bytes(codec, n))
+    L.lpar_quantize(dx.ptr(), n, codec, wire.ptr())
+    torch.cuda.synchronize()
+    wire.check()
+    dx.check()
+    assert np.array_equal(wire.host(), O.quantize(x, codec))
+
+
+@pytest.mark.parametrize("codec", QCODECS)
+def test_quantize_every_bf16_value_as_block_absmax_candidate(L, codec):
+    # block p = [bf16 pattern p, 31 fixed values]: every finite BF16 value meets the scale path
+    pats = np.array([p for p in range(0x10000) if (p & 0x7F80) != 0x7F80], np.uint16)
+    pats = np.concatenate([pats, np.zeros((-len(pats)) % 64, np.uint16)])
+    others = random_bf16(31, seed=7, scale=3.0)
+    x = np.empty((len(pats), 32), np.uint16)
+    x[:, 0] = pats
+    x[:, 1:] = others
+    x = x.reshape(-1)
+    n = x.size
+    dx = to_device(x)
+    wire = Guarded(L.lpar_wire_bytes(codec, n))
+    L.lpar_quantize(dx.ptr(), n, codec, wire.ptr())
+    torch.cuda.synchronize()
+    wire.check()
+    assert np.array_equal(wire.host(), O.quantize(x, codec))
+
+
+# ---------------------------------------------------------------------------
+# Stage 3
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("codec", CODECS)
+def test_decode_matches_oracle(L, codec):
+    n = 2048 * 11
+    wire = O.quantize(adversarial_bf16(n, seed=31), codec)
+    dw = Guarded(wire.size)
+    dw.t.copy_(torch.from_numpy(wire))
+    out = Guarded(2 * n)
+    L.lpar_decode(dw.ptr(), n, codec, out.ptr())
+    torch.cuda.synchronize()
+    out.check()
+    assert np.array_equal(host_u16(out), O.decode(wire, n, codec))
+
+
+@pytest.mark.parametrize("codec", ["int4", "int3"])
+def test_decode_arbitrary_code_bytes(L, codec):
+    # any code byte pattern is a valid INT code; keep scales finite
+    n = 2048 * 6
+    rng = np.random.default_rng(32)
+    wire = rng.integers(0, 256, L.lpar_wire_bytes(codec, n), dtype=np.uint8)
+    tb = L.lpar_tile_bytes(codec)
+    for t in range(n // 2048):
+        sc = rng.integers(0, 0x7C00, 64).astype(np.uint16) | (rng.integers(0, 2, 64).astype(np.uint16) << 15)
+        wire[t * tb + tb - 128:t * tb + tb] = sc.view(np.uint8)
+    dw = Guarded(wire.size)
+    dw.t.copy_(torch.from_numpy(wire))
+    out = Guarded(2 * n)
+    L.lpar_decode(dw.ptr(), n, codec, out.ptr())
+    torch.cuda.synchronize()
+    assert np.array_equal(host_u16(out), O.decode(wire, n, codec))
+
+
+# ---------------------------------------------------------------------------
+# Stage 2
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("N", [1, 2, 3, 5, 8])
+def test_reduce_matches_oracle_on_a_tile_range(L, codec, N):
+    tiles = 13
+    n = tiles * 2048
+    wires = [O.quantize(adversarial_bf16(n, seed=200 + r) if r % 2 else random_bf16(n, 300 + r, 10.0 ** (r - 3)),
+                        codec) for r in range(N)]
+    dws = []
+    for w in wires:
+        g = Guarded(w.size)
+        g.t.copy_(torch.from_numpy(w))
+        dws.append(g)
+    out = Guarded(wires[0].size)                      # pre-filled with the canary byte
+    t0, cnt = 2, 9                                    # a ragged range: 2 full CTAs + 1 tile
+    L.lpar_reduce([g.ptr() for g in dws], t0, cnt, codec, out.ptr())
+    torch.cuda.synchronize()
+    out.check()
+    ref = O.reduce(wires, t0, cnt, codec, wire_out=np.full(wires[0].size, CANARY, np.uint8))
+    assert np.array_equal(out.host(), ref)            # tiles outside the range untouched
+
+
+@pytest.mark.parametrize("bits,codec", [(4, "int4"), (3, "int3")])
+def test_reduce_exact_ties_at_stage_two(L, bits, codec):
+    # rank 0 holds q0 * S (absmax qmax * S), rank 1 holds odd multiples of S/2 with
+    # its own absmax qmax * S/2, so every FP32 sum is an exact tie (k + 1/2) S of the
+    # requantisation grid while the block absmax stays qmax * S.
+    qmax = 2 ** (bits - 1) - 1
+    rng = np.random.default_rng(40 + bits)
+    n = 2048 * 5
+    x0 = np.zeros(n, np.float32)
+    x1 = np.zeros(n, np.float32)
+    for b in range(n // 32):
+        S = rng.choice([1.0, 1.25, 1.5, 1.75]) * 2.0 ** rng.integers(-10, 10)
+        q1 = rng.choice(np.arange(-qmax, qmax + 1, 2), 32).astype(np.float32)   # odd multiples
+        q0 = rng.integers(-(qmax // 2), qmax // 2 + 1, 32).astype(np.float32)
+        q0[0], q1[0] = qmax, 0                          # absmax of the sum: qmax * S
+        j = 1 + rng.integers(31)
+        q0[j], q1[j] = 0, qmax                          # rank 1's own absmax
+        x0[b * 32:(b + 1) * 32] = q0 * S
+        x1[b * 32:(b + 1) * 32] = q1 * S / 2
+    wires = [O.quantize(bf16(x0), codec), O.quantize(bf16(x1), codec)]
+    dws = []
+    for w in wires:
+        g = Guarded(w.size)
+        g.t.copy_(torch.from_numpy(w))
+        dws.append(g)
+    out = Guarded(wires[0].size)
+    L.lpar_reduce([g.ptr() for g in dws], 0, n // 2048, codec, out.ptr())
+    torch.cuda.synchronize()
+    ref = O.reduce(wires, 0, n // 2048, codec)
+    assert np.array_equal(out.host(), ref)
+    # the construction really produced ties: sums are odd multiples of S/2
+    v = np.concatenate([O.dequant_tile(wires[0][t * len(wires[0]) // 5:(t + 1) * len(wires[0]) // 5], codec)
+                        + O.dequant_tile(wires[1][t * len(wires[1]) // 5:(t + 1) * len(wires[1]) // 5], codec)
+                        for t in range(5)])
+    assert np.count_nonzero(v) > n // 2
+
+
+def test_reduce_bf16_rounding_ties(L):
+    # 1 + 2^-8 is halfway between two BF16 neighbours; 1 + 3*2^-8 likewise
+    n = 2048
+    a = np.full(n, 0x3F80, np.uint16)                            # 1.0
+    b = bf16(np.where(np.arange(n) % 2 == 0, 2.0 ** -8, 3 * 2.0 ** -8).astype(np.float32))
+    wires = [a.view(np.uint8).copy(), b.view(np.uint8).copy()]
+    dws = []
+    for w in wires:
+        g = Guarded(w.size)
+        g.t.copy_(torch.from_numpy(w))
+        dws.append(g)
+    out = Guarded(2 * n)
+    L.lpar_reduce([g.ptr() for g in dws], 0, 1, "bf16", out.ptr())
+    torch.cuda.synchronize()
+    assert np.array_equal(out.host(), O.reduce(wires, 0, 1, "bf16"))
+
+
+# ---------------------------------------------------------------------------
+# The whole all-reduce
+# ---------------------------------------------------------------------------
+def run_allreduce(L, xs, codec, schedule="fused", min_quant_bytes=0, inplace=False):
+    N, n = len(xs), xs[0].size
+    ins = [to_device(x) for x in xs]
+    outs = ins if inplace else [Guarded(2 * n, fill=0x00) for _ in range(N)]
+    ws = Guarded(L.lpar_workspace_bytes(N, n, L.lpar_effective_codec(n, codec, min_quant_bytes)))
+    L.lpar_allreduce([g.ptr() for g in ins], n, codec, [g.ptr() for g in outs], ws.ptr(), ws.nbytes,
+                     min_quant_bytes=min_quant_bytes, schedule=schedule)
+    torch.cuda.synchronize()
+    for g in outs + [ws] + ([] if inplace else ins):
+        g.check()
+    return [host_u16(g) for g in outs], ws
+
+
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("N", [1, 2, 3, 8])
+@pytest.mark.parametrize("schedule", ["fused", "three_stage"])
+def test_allreduce_matches_oracle(L, codec, N, schedule):
+    tiles = 9                                          # 2 CTAs + a ragged one per rank
+    n = tiles * 2048
+    xs = [adversarial_bf16(n, 500 + r) if r % 2 else random_bf16(n, 600 + r) for r in range(N)]
+    outs, ws = run_allreduce(L, xs, codec, schedule)
+    ref, used = O.allreduce(xs, codec)
+    assert used == codec
+    for o in outs:
+        assert np.array_equal(o, ref[0])
+    if codec != "bf16":
+        # the workspace holds the stage-1 wires and the gathered wire, as the oracle's
+        wb = L.lpar_wire_bytes(codec, n)
+        host = ws.host()
+        wires = [O.quantize(x, codec) for x in xs]
+        for r in range(N):
+            assert np.array_equal(host[r * wb:(r + 1) * wb], wires[r])
+        assert np.array_equal(host[N * wb:(N + 1) * wb], O.reduce(wires, 0, tiles, codec))
+
+
+@pytest.mark.parametrize("codec", CODECS)
+def test_allreduce_in_place(L, codec):
+    n = 2048 * 6
+    xs = [random_bf16(n, 700 + r, 2.0) for r in range(3)]
+    outs, _ = run_allreduce(L, xs, codec, inplace=True)
+    ref, _ = O.allreduce(xs, codec)
+    for o in outs:
+        assert np.array_equal(o, ref[0])
+
+
+def test_threshold_sends_small_messages_to_bf16(L):
+    w = W.WORKLOADS["decode_int3"]
+    thr = w.min_quant_bytes
+    for n, expect in ((w.n, "int3"), (w.n - 2048, "bf16")):
+        xs = [t.view(torch.int16).numpy().view(np.uint16) for t in W.make_inputs(w, "cpu", n=n)]
+        outs, _ = run_allreduce(L, xs, "int3", min_quant_bytes=thr)
+        ref, used = O.allreduce(xs, "int3", min_quant_bytes=thr)
+        assert used == expect
+        assert np.array_equal(outs[0], ref[0]) and np.array_equal(outs[1], ref[0])
+
+
+def test_empty_message_is_a_no_op(L):
+    ws = Guarded(16)
+    L.lpar_allreduce([ws.ptr()], 0, "int4", [ws.ptr()], ws.ptr(), 16)
+    L.lpar_quantize(ws.ptr(), 0, "int3", ws.ptr())
+    L.lpar_decode(ws.ptr(), 0, "fp8", ws.ptr())
+    L.lpar_reduce([ws.ptr()], 0, 0, "int4", ws.ptr())
+    torch.cuda.synchronize()
+    assert torch.all(ws.buf == CANARY)
+
+
+# ---------------------------------------------------------------------------
+# The named workloads
+# ---------------------------------------------------------------------------
+def workload_bits(w, n=None):
+    return [t.view(torch.int16).numpy().view(np.uint16) for t in W.make_inputs(w, "cpu", n=n)]
+
+
+@pytest.mark.parametrize("name", ["small_int4", "decode_int3"])
+def test_workload_full_oracle(L, name):
+    w = W.WORKLOADS[name]
+    xs = workload_bits(w)
+    for codec in w.codecs:
+        for schedule in ("fused", "three_stage"):
+            outs, _ = run_allreduce(L, xs, codec, schedule, min_quant_bytes=w.min_quant_bytes)
+            ref, used = O.allreduce(xs, codec, min_quant_bytes=w.min_quant_bytes)
+            assert used == codec
+            for o in outs:
+                assert np.array_equal(o, ref[0])
+
+
+def test_workload_prefill_fp8_full_oracle_and_error_report(L):
+    w = W.WORKLOADS["prefill_fp8"]
+    xs = workload_bits(w)
+    exact = np.zeros(w.n, np.float64)
+    for x in xs:
+        exact += O.bf16_bits_to_f32(x).astype(np.float64)
+    errs = {}
+    for codec in w.codecs:                               # FP8, then the uncompressed BF16 sum
+        outs, _ = run_allreduce(L, xs, codec)
+        ref, _ = O.allreduce(xs, codec)
+        for o in outs:
+            assert np.array_equal(o, ref[0])
+        e = O.bf16_bits_to_f32(outs[0]).astype(np.float64) - exact
+        errs[codec] = (float(np.max(np.abs(e))), float(np.sqrt(np.mean(e * e))))
+    print("prefill_fp8 error vs exact sum (max, rms):", errs)
+    assert errs["bf16"][1] <= errs["fp8"][1]
+
+
+def test_workload_large_sampled_tiles(L):
+    """1 GiB per rank, INT3 then INT4, in the launch configuration the bench times;
+    compared on 1024 seeded random tiles plus the first and the last (tiles are
+    independent, so a tile's result depends only on that tile of every rank)."""
+    w = W.WORKLOADS["large_int3_int4"]
+    xs = W.make_inputs(w, "cuda")
+    T = w.n // 2048
+    rng = np.random.default_rng(4)
+    tiles = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 1024, replace=False)]))
+    idx = torch.from_numpy((tiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
+    sample_in = [x[idx].view(torch.int16).cpu().numpy().view(np.uint16) for x in xs]
+    for codec in w.codecs:
+        outs = [torch.empty_like(x) for x in xs]
+        ws = torch.empty(L.lpar_workspace_bytes(w.N, w.n, codec), dtype=torch.uint8, device="cuda")
+        L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel())
+        torch.cuda.synchronize()
+        ref, _ = O.allreduce(sample_in, codec)
+        for o in outs:
+            got = o[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+            assert np.array_equal(got, ref[0])
+        del outs, ws
+    torch.cuda.empty_cache()

@@ -62,6 +62,16 @@ WORKLOADS = {
              "INT3 then INT4 back to back"),
 }
 
+# A smaller case of the large workload for ncu captures: inputs (256 MiB) still
+# exceed the 126 MB L2, while the whole footprint stays under 1 GiB.
+PROFILE_WORKLOADS = {
+    "profile_int3_int4": Workload(
+        "profile_int3_int4", N=2, n=64 * 1024 * 1024, dist="normal", sigma=0.02, seed=4,
+        codecs=("int3", "int4"),
+        note="profiling case: N=2 x 64 Mi BF16 (128 MiB per rank), N(0, 0.02^2), INT3 then INT4"),
+}
+WORKLOADS.update(PROFILE_WORKLOADS)
+
 SWEEP_SIZES_BYTES = [1 << k for k in range(17, 31)]    # 128 KiB ... 1 GiB per rank
 SWEEP_RANKS = (2, 4, 8)
 SWEEP_CODECS = ("bf16", "fp8", "int4", "int3")
