@@ -206,6 +206,11 @@ def run_ours(args, rank, world, device):
     # (2) per-kernel durations, live: stage events recorded between the kernels
     ksteps = max(1, min(args.steps, 200))
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in w.codecs] for _ in range(ksteps)]
+    for per_step in evs:                     # torch creates the CUDA event on its first record()
+        for per_codec in per_step:
+            for ev in per_codec:
+                ev.record(stream)
+    torch.cuda.synchronize(device)
     for s in range(ksteps):
         step(evs[s])
     torch.cuda.synchronize(device)

@@ -12,13 +12,38 @@
 //   FP8 E4M3:  s = fl32(absmax / 448), zero block when s < 2^-126,
 //              code = e4m3_rne_satfinite(fl32(x * fl32(1 / s))).
 //
-// Exact RNE(x / s) without a per-element division.  With h = fl(x * fl(1/s))
-// (relative error < 2^-22) let k = RNE(h - 1/2); k is RNE(x/s) or one less.
+// Exact RNE(x / s) without a per-element division
+// -----------------------------------------------
+// Fast path (normal, unsaturated binary16 scale, so |x/s| <= qmax(1 + 2^-11)):
+// r approximates 1/s within 2^-23 (one hardware reciprocal), so the exact
+// product x*r is within 7.01 * 2^-23 < 2^-19.9 of Q = x/s.  Two FMAs round that
+// exact product with the add-magic trick: fl(x*r + M), M = 1.5*2^23 (ulp 1),
+// gives k0 = RNE(x*r); fl(x*r + 2M) (ulp 2) gives 2*k2, the even integer
+// nearest to x*r.  With f = fl(x*r - k0):
+//   |f| <  1/2 - 2^-18  =>  |Q - k0| < 1/2, so k0 = RNE(Q) (and Q is no tie);
+//   Q an exact tie k + 1/2  =>  |f| >= 1/2 - 2^-18 and 2*k2 is the even one of
+//                               k, k+1, i.e. RNE(Q).
+// So q = (|f| >= 1/2 - 2^-18) ? 2*k2 : k0.  At stage 1 (BF16 x, 8-bit
+// significand; binary16 s, 11 bits) a non-tie quotient is at least 2^-12 from a
+// half-integer, so |f| >= 1/2 - 2^-18 only at exact ties and the fast path is
+// exact as it stands.  At stage 2 (binary32 sums) such an element is accepted
+// only when the exact residual x - k0*s (one FMA, exact) equals +-s/2;
+// otherwise the block is redone on the exact path (a near tie, rare).
+// Blocks with a subnormal, zero or saturated scale take the exact path.
+//
+// Exact path: k = RNE(fl(x*r) - 1/2) is RNE(x/s) or one less; the midpoint
 // m = (k + 1/2) * s is exact in binary32 ((2k+1) has <= 5 bits, s <= 11 bits),
-// so comparing x with m decides the last step exactly: q = k + 1 when x > m,
-// or when x == m (a tie) and k is odd (ties to even); otherwise q = k.
-// k is found with the add-magic trick: fl(h' + (1.5*2^23 + bias)) puts
-// k + bias in the low mantissa bits, which is the offset-binary code itself.
+// so comparing x with m decides exactly: q = k + 1 when x > m, or when x == m
+// and k is odd (ties to even); otherwise q = k.
+//
+// Scale: fl32(absmax / qmax) by Markstein's correction (IBM J. Res. Dev. 34,
+// 1990): y = RN(1/qmax), q0 = RN(a*y), rem = fma(-q0, qmax, a) (exact),
+// result = RN(q0 + rem*y).  For qmax = 7 and 3 this equals the IEEE quotient for
+// every non-negative binary32 a (checked exhaustively on the host).
+//
+// Codes are packed with exact binary32 polynomials: for codes c_m of a group,
+// Sum c_m 2^(w m) is formed by an FMA chain (< 2^24, exact) and added to M,
+// which puts the packed bits in the low mantissa of the result.
 #pragma once
 
 #include <cstdint>
@@ -54,11 +79,80 @@ template <> struct Packed<kINT4> { uint32_t w[4]; uint16_t scale; };          //
 template <> struct Packed<kINT3> { uint32_t q2w[2]; uint32_t q1w; uint16_t scale; };
 template <> struct Packed<kFP8> { uint32_t w[8]; float scale; };              // 32 B codes
 
+constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23: ulp 1, bits 0x4B400000
+constexpr float kMagic2 = 25165824.0f;                // 3 * 2^23 = 1.5 * 2^24: ulp 2
+constexpr float kTieTh = 0.5f - 0x1p-18f;             // |f| >= kTieTh: tie (or, at stage 2, a near tie)
+
 // ---------------------------------------------------------------------------
 // Small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Packed binary32 pairs (sm_100 f32x2 arithmetic; each lane rounds like the
+// scalar instruction, to nearest even, subnormals kept).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
+
+// fl32(a * s + c) with a, s binary16 (the low or high half of a packed word):
+// the product of two binary16 values is exact in binary32, so this rounds once.
+__device__ __forceinline__ float fma_h(uint32_t a_pair, int hi, uint16_t s, float c) {
+    float d;
+    if (hi)
+        asm("{.reg .f16 l, h, s;\n\tmov.b32 {l, h}, %1;\n\tmov.b16 s, %2;\n\t"
+            "fma.rn.f32.f16 %0, h, s, %3;}" : "=f"(d) : "r"(a_pair), "h"(s), "f"(c));
+    else
+        asm("{.reg .f16 l, h, s;\n\tmov.b32 {l, h}, %1;\n\tmov.b16 s, %2;\n\t"
+            "fma.rn.f32.f16 %0, l, s, %3;}" : "=f"(d) : "r"(a_pair), "h"(s), "f"(c));
+    return d;
+}
+
+// Exact binary32 value of one half of a packed binary16 pair.
+__device__ __forceinline__ float h2f(uint32_t pair, int hi) {
+    return fma_h(pair, hi, 0x3C00u /* 1.0 */, -0.0f);
+}
+
+// Packed binary16 pair minus a packed constant (exact for the small integers used here).
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 // Two binary32 -> packed BF16x2, round to nearest even; lo lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -74,12 +168,11 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
     return d;
 }
 
-// Packed E4M3x2 (16 bits) -> two exact binary32 values (E4M3 is a subset of binary16).
-__device__ __forceinline__ void unpack_e4m3x2(uint32_t two, float &lo, float &hi) {
+// Packed E4M3x2 (16 bits) -> packed binary16 pair (exact: E4M3 is a subset of binary16).
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two));
-    lo = __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFF)));
-    hi = __half2float(__ushort_as_half((uint16_t)(h2 >> 16)));
+    return h2;
 }
 
 // Maximum of |bf16| over a packed pair, as a packed pair; the sign bits are
@@ -104,53 +197,75 @@ __device__ __forceinline__ float absmax_bf16x32(const uint32_t (&w)[16]) {
     return __uint_as_float((lo > hi ? lo : hi) << 16);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ float absmax_f32x32(const float (&x)[32]) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    float a[11];
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-        a0 = fmaxf(a0, fabsf(x[j]));
-        a1 = fmaxf(a1, fabsf(x[j + 1]));
-        a2 = fmaxf(a2, fabsf(x[j + 2]));
-        a3 = fmaxf(a3, fabsf(x[j + 3]));
-    }
-    return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    for (int i = 0; i < 10; ++i) a[i] = max3(fabsf(x[3 * i]), fabsf(x[3 * i + 1]), fabsf(x[3 * i + 2]));
+    a[10] = fmaxf(fabsf(x[30]), fabsf(x[31]));
+    const float b0 = max3(a[0], a[1], a[2]), b1 = max3(a[3], a[4], a[5]);
+    const float b2 = max3(a[6], a[7], a[8]), b3 = fmaxf(a[9], a[10]);
+    return fmaxf(max3(b0, b1, b2), b3);
 }
 
 // ---------------------------------------------------------------------------
-// INT4 / INT3 block quantiser.  x[32] in binary32 (exact BF16 values at stage 1,
-// FP32 sums at stage 2), a = max|x|.
+// INT4 / INT3 block scale.
 // ---------------------------------------------------------------------------
 struct IntScale {
     uint16_t bits;   // binary16 scale as stored in the tile
     float s;         // its value
     float r;         // fl(1/s), or 0 when s == 0
     float hs;        // s/2, or +inf when s == 0 (nothing ever rounds up)
-    float lim;       // (qmax + 1) * s: bound applied on the slow path
+    float lim;       // (qmax + 1) * s: bound applied on the exact path
     bool fast;       // normal, unsaturated scale: |x/s| <= qmax (1 + 2^-11), no clamp needed
 };
+
+// fl32(a / qmax), equal to the IEEE quotient (see the header comment).
+template <int BITS>
+__device__ __forceinline__ float div_qmax(float a) {
+    constexpr float q = (float)((1 << (BITS - 1)) - 1);
+    const float y = __uint_as_float(BITS == 4 ? 0x3E124925u : 0x3EAAAAABu);   // RN(1/7), RN(1/3)
+    const float q0 = __fmul_rn(a, y);
+    const float rem = __fmaf_rn(-q0, q, a);
+    return __fmaf_rn(rem, y, q0);
+}
+
+// Hardware reciprocal, relative error below 2^-23.
+__device__ __forceinline__ float rcp_approx(float s) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
+}
 
 template <int BITS>
 __device__ __forceinline__ IntScale int_scale(float a) {
     constexpr int kQmax = (1 << (BITS - 1)) - 1;
     IntScale k;
-    const float ratio = __fdiv_rn(a, (float)kQmax);                  // one IEEE division per block
+    const float ratio = div_qmax<BITS>(a);
     uint16_t sb = __half_as_ushort(__float2half_rn(ratio));
     if (sb == 0x7C00u) sb = 0x7BFFu;                                   // saturate at 65504
     k.bits = sb;
     k.s = __half2float(__ushort_as_half(sb));
     k.fast = (sb >= 0x0400u) && (sb != 0x7BFFu);
-    k.r = (k.s != 0.f) ? __frcp_rn(k.s) : 0.f;
+    k.r = (k.s != 0.f) ? rcp_approx(k.s) : 0.f;
     k.hs = (k.s != 0.f) ? 0.5f * k.s : __int_as_float(0x7F800000);
     k.lim = (float)(kQmax + 1) * k.s;                                 // exact
     return k;
 }
 
-// Offset-binary code of one element (low byte) and, when wanted, q * s.
+// ---------------------------------------------------------------------------
+// Exact path (any scale; used for flagged blocks).
+// ---------------------------------------------------------------------------
 template <int BITS, bool FAST, bool WANT_V>
 __device__ __forceinline__ uint32_t int_code(float x, const IntScale &k, float &v) {
     constexpr int kQmax = (1 << (BITS - 1)) - 1;
     constexpr int kBias = 1 << (BITS - 1);
-    const float magic = 12582912.0f + (float)kBias;                   // 1.5 * 2^23 + bias
+    const float magic = kMagic + (float)kBias;                        // 1.5 * 2^23 + bias
     if (!FAST) x = fminf(fmaxf(x, -k.lim), k.lim);                    // keeps |x/s| <= qmax + 1
     const float hm = __fmaf_rn(x, k.r, -0.5f);                        // ~ x/s - 1/2
     const float C = __fadd_rn(hm, magic);                             // magic + RNE(hm)
@@ -167,115 +282,96 @@ __device__ __forceinline__ uint32_t int_code(float x, const IntScale &k, float &
     return c;
 }
 
-// INT4: 8 codes of elements 8i..8i+7 -> one word (element 8i in the low nibble).
-template <bool FAST, bool WANT_V>
-__device__ __forceinline__ void int4_body(const float (&x)[32], const IntScale &k, uint32_t (&w)[4],
-                                          uint32_t (&o)[16]) {
+// ---------------------------------------------------------------------------
+// Fast path.  Returns false when some element is near a tie (the caller then
+// redoes the block on the exact path); outputs are only valid when true.
+// ---------------------------------------------------------------------------
+
+// One element pair -> -q (q = RNE(x/s), exact, see the header comment).
+// STAGE2: sets `bad` when a tie-like residual is not an exact tie.
+template <bool STAGE2>
+__device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, bool &bad) {
+    const float2 r2 = splat(k.r), M2 = splat(kMagic), M4 = splat(kMagic2);
+    const float2 C = fma2(xv, r2, M2);                 // M + RNE(x r), exact product inside
+    const float2 nk = sub2(M2, C);                     // -k0
+    const float2 C2 = fma2(xv, r2, M4);                // 2M + 2 RNE(x r / 2)
+    const float2 nq2 = sub2(M4, C2);                   // -2 k2
+    const float2 f = fma2(xv, r2, nk);                 // x r - k0
+    const bool tx = fabsf(f.x) >= kTieTh, ty = fabsf(f.y) >= kTieTh;
+    if (STAGE2) {
+        const float2 e = fma2(nk, splat(k.s), xv);     // x - k0 s, exact
+        bad |= (tx && fabsf(e.x) != k.hs) || (ty && fabsf(e.y) != k.hs);
+    }
+    return make_float2(tx ? nq2.x : nk.x, ty ? nq2.y : nk.y);
+}
+
+// INT4: lanes hold elements (8i + m, 8i + 4 + m); each lane packs 4 nibbles
+// (16 bits) with Q = Sum_m (-q_m) 16^m, P = (M + 0x8888) - Q.
+// Decoded BF16 output goes to `sink.put(piece, uint4)`: piece j holds the
+// packed words 4j..4j+3 (elements 8j..8j+7), written as soon as they exist.
+template <bool STAGE2, bool WANT_V, class Sink>
+__device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &k, uint32_t (&w)[4],
+                                          const Sink &sink) {
+    const float2 ns2 = splat(-k.s), S16 = splat(16.f);
+    bool bad = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        uint32_t c[8];
-        float v[8];
+        float2 nq[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c[j] = int_code<4, FAST, WANT_V>(x[8 * i + j], k, v[j]);
-        const uint32_t b0 = c[0] | (c[1] << 4), b1 = c[2] | (c[3] << 4);
-        const uint32_t b2 = c[4] | (c[5] << 4), b3 = c[6] | (c[7] << 4);
-        w[i] = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+        for (int m = 0; m < 4; ++m) nq[m] = round_pair<STAGE2>(make_float2(x[8 * i + m], x[8 * i + 4 + m]), k, bad);
+        float2 Q = fma2(nq[3], S16, nq[2]);
+        Q = fma2(Q, S16, nq[1]);
+        Q = fma2(Q, S16, nq[0]);
+        const float2 P = sub2(splat(kMagic + 34952.0f), Q);     // 34952 = 0x8888: bias 8 per nibble
+        w[i] = __byte_perm(__float_as_uint(P.x), __float_as_uint(P.y), 0x5410);
         if (WANT_V) {
+            float2 v[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) o[4 * i + q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+            for (int m = 0; m < 4; ++m) v[m] = fma2(nq[m], ns2, splat(0.f));   // q s (+0 for q = 0)
+            sink.put(i, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
+                                   pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y)));
         }
     }
+    return !bad;
 }
 
-// INT3: 4 codes of elements 4g..4g+3 -> q2w byte g (2 bits each) and q1w bits 4g..4g+3.
-template <bool FAST, bool WANT_V>
-__device__ __forceinline__ void int3_body(const float (&x)[32], const IntScale &k, uint32_t (&q2w)[2],
-                                          uint32_t &q1w, uint32_t (&o)[16]) {
-    q2w[0] = q2w[1] = 0u;
-    q1w = 0u;
+// INT3: lanes hold elements (16p + m, 16p + 8 + m).  hi = (q >= 0) comes from
+// RNE(q/4 + 5/8); low2 = q + 4 - 4 hi.  Chains (m = 7 .. 0) pack 8 elements per
+// lane: q2 bits Sum low2_m 4^m (16 bits), q1 bits Sum hi_m 2^m (8 bits).
+template <bool STAGE2, bool WANT_V, class Sink>
+__device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &k, uint32_t (&q2w)[2],
+                                          uint32_t &q1w, const Sink &sink) {
+    const float2 ns2 = splat(-k.s), M2 = splat(kMagic);
+    const float2 F4 = splat(4.f), F2 = splat(2.f), Q25 = splat(-0.25f), C58 = splat(0.625f);
+    bool bad = false;
+    uint32_t q1b[2];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        uint32_t c[4];
-        float v[4];
+    for (int p = 0; p < 2; ++p) {
+        float2 Q = splat(0.f), R = splat(0.f);
+        float2 v[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) c[j] = int_code<3, FAST, WANT_V>(x[4 * g + j], k, v[j]);
-        const uint32_t w = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
-        uint32_t lo = w & 0x03030303u;                 // low two bits of each code, one per byte
-        lo |= lo >> 6;                                 // element 4g+1 -> bits 2..3
-        lo |= lo >> 12;                                // elements 4g+2, 4g+3 -> bits 4..7
-        q2w[g >> 2] |= (lo & 0xFFu) << (8 * (g & 3));
-        const uint32_t hb = (w >> 2) & 0x01010101u;    // high bit of each code, one per byte
-        q1w |= ((hb * 0x01020408u) >> 24) << (4 * g);  // gather the 4 bits (no carries)
+        for (int m = 7; m >= 0; --m) {
+            const float2 nq = round_pair<STAGE2>(make_float2(x[16 * p + m], x[16 * p + 8 + m]), k, bad);
+            const float2 t = fma2(nq, Q25, C58);                    // q/4 + 5/8, exact
+            const float2 hi = sub2(add2(t, M2), M2);                // RNE(t) = (q >= 0)
+            const float2 u = fma2(hi, F4, nq);                      // 4 hi - q = 4 - low2
+            Q = fma2(Q, F4, u);
+            R = fma2(R, F2, hi);
+            if (WANT_V) v[m] = fma2(nq, ns2, splat(0.f));
+        }
+        const float2 P2 = sub2(splat(kMagic + 87380.0f), Q);       // 87380 = Sum_m 4 * 4^m
+        const float2 P1 = add2(R, M2);
+        q2w[p] = __byte_perm(__float_as_uint(P2.x), __float_as_uint(P2.y), 0x5410);
+        q1b[p] = __byte_perm(__float_as_uint(P1.x), __float_as_uint(P1.y), 0x0040);
         if (WANT_V) {
-            o[2 * g] = pack_bf16x2(v[0], v[1]);
-            o[2 * g + 1] = pack_bf16x2(v[2], v[3]);
+            sink.put(2 * p, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
+                                       pack_bf16x2(v[4].x, v[5].x), pack_bf16x2(v[6].x, v[7].x)));
+            sink.put(2 * p + 1, make_uint4(pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y),
+                                           pack_bf16x2(v[4].y, v[5].y), pack_bf16x2(v[6].y, v[7].y)));
         }
     }
-}
-
-// ---------------------------------------------------------------------------
-// Dequantise one block and add it to acc[32] (acc = fl32(acc + q*s); the
-// product is exact for INT codes, so one FMA rounds exactly once).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float magic_code_to_float(uint32_t bytes, int b) {
-    // byte b of `bytes` as the low mantissa bits of 2^23: value 2^23 + byte
-    return __uint_as_float(__byte_perm(bytes, 0x4B000000u, 0x7540 + b));
-}
-
-__device__ __forceinline__ void accumulate_int4(const Packed<kINT4> &p, float (&acc)[32]) {
-    const float s = __half2float(__ushort_as_half(p.scale));
-    const float off = 8388608.0f + 8.0f;                            // 2^23 + bias
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = p.w[i] & 0x0F0F0F0Fu;                   // even elements
-        const uint32_t hi = (p.w[i] >> 4) & 0x0F0F0F0Fu;            // odd elements
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float q0 = __fsub_rn(magic_code_to_float(lo, b), off);
-            const float q1 = __fsub_rn(magic_code_to_float(hi, b), off);
-            acc[8 * i + 2 * b] = __fmaf_rn(q0, s, acc[8 * i + 2 * b]);
-            acc[8 * i + 2 * b + 1] = __fmaf_rn(q1, s, acc[8 * i + 2 * b + 1]);
-        }
-    }
-}
-
-// Four INT3 codes of elements 4g..4g+3, one per byte.
-__device__ __forceinline__ uint32_t int3_codes4(const Packed<kINT3> &p, int g) {
-    const uint32_t q2 = (p.q2w[g >> 2] >> (8 * (g & 3))) & 0xFFu;     // 4 x 2 bits
-    uint32_t lo = q2 | (q2 << 6) | (q2 << 12) | (q2 << 18);           // field m -> byte m
-    lo &= 0x03030303u;
-    const uint32_t nib = (p.q1w >> (4 * g)) & 0xFu;                   // 4 x 1 bit
-    const uint32_t hi = (nib * 0x00204081u) & 0x01010101u;            // bit m -> byte m
-    return lo | (hi << 2);
-}
-
-__device__ __forceinline__ void accumulate_int3(const Packed<kINT3> &p, float (&acc)[32]) {
-    const float s = __half2float(__ushort_as_half(p.scale));
-    const float off = 8388608.0f + 4.0f;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const uint32_t c4 = int3_codes4(p, g);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float q = __fsub_rn(magic_code_to_float(c4, b), off);
-            acc[4 * g + b] = __fmaf_rn(q, s, acc[4 * g + b]);
-        }
-    }
-}
-
-// FP8: v = fl32(e4m3(code) * s), then acc = fl32(acc + v) (two roundings, no FMA).
-__device__ __forceinline__ void accumulate_fp8(const Packed<kFP8> &p, float (&acc)[32]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float e0, e1;
-            unpack_e4m3x2(p.w[i] >> (16 * h), e0, e1);
-            const int j = 4 * i + 2 * h;
-            acc[j] = __fadd_rn(acc[j], __fmul_rn(e0, p.scale));
-            acc[j + 1] = __fadd_rn(acc[j + 1], __fmul_rn(e1, p.scale));
-        }
-    }
+    q1w = __byte_perm(q1b[0], q1b[1], 0x5410);
+    return !bad;
 }
 
 // ---------------------------------------------------------------------------
@@ -283,24 +379,87 @@ __device__ __forceinline__ void accumulate_fp8(const Packed<kFP8> &p, float (&ac
 // WANT_V additionally returns the decoded result of the block as BF16 pairs
 // (the value the gathered wire decodes to), for the fused decode.
 // ---------------------------------------------------------------------------
-template <bool WANT_V>
-__device__ __forceinline__ void encode_int4(const float (&x)[32], float a, Packed<kINT4> &p, uint32_t (&o)[16]) {
-    const IntScale k = int_scale<4>(a);
-    p.scale = k.bits;
-    if (k.fast) int4_body<true, WANT_V>(x, k, p.w, o);
-    else int4_body<false, WANT_V>(x, k, p.w, o);
+// Out-of-line exact path.  It is rare (near ties at stage 2, subnormal or
+// saturated scales), so it runs one element at a time from local memory with a
+// rolled loop: few registers, so the hot path keeps a small register allocation.
+template <int BITS, bool WANT_V>
+__device__ __noinline__ void int_exact_codes(const float *x, IntScale k, uint8_t *code, float *v) {
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+        float vj = 0.f;
+        const uint32_t c = k.fast ? int_code<BITS, true, WANT_V>(x[j], k, vj) : int_code<BITS, false, WANT_V>(x[j], k, vj);
+        code[j] = (uint8_t)c;
+        if (WANT_V) v[j] = vj;
+    }
 }
 
-template <bool WANT_V>
-__device__ __forceinline__ void encode_int3(const float (&x)[32], float a, Packed<kINT3> &p, uint32_t (&o)[16]) {
-    const IntScale k = int_scale<3>(a);
-    p.scale = k.bits;
-    if (k.fast) int3_body<true, WANT_V>(x, k, p.q2w, p.q1w, o);
-    else int3_body<false, WANT_V>(x, k, p.q2w, p.q1w, o);
+template <bool WANT_V, class Sink>
+__device__ __forceinline__ void bf16_from_local(const float *v, const Sink &sink) {
+    if (WANT_V) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            sink.put(j, make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                   pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7])));
+    }
 }
 
-template <bool WANT_V>
-__device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed<kFP8> &p, uint32_t (&o)[16]) {
+__device__ __forceinline__ void pack_int4_local(const uint8_t *cs, Packed<kINT4> &p) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w |= (uint32_t)cs[8 * i + j] << (4 * j);
+        p.w[i] = w;
+    }
+}
+
+__device__ __forceinline__ void pack_int3_local(const uint8_t *cs, Packed<kINT3> &p) {
+    uint32_t q2[2] = {0u, 0u}, q1 = 0u;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        q2[j >> 4] |= ((uint32_t)cs[j] & 3u) << (2 * (j & 15));
+        q1 |= ((uint32_t)cs[j] >> 2) << j;
+    }
+    p.q2w[0] = q2[0];
+    p.q2w[1] = q2[1];
+    p.q1w = q1;
+}
+
+// Exact encoding of a block whose values are in local memory (rare path):
+// scale, codes, packing and the decoded values.
+template <int C, bool WANT_V, class Sink>
+__device__ __forceinline__ void encode_int_exact_local(const float *xs, const IntScale &k, Packed<C> &p,
+                                                       const Sink &sink) {
+    float vs[32];
+    uint8_t cs[32];
+    int_exact_codes<Layout<C>::kBits, WANT_V>(xs, k, cs, vs);
+    if constexpr (C == kINT4) pack_int4_local(cs, p);
+    else pack_int3_local(cs, p);
+    bf16_from_local<WANT_V>(vs, sink);
+}
+
+// Stage 1 (and any caller that keeps x): fast path, else copy x to local
+// memory and take the exact path.
+template <int C, bool STAGE2, bool WANT_V, class Sink>
+__device__ __forceinline__ void encode_int(const float (&x)[32], float a, Packed<C> &p, const Sink &sink) {
+    const IntScale k = int_scale<Layout<C>::kBits>(a);
+    p.scale = k.bits;
+    bool ok = k.fast;
+    if constexpr (C == kINT4) {
+        if (ok) ok = int4_fast<STAGE2, WANT_V>(x, k, p.w, sink);
+    } else {
+        if (ok) ok = int3_fast<STAGE2, WANT_V>(x, k, p.q2w, p.q1w, sink);
+    }
+    if (!ok) {
+        float xs[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) xs[j] = x[j];
+        encode_int_exact_local<C, WANT_V>(xs, k, p, sink);
+    }
+}
+
+template <bool WANT_V, class Sink>
+__device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed<kFP8> &p, const Sink &sink) {
     const float s = __fdiv_rn(a, 448.0f);
     if (!(s >= 1.17549435e-38f)) {                    // below 2^-126 (or zero): zero block
 #pragma unroll
@@ -308,56 +467,132 @@ __device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed
         p.scale = 0.f;
         if (WANT_V) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = 0u;
+            for (int j = 0; j < 4; ++j) sink.put(j, make_uint4(0u, 0u, 0u, 0u));
         }
         return;
     }
     const float inv = __frcp_rn(s);                   // fl32(1 / s)
+    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 8; ++i) {                     // scalar IEEE products (subnormals kept)
         const uint32_t lo = pack_e4m3x2(__fmul_rn(x[4 * i], inv), __fmul_rn(x[4 * i + 1], inv));
         const uint32_t hi = pack_e4m3x2(__fmul_rn(x[4 * i + 2], inv), __fmul_rn(x[4 * i + 3], inv));
         p.w[i] = lo | (hi << 16);
-        if (WANT_V) {
-            float e0, e1, e2, e3;
-            unpack_e4m3x2(lo, e0, e1);
-            unpack_e4m3x2(hi, e2, e3);
-            o[2 * i] = pack_bf16x2(__fmul_rn(e0, s), __fmul_rn(e1, s));
-            o[2 * i + 1] = pack_bf16x2(__fmul_rn(e2, s), __fmul_rn(e3, s));
+        if (WANT_V) {                                 // scalar: e * s may be subnormal
+            const uint32_t h0 = e4m3x2_to_h2(lo), h1 = e4m3x2_to_h2(hi);
+            o[2 * (i & 1)] = pack_bf16x2(__fmul_rn(h2f(h0, 0), s), __fmul_rn(h2f(h0, 1), s));
+            o[2 * (i & 1) + 1] = pack_bf16x2(__fmul_rn(h2f(h1, 0), s), __fmul_rn(h2f(h1, 1), s));
+            if (i & 1) sink.put(i >> 1, make_uint4(o[0], o[1], o[2], o[3]));
         }
     }
     p.scale = s;
 }
 
-// Decode one block to BF16 (RNE), 16 packed words (element 2k in the low half).
-// The value is q * s (one exact product), rounded once to BF16.
-__device__ __forceinline__ void decode_int4(const Packed<kINT4> &p, uint32_t (&o)[16]) {
-    const float s = __half2float(__ushort_as_half(p.scale));
-    const float off = 8388608.0f + 8.0f;
+// ---------------------------------------------------------------------------
+// Dequantisation.  INT codes become exact binary16 integers q (magic 1024 +
+// code, minus 1024 + bias), and acc = fl32(acc + q*s) is one mixed-precision
+// FMA with the binary16 scale: q*s is exact in binary32, so it rounds once,
+// exactly like the definition's acc + (float)q * s.
+// ---------------------------------------------------------------------------
+
+// INT4 word (elements 8i..8i+7) -> four packed binary16 pairs of q:
+// h[0] = (e0, e2), h[1] = (e4, e6), h[2] = (e1, e3), h[3] = (e5, e7).
+__device__ __forceinline__ void int4_word_to_h2(uint32_t w, uint32_t (&h)[4]) {
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    const uint32_t bias = 0x64086408u;                 // (1032, 1032) in binary16
+    h[0] = hsub2(__byte_perm(lo, 0x64646464u, 0x4140), bias);
+    h[1] = hsub2(__byte_perm(lo, 0x64646464u, 0x4342), bias);
+    h[2] = hsub2(__byte_perm(hi, 0x64646464u, 0x4140), bias);
+    h[3] = hsub2(__byte_perm(hi, 0x64646464u, 0x4342), bias);
+}
+
+// INT3 group g (elements 4g..4g+3) -> two packed binary16 pairs of q: (e0, e1), (e2, e3).
+__device__ __forceinline__ void int3_group_to_h2(const Packed<kINT3> &p, int g, uint32_t (&h)[2]) {
+    const uint32_t q2 = (p.q2w[g >> 2] >> (8 * (g & 3))) & 0xFFu;     // 4 x 2 bits
+    const uint32_t nib = (p.q1w >> (4 * g)) & 0xFu;                   // 4 x 1 bit
+    // low two bits: element 4g (bits 0..1) -> bits 0..1, 4g+1 (bits 2..3) -> bits 16..17
+    const uint32_t l01 = (q2 * 0x4001u) & 0x00030003u;
+    const uint32_t l23 = ((q2 >> 4) * 0x4001u) & 0x00030003u;
+    // high bit: element 4g (bit 0) -> bit 2, 4g+1 (bit 1) -> bit 18
+    const uint32_t h01 = (nib * 0x20004u) & 0x00040004u;
+    const uint32_t h23 = ((nib >> 2) * 0x20004u) & 0x00040004u;
+    const uint32_t bias = 0x64046404u;                 // (1028, 1028) in binary16
+    h[0] = hsub2(l01 | h01 | 0x64006400u, bias);
+    h[1] = hsub2(l23 | h23 | 0x64006400u, bias);
+}
+
+__device__ __forceinline__ void accumulate_int4(const Packed<kINT4> &p, float (&acc)[32]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = p.w[i] & 0x0F0F0F0Fu;
-        const uint32_t hi = (p.w[i] >> 4) & 0x0F0F0F0Fu;
+        uint32_t h[4];
+        int4_word_to_h2(p.w[i], h);
+        acc[8 * i + 0] = fma_h(h[0], 0, p.scale, acc[8 * i + 0]);
+        acc[8 * i + 2] = fma_h(h[0], 1, p.scale, acc[8 * i + 2]);
+        acc[8 * i + 4] = fma_h(h[1], 0, p.scale, acc[8 * i + 4]);
+        acc[8 * i + 6] = fma_h(h[1], 1, p.scale, acc[8 * i + 6]);
+        acc[8 * i + 1] = fma_h(h[2], 0, p.scale, acc[8 * i + 1]);
+        acc[8 * i + 3] = fma_h(h[2], 1, p.scale, acc[8 * i + 3]);
+        acc[8 * i + 5] = fma_h(h[3], 0, p.scale, acc[8 * i + 5]);
+        acc[8 * i + 7] = fma_h(h[3], 1, p.scale, acc[8 * i + 7]);
+    }
+}
+
+__device__ __forceinline__ void accumulate_int3(const Packed<kINT3> &p, float (&acc)[32]) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float q0 = __fsub_rn(magic_code_to_float(lo, b), off);
-            const float q1 = __fsub_rn(magic_code_to_float(hi, b), off);
-            o[4 * i + b] = pack_bf16x2(__fmul_rn(q0, s), __fmul_rn(q1, s));
+    for (int g = 0; g < 8; ++g) {
+        uint32_t h[2];
+        int3_group_to_h2(p, g, h);
+        acc[4 * g + 0] = fma_h(h[0], 0, p.scale, acc[4 * g + 0]);
+        acc[4 * g + 1] = fma_h(h[0], 1, p.scale, acc[4 * g + 1]);
+        acc[4 * g + 2] = fma_h(h[1], 0, p.scale, acc[4 * g + 2]);
+        acc[4 * g + 3] = fma_h(h[1], 1, p.scale, acc[4 * g + 3]);
+    }
+}
+
+// FP8: v = fl32(e4m3(code) * s), then acc = fl32(acc + v) (two roundings, no FMA).
+// Scalar IEEE operations: e * s can be subnormal (s may be as small as 2^-126),
+// and the packed f32x2 forms are not relied on for subnormal results.
+__device__ __forceinline__ void accumulate_fp8(const Packed<kFP8> &p, float (&acc)[32]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t e = e4m3x2_to_h2(p.w[i] >> (16 * h));
+            const int j = 4 * i + 2 * h;
+            acc[j] = __fadd_rn(acc[j], __fmul_rn(h2f(e, 0), p.scale));
+            acc[j + 1] = __fadd_rn(acc[j + 1], __fmul_rn(h2f(e, 1), p.scale));
         }
     }
 }
 
+// Decode one block to BF16 (RNE), 16 packed words (element 2k in the low half).
+// The value is q * s (one exact product; -0 addend keeps the product's zero sign).
+__device__ __forceinline__ void decode_int4(const Packed<kINT4> &p, uint32_t (&o)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h[4];
+        int4_word_to_h2(p.w[i], h);
+        float v[8];
+        v[0] = fma_h(h[0], 0, p.scale, -0.0f);
+        v[2] = fma_h(h[0], 1, p.scale, -0.0f);
+        v[4] = fma_h(h[1], 0, p.scale, -0.0f);
+        v[6] = fma_h(h[1], 1, p.scale, -0.0f);
+        v[1] = fma_h(h[2], 0, p.scale, -0.0f);
+        v[3] = fma_h(h[2], 1, p.scale, -0.0f);
+        v[5] = fma_h(h[3], 0, p.scale, -0.0f);
+        v[7] = fma_h(h[3], 1, p.scale, -0.0f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[4 * i + q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+    }
+}
+
 __device__ __forceinline__ void decode_int3(const Packed<kINT3> &p, uint32_t (&o)[16]) {
-    const float s = __half2float(__ushort_as_half(p.scale));
-    const float off = 8388608.0f + 4.0f;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-        const uint32_t c4 = int3_codes4(p, g);
-        float q[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) q[b] = __fsub_rn(magic_code_to_float(c4, b), off);
-        o[2 * g] = pack_bf16x2(__fmul_rn(q[0], s), __fmul_rn(q[1], s));
-        o[2 * g + 1] = pack_bf16x2(__fmul_rn(q[2], s), __fmul_rn(q[3], s));
+        uint32_t h[2];
+        int3_group_to_h2(p, g, h);
+        o[2 * g] = pack_bf16x2(fma_h(h[0], 0, p.scale, -0.0f), fma_h(h[0], 1, p.scale, -0.0f));
+        o[2 * g + 1] = pack_bf16x2(fma_h(h[1], 0, p.scale, -0.0f), fma_h(h[1], 1, p.scale, -0.0f));
     }
 }
 
@@ -366,9 +601,8 @@ __device__ __forceinline__ void decode_fp8(const Packed<kFP8> &p, uint32_t (&o)[
     for (int i = 0; i < 8; ++i) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float e0, e1;
-            unpack_e4m3x2(p.w[i] >> (16 * h), e0, e1);
-            o[2 * i + h] = pack_bf16x2(__fmul_rn(e0, p.scale), __fmul_rn(e1, p.scale));
+            const uint32_t e = e4m3x2_to_h2(p.w[i] >> (16 * h));
+            o[2 * i + h] = pack_bf16x2(__fmul_rn(h2f(e, 0), p.scale), __fmul_rn(h2f(e, 1), p.scale));
         }
     }
 }

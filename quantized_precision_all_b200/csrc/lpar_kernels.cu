@@ -81,21 +81,58 @@ __device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<k
     *reinterpret_cast<float *>(tile + Layout<kFP8>::kScaleOff + 4 * b) = p.scale;
 }
 
-template <int C, bool WANT_V>
-__device__ __forceinline__ void encode(const float (&x)[32], float a, Packed<C> &p, uint32_t (&o)[16]) {
-    if constexpr (C == kINT4) encode_int4<WANT_V>(x, a, p, o);
-    else if constexpr (C == kINT3) encode_int3<WANT_V>(x, a, p, o);
-    else encode_fp8<WANT_V>(x, a, p, o);
+// Destinations for the decoded BF16 words of a block (piece j = 16 B).
+struct NoSink {
+    __device__ __forceinline__ void put(int, uint4) const {}
+};
+struct StageSink {                                   // thread t's 64-B region of the stage
+    uint8_t *stage;
+    int t;
+    __device__ __forceinline__ void put(int j, uint4 v) const {
+        *reinterpret_cast<uint4 *>(stage + swz(t, j)) = v;
+    }
+};
+
+// Stage-2 rare path: recompute the block's FP32 sums from the N wires (same
+// arithmetic, so the same values) and requantise it exactly, one element at a
+// time.  Re-reading the wires lets the hot path drop the sums as it goes.
+template <int C, bool WANT_V, class Sink>
+__device__ __noinline__ void reduce_block_exact(const uint8_t *const *wp, int N, size_t tile, int b, Packed<C> *g,
+                                                Sink sink) {
+    constexpr int kBits = Layout<C>::kBits;
+    constexpr int kBias = 1 << (kBits - 1);
+    float acc[32];
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+#pragma unroll 1
+    for (int r = 0; r < N; ++r) {
+        const uint8_t *tb = wp[r] + tile * Layout<C>::kTileBytes;
+        const float s = __half2float(__ushort_as_half(
+            *reinterpret_cast<const uint16_t *>(tb + Layout<C>::kScaleOff + 2 * b)));
+#pragma unroll 1
+        for (int j = 0; j < 32; ++j) {
+            int code;
+            if constexpr (C == kINT4) {
+                code = (tb[16 * b + j / 2] >> (4 * (j & 1))) & 0xF;
+            } else {
+                code = ((tb[8 * b + j / 4] >> (2 * (j & 3))) & 3) |
+                       (((tb[Layout<kINT3>::kQ1wOff + 4 * b + j / 8] >> (j & 7)) & 1) << 2);
+            }
+            acc[j] = __fadd_rn(acc[j], __fmul_rn((float)(code - kBias), s));   // exact product
+        }
+    }
+    float a = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) a = fmaxf(a, fabsf(acc[j]));
+    const IntScale k = int_scale<kBits>(a);
+    g->scale = k.bits;
+    encode_int_exact_local<C, WANT_V>(acc, k, *g, sink);
 }
 
-// Pointer r of a parameter array, selected without dynamic indexing (which
-// would copy the whole array to local memory).
-template <class P>
-__device__ __forceinline__ auto pick(const P &a, int r) -> decltype(a.p[0]) {
-    auto q = a.p[0];
-#pragma unroll
-    for (int i = 1; i < kMaxRanks; ++i) q = (r == i) ? a.p[i] : q;
-    return q;
+template <int C, bool STAGE2, bool WANT_V, class Sink>
+__device__ __forceinline__ void encode(const float (&x)[32], float a, Packed<C> &p, const Sink &sink) {
+    if constexpr (C == kFP8) encode_fp8<WANT_V>(x, a, p, sink);
+    else encode_int<C, STAGE2, WANT_V>(x, a, p, sink);
 }
 
 template <int C>
@@ -146,13 +183,14 @@ __device__ __forceinline__ void stage_to_outputs(const uint8_t *stage, const Out
 // K1: stage 1 for every rank.  grid = (ceil(tiles / 4), N).
 // ---------------------------------------------------------------------------
 template <int C>
-__global__ void __launch_bounds__(kThreads) k_quantize(InPtrs in, OutPtrs wire, size_t tiles) {
+__global__ void __launch_bounds__(kThreads) k_quantize(const __grid_constant__ InPtrs in,
+                                                       const __grid_constant__ OutPtrs wire, size_t tiles) {
     __shared__ __align__(128) uint8_t stage[kStageBytes];
     const int r = blockIdx.y;
     const int t = threadIdx.x;
     const size_t tile0 = (size_t)blockIdx.x * kTilesPerCta;
     const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
-    const uint8_t *src = pick(in, r) + tile0 * (kTileElems * 2);
+    const uint8_t *src = in.p[r] + tile0 * (kTileElems * 2);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int g = t + kThreads * k;
@@ -169,9 +207,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize(InPtrs in, OutPtrs wire, 
     for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(w[k]); x[2 * k + 1] = bf16hi(w[k]); }
     const float a = absmax_bf16x32(w);
     Packed<C> p;
-    uint32_t unused[16];
-    encode<C, false>(x, a, p, unused);
-    store_block(pick(wire, r) + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
+    encode<C, false, false>(x, a, p, NoSink{});
+    store_block(wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
 }
 
 // ---------------------------------------------------------------------------
@@ -179,8 +216,9 @@ __global__ void __launch_bounds__(kThreads) k_quantize(InPtrs in, OutPtrs wire, 
 // when FUSED, the decoded BF16 result into every out[r]).
 // ---------------------------------------------------------------------------
 template <int C, int N, bool FUSED>
-__global__ void __launch_bounds__(kThreads) k_reduce(InPtrs wires, uint8_t *gather, OutPtrs out,
-                                                     size_t tile_begin, size_t tile_end) {
+__global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InPtrs wires, uint8_t *gather,
+                                                     const __grid_constant__ OutPtrs out, size_t tile_begin,
+                                                     size_t tile_end) {
     __shared__ __align__(128) uint8_t stage[FUSED ? kStageBytes : 16];
     const int t = threadIdx.x;
     const size_t tile0 = tile_begin + (size_t)blockIdx.x * kTilesPerCta;
@@ -198,10 +236,24 @@ __global__ void __launch_bounds__(kThreads) k_reduce(InPtrs wires, uint8_t *gath
         for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
         const float a = absmax_f32x32(acc);
         Packed<C> g;
-        uint32_t o[16];
-        encode<C, FUSED>(acc, a, g, o);
+        const auto sink = [&]() {
+            if constexpr (FUSED) return StageSink{stage, t};
+            else return NoSink{};
+        }();
+        if constexpr (C == kFP8) {
+            encode_fp8<FUSED>(acc, a, g, sink);
+        } else {
+            const IntScale k = int_scale<Layout<C>::kBits>(a);
+            g.scale = k.bits;
+            bool ok = k.fast;
+            if constexpr (C == kINT4) {
+                if (ok) ok = int4_fast<true, FUSED>(acc, k, g.w, sink);
+            } else {
+                if (ok) ok = int3_fast<true, FUSED>(acc, k, g.q2w, g.q1w, sink);
+            }
+            if (!ok) reduce_block_exact<C, FUSED>(wires.p, N, tile, b, &g, sink);
+        }
         store_block(gather + tile * Layout<C>::kTileBytes, b, g);
-        if (FUSED) stage_write(stage, t, o);
     }
     if (FUSED) {
         __syncthreads();

@@ -252,6 +252,76 @@ def test_reduce_exact_ties_at_stage_two(L, bits, codec):
     assert np.count_nonzero(v) > n // 2
 
 
+@pytest.mark.parametrize("N", [1, 2, 3])
+def test_fp8_subnormal_products_and_inputs(L, N):
+    # scales near 2^-126 make e4m3(code) * s subnormal; tiny elements next to a
+    # normal absmax make x * (1/s) and the FP32 sums subnormal or near it
+    rng = np.random.default_rng(77 + N)
+    n = 2048 * 3
+    xs = []
+    for r in range(N):
+        x = np.zeros((n // 32, 32), np.float32)
+        for b in range(n // 32):
+            e = rng.integers(-126, -100) if b % 2 else rng.integers(-20, 5)
+            x[b] = rng.standard_normal(32) * 2.0 ** e
+            x[b, rng.integers(32)] = 2.0 ** rng.integers(-125, -118) * rng.choice([-1, 1])
+            x[b, rng.integers(32)] = rng.choice([1e-39, -1e-39, 3e-40])
+        xs.append(bf16(x.reshape(-1)))
+    outs, _ = run_allreduce(L, xs, "fp8")
+    ref, _ = O.allreduce(xs, "fp8")
+    for o in outs:
+        assert np.array_equal(o, ref[0])
+    wire = O.quantize(xs[0], "fp8")
+    dx = to_device(xs[0])
+    dw = Guarded(wire.size)
+    L.lpar_quantize(dx.ptr(), n, "fp8", dw.ptr())
+    torch.cuda.synchronize()
+    assert np.array_equal(dw.host(), wire)
+
+
+@pytest.mark.parametrize("bits,codec", [(4, "int4"), (3, "int3")])
+@pytest.mark.parametrize("entry", ["reduce", "allreduce"])
+def test_stage_two_near_ties_take_the_exact_path(L, bits, codec, entry):
+    # ranks 0 and 1 sit on the grid S/2 (their sum's absmax is qmax * S, so the
+    # requantisation scale is S); rank 2 adds q2 * S * 2^-20.  Sums land within
+    # 2^-18 of a half-integer multiple of S without being ties, which the fast
+    # path must hand to the exact path.
+    qmax = 2 ** (bits - 1) - 1
+    rng = np.random.default_rng(50 + bits)
+    n = 2048 * 3
+    xs = [np.zeros(n, np.float32) for _ in range(3)]
+    for b in range(n // 32):
+        S = 2.0 ** rng.integers(-3, 4)
+        q0 = rng.integers(-qmax, qmax + 1, 32).astype(np.float32)
+        q1 = rng.integers(-qmax, qmax + 1, 32).astype(np.float32)
+        q0[0] = q1[0] = qmax                              # element 0: qmax S, the absmax
+        q0[1:] = np.clip(q0[1:], -qmax // 2 - 1, qmax // 2)
+        q1[1:] = np.where(np.abs(q0[1:] + q1[1:]) > qmax, 0, q1[1:])
+        q2 = rng.integers(-4, 5, 32).astype(np.float32)
+        q2[2] = qmax                                      # rank 2's own absmax
+        xs[0][b * 32:(b + 1) * 32] = q0 * S / 2
+        xs[1][b * 32:(b + 1) * 32] = q1 * S / 2
+        xs[2][b * 32:(b + 1) * 32] = q2 * S * 2.0 ** -20
+    bits16 = [bf16(x) for x in xs]
+    assert all(np.array_equal(O.bf16_bits_to_f32(b16), x) for b16, x in zip(bits16, xs))
+    if entry == "reduce":
+        wires = [O.quantize(x, codec) for x in bits16]
+        dws = []
+        for w in wires:
+            g = Guarded(w.size)
+            g.t.copy_(torch.from_numpy(w))
+            dws.append(g)
+        out = Guarded(wires[0].size)
+        L.lpar_reduce([g.ptr() for g in dws], 0, n // 2048, codec, out.ptr())
+        torch.cuda.synchronize()
+        assert np.array_equal(out.host(), O.reduce(wires, 0, n // 2048, codec))
+    else:
+        outs, _ = run_allreduce(L, bits16, codec)
+        ref, _ = O.allreduce(bits16, codec)
+        for o in outs:
+            assert np.array_equal(o, ref[0])
+
+
 def test_reduce_bf16_rounding_ties(L):
     # 1 + 2^-8 is halfway between two BF16 neighbours; 1 + 3*2^-8 likewise
     n = 2048
