@@ -44,7 +44,8 @@
  *  - All data pointers are DEVICE pointers on the current CUDA device; the
  *    pointer ARRAYS (inputs, out, wires) are HOST arrays of N device pointers.
  *  - n is the number of BF16 elements per rank and must be a multiple of
- *    LPAR_TILE_ELEMS; n == 0 is a valid no-op.  N must be in [1, LPAR_MAX_RANKS].
+ *    LPAR_TILE_ELEMS, at most 2^44; n == 0 is a valid no-op.  N must be in
+ *    [1, LPAR_MAX_RANKS].
  *  - Every data pointer must be 16-byte aligned.
  *  - The caller owns all memory.  The library allocates nothing, frees
  *    nothing, never synchronises and keeps no pointer after a call returns.

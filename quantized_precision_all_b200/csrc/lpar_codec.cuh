@@ -16,20 +16,24 @@
 // -----------------------------------------------
 // Fast path (normal, unsaturated binary16 scale, so |x/s| <= qmax(1 + 2^-11)):
 // r approximates 1/s within 2^-23 (one hardware reciprocal), so the exact
-// product x*r is within 7.01 * 2^-23 < 2^-19.9 of Q = x/s.  Two FMAs round that
-// exact product with the add-magic trick: fl(x*r + M), M = 1.5*2^23 (ulp 1),
-// gives k0 = RNE(x*r); fl(x*r + 2M) (ulp 2) gives 2*k2, the even integer
-// nearest to x*r.  With f = fl(x*r - k0):
-//   |f| <  1/2 - 2^-18  =>  |Q - k0| < 1/2, so k0 = RNE(Q) (and Q is no tie);
-//   Q an exact tie k + 1/2  =>  |f| >= 1/2 - 2^-18 and 2*k2 is the even one of
-//                               k, k+1, i.e. RNE(Q).
-// So q = (|f| >= 1/2 - 2^-18) ? 2*k2 : k0.  At stage 1 (BF16 x, 8-bit
-// significand; binary16 s, 11 bits) a non-tie quotient is at least 2^-12 from a
-// half-integer, so |f| >= 1/2 - 2^-18 only at exact ties and the fast path is
-// exact as it stands.  At stage 2 (binary32 sums) such an element is accepted
-// only when the exact residual x - k0*s (one FMA, exact) equals +-s/2;
-// otherwise the block is redone on the exact path (a near tie, rare).
-// Blocks with a subnormal, zero or saturated scale take the exact path.
+// product x*r is within 7.01 * 2^-23 < 2^-20 of Q = x/s.  Three roundings,
+// all FMAs on exact operands, give q:
+//   C2 = fl(x*r + 2M)   (M = 1.5*2^23; 2M has ulp 2): 2M + 2*k2, 2*k2 = the even
+//                        integer nearest to x*r;
+//   f2 = fl(x*r - 2*k2)  in [-1, 1];
+//   C3 = fl(f2*eta + (M + 2*k2)), eta = 1 - 2^-18 (ulp 1): M + q with
+//        q = 2*k2 + RNE(f2 * eta).
+// If Q is an exact tie m + 1/2, 2*k2 is the even one of m, m+1 and
+// |f2| <= 1/2 + 2^-20, so |f2 * eta| < 1/2 and q = 2*k2 = RNE(Q).  Otherwise q
+// is RNE(Q) unless Q lies within 2^-18 + 2^-20 of a half-integer on its odd
+// side.  At stage 1 (BF16 x, 8-bit significand; binary16 s, 11 bits) a non-tie
+// quotient is at least 1/(2S) > 2^-12 from a half-integer, so stage 1 is exact
+// as it stands.  At stage 2 (binary32 sums) each q is verified: e = x - q*s is
+// exact; a wrong q has |e| > s/2, and since e - (+-s/2) is a nonzero multiple
+// of ulp(s/2) >= (s/2) 2^-24, e^2 - (s/2)^2 > (s/2)^2 2^-23 >= ulp((s/2)^2): the
+// sign of e^2 - nextafter((s/2)^2) flags it, while an exact tie (|e| = s/2) and
+// every correct q pass.  A flagged block (rare) is redone on the exact path.  Blocks with a subnormal, zero or saturated scale take the exact
+// path.
 //
 // Exact path: k = RNE(fl(x*r) - 1/2) is RNE(x/s) or one less; the midpoint
 // m = (k + 1/2) * s is exact in binary32 ((2k+1) has <= 5 bits, s <= 11 bits),
@@ -81,7 +85,7 @@ template <> struct Packed<kFP8> { uint32_t w[8]; float scale; };              //
 
 constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23: ulp 1, bits 0x4B400000
 constexpr float kMagic2 = 25165824.0f;                // 3 * 2^23 = 1.5 * 2^24: ulp 2
-constexpr float kTieTh = 0.5f - 0x1p-18f;             // |f| >= kTieTh: tie (or, at stage 2, a near tie)
+constexpr float kEta = 1.0f - 0x1p-18f;               // shrinks exact ties below 1/2
 
 // ---------------------------------------------------------------------------
 // Small helpers
@@ -222,6 +226,7 @@ struct IntScale {
     float r;         // fl(1/s), or 0 when s == 0
     float hs;        // s/2, or +inf when s == 0 (nothing ever rounds up)
     float lim;       // (qmax + 1) * s: bound applied on the exact path
+    float t2;        // next binary32 above (s/2)^2: stage-2 verification threshold
     bool fast;       // normal, unsaturated scale: |x/s| <= qmax (1 + 2^-11), no clamp needed
 };
 
@@ -255,6 +260,8 @@ __device__ __forceinline__ IntScale int_scale(float a) {
     k.r = (k.s != 0.f) ? rcp_approx(k.s) : 0.f;
     k.hs = (k.s != 0.f) ? 0.5f * k.s : __int_as_float(0x7F800000);
     k.lim = (float)(kQmax + 1) * k.s;                                 // exact
+    const float hs2 = __fmul_rn(0.5f * k.s, 0.5f * k.s);              // exact (11-bit s)
+    k.t2 = __uint_as_float(__float_as_uint(hs2) + 1u);                // one ulp above
     return k;
 }
 
@@ -287,22 +294,30 @@ __device__ __forceinline__ uint32_t int_code(float x, const IntScale &k, float &
 // redoes the block on the exact path); outputs are only valid when true.
 // ---------------------------------------------------------------------------
 
-// One element pair -> -q (q = RNE(x/s), exact, see the header comment).
-// STAGE2: sets `bad` when a tie-like residual is not an exact tie.
+// Saturating add: clamp(a + b, 0, 1).
+__device__ __forceinline__ float add_sat(float a, float b) {
+    float d;
+    asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// One element pair -> -q (q = RNE(x/s), see the header comment).
+// STAGE2: clears bit 31 of `ok` when some q fails the exact verification.
 template <bool STAGE2>
-__device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, bool &bad) {
+__device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, uint32_t &ok) {
     const float2 r2 = splat(k.r), M2 = splat(kMagic), M4 = splat(kMagic2);
-    const float2 C = fma2(xv, r2, M2);                 // M + RNE(x r), exact product inside
-    const float2 nk = sub2(M2, C);                     // -k0
-    const float2 C2 = fma2(xv, r2, M4);                // 2M + 2 RNE(x r / 2)
+    const float2 C2 = fma2(xv, r2, M4);                // 2M + 2 k2 (exact product inside)
     const float2 nq2 = sub2(M4, C2);                   // -2 k2
-    const float2 f = fma2(xv, r2, nk);                 // x r - k0
-    const bool tx = fabsf(f.x) >= kTieTh, ty = fabsf(f.y) >= kTieTh;
+    const float2 B = sub2(C2, M2);                     // M + 2 k2
+    const float2 f2 = fma2(xv, r2, nq2);               // x r - 2 k2
+    const float2 C3 = fma2(f2, splat(kEta), B);        // M + q
+    const float2 nq = sub2(M2, C3);                    // -q (exact)
     if (STAGE2) {
-        const float2 e = fma2(nk, splat(k.s), xv);     // x - k0 s, exact
-        bad |= (tx && fabsf(e.x) != k.hs) || (ty && fabsf(e.y) != k.hs);
+        const float2 e = fma2(nq, splat(k.s), xv);     // x - q s, exact
+        const float2 d = fma2(e, e, splat(-k.t2));     // < 0 iff |e| <= s/2
+        ok &= __float_as_uint(d.x) & __float_as_uint(d.y);
     }
-    return make_float2(tx ? nq2.x : nk.x, ty ? nq2.y : nk.y);
+    return nq;
 }
 
 // INT4: lanes hold elements (8i + m, 8i + 4 + m); each lane packs 4 nibbles
@@ -313,12 +328,12 @@ template <bool STAGE2, bool WANT_V, class Sink>
 __device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &k, uint32_t (&w)[4],
                                           const Sink &sink) {
     const float2 ns2 = splat(-k.s), S16 = splat(16.f);
-    bool bad = false;
+    uint32_t ok = 0xFFFFFFFFu;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float2 nq[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) nq[m] = round_pair<STAGE2>(make_float2(x[8 * i + m], x[8 * i + 4 + m]), k, bad);
+        for (int m = 0; m < 4; ++m) nq[m] = round_pair<STAGE2>(make_float2(x[8 * i + m], x[8 * i + 4 + m]), k, ok);
         float2 Q = fma2(nq[3], S16, nq[2]);
         Q = fma2(Q, S16, nq[1]);
         Q = fma2(Q, S16, nq[0]);
@@ -332,18 +347,18 @@ __device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &
                                    pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y)));
         }
     }
-    return !bad;
+    return (ok >> 31) != 0u;
 }
 
-// INT3: lanes hold elements (16p + m, 16p + 8 + m).  hi = (q >= 0) comes from
-// RNE(q/4 + 5/8); low2 = q + 4 - 4 hi.  Chains (m = 7 .. 0) pack 8 elements per
+// INT3: lanes hold elements (16p + m, 16p + 8 + m).  hi = (q >= 0) =
+// clamp(1 + q, 0, 1) (one saturating add); low2 = q + 4 - 4 hi.  Chains (m = 7 .. 0) pack 8 elements per
 // lane: q2 bits Sum low2_m 4^m (16 bits), q1 bits Sum hi_m 2^m (8 bits).
 template <bool STAGE2, bool WANT_V, class Sink>
 __device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &k, uint32_t (&q2w)[2],
                                           uint32_t &q1w, const Sink &sink) {
     const float2 ns2 = splat(-k.s), M2 = splat(kMagic);
-    const float2 F4 = splat(4.f), F2 = splat(2.f), Q25 = splat(-0.25f), C58 = splat(0.625f);
-    bool bad = false;
+    const float2 F4 = splat(4.f), F2 = splat(2.f);
+    uint32_t ok = 0xFFFFFFFFu;
     uint32_t q1b[2];
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
@@ -351,9 +366,8 @@ __device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &
         float2 v[8];
 #pragma unroll
         for (int m = 7; m >= 0; --m) {
-            const float2 nq = round_pair<STAGE2>(make_float2(x[16 * p + m], x[16 * p + 8 + m]), k, bad);
-            const float2 t = fma2(nq, Q25, C58);                    // q/4 + 5/8, exact
-            const float2 hi = sub2(add2(t, M2), M2);                // RNE(t) = (q >= 0)
+            const float2 nq = round_pair<STAGE2>(make_float2(x[16 * p + m], x[16 * p + 8 + m]), k, ok);
+            const float2 hi = make_float2(add_sat(1.f, -nq.x), add_sat(1.f, -nq.y));   // (q >= 0)
             const float2 u = fma2(hi, F4, nq);                      // 4 hi - q = 4 - low2
             Q = fma2(Q, F4, u);
             R = fma2(R, F2, hi);
@@ -371,7 +385,7 @@ __device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &
         }
     }
     q1w = __byte_perm(q1b[0], q1b[1], 0x5410);
-    return !bad;
+    return (ok >> 31) != 0u;
 }
 
 // ---------------------------------------------------------------------------

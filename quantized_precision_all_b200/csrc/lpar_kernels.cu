@@ -4,7 +4,7 @@
 // platforms", Direct Data Access: reduce-scatter then all-gather; FP32
 // compute per its Low-Precision Collectives section; tile formats per
 // "QuickReduce INT3 Quantization and Benchmarking on MI355", Summary/Method):
-//   K1  k_quantize      BF16 -> wire, all N ranks in one launch (grid.y = rank)
+//   K1  k_quantize      BF16 -> wire, all N ranks in one persistent launch
 //   K2  k_reduce<.., false>  N wires -> FP32 sum in rank order -> requantised
 //                        gathered wire
 //   K23 k_reduce<.., true>   K2 plus the decode of the gathered block straight
@@ -22,6 +22,8 @@
 #include "lpar.h"
 #include "lpar_codec.cuh"
 
+#include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -31,6 +33,8 @@ constexpr int kThreads = 256;
 constexpr int kTilesPerCta = kThreads / kBlocksPerTile;     // 4
 constexpr int kStageBytes = kThreads * 64;                  // 16 KiB of BF16 per CTA
 constexpr int kMaxRanks = LPAR_MAX_RANKS;
+constexpr int kMaxDevices = 64;
+constexpr size_t kMaxTiles = (size_t)1 << 33;               // 2^44 elements per rank: chunk indices fit 32 bits
 
 struct InPtrs { const uint8_t *p[kMaxRanks]; };
 struct OutPtrs { uint8_t *p[kMaxRanks]; };
@@ -180,35 +184,68 @@ __device__ __forceinline__ void stage_to_outputs(const uint8_t *stage, const Out
 }
 
 // ---------------------------------------------------------------------------
-// K1: stage 1 for every rank.  grid = (ceil(tiles / 4), N).
+// K1: stage 1 for every rank.  Persistent: CTA b handles the work items
+// (chunk c, rank r) for c = b, b + gridDim.x, ... and r = 0..N-1 (a chunk is 4
+// tiles).  The BF16 chunk of the next item is copied into the other half of a
+// double-buffered stage (cp.async) while the current one is encoded.
 // ---------------------------------------------------------------------------
-template <int C>
-__global__ void __launch_bounds__(kThreads) k_quantize(const __grid_constant__ InPtrs in,
-                                                       const __grid_constant__ OutPtrs wire, size_t tiles) {
-    __shared__ __align__(128) uint8_t stage[kStageBytes];
-    const int r = blockIdx.y;
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+__device__ __forceinline__ void stage_load_chunk(uint8_t *stage, const uint8_t *src, int ntiles) {
     const int t = threadIdx.x;
-    const size_t tile0 = (size_t)blockIdx.x * kTilesPerCta;
-    const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
-    const uint8_t *src = in.p[r] + tile0 * (kTileElems * 2);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int g = t + kThreads * k;
         if (g < ntiles * 256) cp_async16(stage + swz(g >> 2, g & 3), src + 16 * (size_t)g);
     }
-    cp_async_wait_all();
-    __syncthreads();
-    if (t >= ntiles * kBlocksPerTile) return;
+}
 
-    uint32_t w[16];
-    stage_read(stage, t, w);
-    float x[32];
+template <int C>
+__global__ void __launch_bounds__(kThreads, 5) k_quantize(const __grid_constant__ InPtrs in,
+                                                       const __grid_constant__ OutPtrs wire, size_t tiles,
+                                                       unsigned chunks, int N) {
+    __shared__ __align__(128) uint8_t stage[2][kStageBytes];
+    const int t = threadIdx.x;
+    // work item = (chunk c, rank r); a CTA walks r = 0..N-1, then c += gridDim.x
+    unsigned c = blockIdx.x;
+    int r = 0;
+    if (c < chunks) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        stage_load_chunk(stage[0], in.p[0] + tile0 * (kTileElems * 2), (int)min((size_t)kTilesPerCta, tiles - tile0));
+    }
+    cp_async_commit();
+    int buf = 0;
+    while (c < chunks) {
+        unsigned cn = c;
+        int rn = r + 1;
+        if (rn == N) { rn = 0; cn += gridDim.x; }
+        if (cn < chunks) {
+            const size_t tn = (size_t)cn * kTilesPerCta;
+            stage_load_chunk(stage[buf ^ 1], in.p[rn] + tn * (kTileElems * 2),
+                             (int)min((size_t)kTilesPerCta, tiles - tn));
+        }
+        cp_async_commit();
+        cp_async_wait_prev();                          // this item's copies have landed
+        __syncthreads();
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+        if (t < ntiles * kBlocksPerTile) {
+            uint32_t x16[16];
+            stage_read(stage[buf], t, x16);
+            float x[32];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(w[k]); x[2 * k + 1] = bf16hi(w[k]); }
-    const float a = absmax_bf16x32(w);
-    Packed<C> p;
-    encode<C, false, false>(x, a, p, NoSink{});
-    store_block(wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
+            for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
+            const float a = absmax_bf16x32(x16);
+            Packed<C> p;
+            encode<C, false, false>(x, a, p, NoSink{});
+            store_block(wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t % kBlocksPerTile, p);
+        }
+        __syncthreads();                               // stage[buf] is refilled next iteration
+        buf ^= 1;
+        c = cn;
+        r = rn;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -327,12 +364,38 @@ __global__ void __launch_bounds__(kThreads) k_broadcast(const uint8_t *src, OutP
 // ---------------------------------------------------------------------------
 static inline unsigned grid_for_tiles(size_t tiles) { return (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta); }
 
+// Resident CTAs of a kernel on the current device (SM count x occupancy), cached
+// per device and kernel; 0 when the query fails.
+template <class K>
+static unsigned resident_ctas(K kernel) {
+    static std::atomic<unsigned> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    unsigned v = cache[dev].load(std::memory_order_relaxed);
+    if (v) return v;
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess) return 0;
+    v = (unsigned)(sms * (per_sm > 0 ? per_sm : 1));
+    cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+template <int C>
+static void launch_quantize_c(const InPtrs &in, const OutPtrs &wire, int N, size_t tiles, cudaStream_t st) {
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned res = resident_ctas(k_quantize<C>);
+    // every CTA walks all N ranks of its chunks: size the grid in chunks
+    const unsigned per_rank = (res ? res : 148u * 4u);
+    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, per_rank));
+    k_quantize<C><<<grid, kThreads, 0, st>>>(in, wire, tiles, chunks, N);
+}
+
 static void launch_quantize(int codec, const InPtrs &in, const OutPtrs &wire, int N, size_t tiles, cudaStream_t st) {
-    const dim3 grid(grid_for_tiles(tiles), N);
     switch (codec) {
-    case kINT4: k_quantize<kINT4><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
-    case kINT3: k_quantize<kINT3><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
-    case kFP8: k_quantize<kFP8><<<grid, kThreads, 0, st>>>(in, wire, tiles); break;
+    case kINT4: launch_quantize_c<kINT4>(in, wire, N, tiles, st); break;
+    case kINT3: launch_quantize_c<kINT3>(in, wire, N, tiles, st); break;
+    case kFP8: launch_quantize_c<kFP8>(in, wire, N, tiles, st); break;
     default: break;
     }
 }
@@ -452,7 +515,7 @@ LPAR_API const char *lpar_status_string(lpar_status_t s) {
 LPAR_API lpar_status_t lpar_quantize(const void *in_bf16, size_t n, lpar_codec_t codec, void *wire,
                                      cudaStream_t stream) {
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
-    if (n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
     if (!in_bf16 || !wire) return LPAR_ERR_INVALID_ARG;
     if (!aligned16(in_bf16) || !aligned16(wire)) return LPAR_ERR_MISALIGNED;
@@ -473,7 +536,7 @@ LPAR_API lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_
                                    lpar_codec_t codec, void *wire_out, cudaStream_t stream) {
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     if (N < 1 || N > kMaxRanks || !wires) return LPAR_ERR_INVALID_ARG;
-    if (tile_begin + tile_count < tile_begin) return LPAR_ERR_INVALID_ARG;
+    if (tile_begin + tile_count < tile_begin || tile_count > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (tile_count == 0) return LPAR_OK;
     if (!wire_out) return LPAR_ERR_INVALID_ARG;
     InPtrs w{};
@@ -498,7 +561,7 @@ LPAR_API lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_
 LPAR_API lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec, void *out_bf16,
                                    cudaStream_t stream) {
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
-    if (n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
     if (!wire || !out_bf16) return LPAR_ERR_INVALID_ARG;
     if (!aligned16(wire) || !aligned16(out_bf16)) return LPAR_ERR_MISALIGNED;
@@ -515,7 +578,7 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     const int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_FUSED;
     if (schedule != LPAR_SCHEDULE_FUSED && schedule != LPAR_SCHEDULE_THREE_STAGE) return LPAR_ERR_UNSUPPORTED;
-    if (N < 1 || N > kMaxRanks || n % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (N < 1 || N > kMaxRanks || n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
     if (!inputs || !out || !workspace) return LPAR_ERR_INVALID_ARG;
     InPtrs in{};

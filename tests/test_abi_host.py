@@ -95,6 +95,7 @@ def test_argument_errors_quantize(L):
     assert status_of(L.lpar_quantize, M, 2048, "int4", A, st) == 2       # misaligned
     assert status_of(L.lpar_quantize, A, 2048, "int3", M, st) == 2
     assert status_of(L.lpar_quantize, 0, 0, "int4", 0, st) == 0          # empty message: no-op
+    assert status_of(L.lpar_quantize, A, 2048 * (2 ** 33 + 1), "int4", A, st) == 1   # beyond 2^44
 
 
 def test_argument_errors_reduce_decode(L):
