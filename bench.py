@@ -105,6 +105,21 @@ def traffic_for(kernel, workload):
     return None
 
 
+# ---- multi-rank aggregation (one process per GPU) -----------------------------------
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank contributes, all receive the max."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(world, bytes_per_rank_step, steps, ms_max):
+    """Whole-job throughput: the bytes of every rank over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
+
+
 # ---- clocks sampled during the timed region -------------------------------------
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -196,12 +211,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
-    ms = start.elapsed_time(end)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end), world, device)
 
     # (2) per-kernel durations, live: stage events recorded between the kernels
     ksteps = max(1, min(args.steps, 200))
@@ -258,13 +268,8 @@ def run_ours(args, rank, world, device):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        bytes_e2e = world * N * 2 * n * len(w.codecs) * e2e_steps
-        e2e = {"value": bytes_e2e / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e_ms = max_over_ranks(s0.elapsed_time(s1), world, device)
+        e2e = {"value": aggregate_gbs(world, N * 2 * n * len(w.codecs), e2e_steps, e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": N * 2 * n, "d2h_bytes_per_step": N * 2 * n * len(w.codecs),
                "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
                "api": "lpar_allreduce with pinned host buffers copied in and out on the same stream"}
@@ -364,7 +369,7 @@ def main():
         peak, peak_src = measured_peaks()
         step_bytes = w.N * 2 * w.n * len(w.codecs)
         ms_per_step = res["ms"] / args.steps
-        value = world * step_bytes * args.steps / (res["ms"] * 1e-3) / 1e9
+        value = aggregate_gbs(world, step_bytes, args.steps, res["ms"])
         kern = res["kern"]
         dom = max(kern, key=lambda k: kern[k]["ms_total"])
         total_ms = sum(d["ms_total"] for d in kern.values())
