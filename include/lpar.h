@@ -146,6 +146,25 @@ lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_co
                              void *const *out, void *workspace, size_t workspace_bytes,
                              const lpar_options_t *opts, cudaStream_t stream);
 
+/* Size of the workspace that lpar_allreduce_static keeps inside the library. */
+#define LPAR_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+
+/* lpar_allreduce without a caller-provided workspace, for callers that cannot
+ * allocate device memory (for example a plugin whose host application owns all
+ * device memory, or a loop held to a fixed memory budget).  The pages have no
+ * counterpart: this is a deployment convenience, not part of the method.
+ * Inputs, outputs, options and stream are as for lpar_allreduce; the workspace
+ * is a 16 MiB array reserved inside the library on every device that loads it
+ * and held until the process exits.  Returns LPAR_ERR_WORKSPACE_TOO_SMALL when
+ * lpar_workspace_bytes(N, n, effective codec) exceeds
+ * LPAR_STATIC_WORKSPACE_BYTES (e.g. INT3 with N = 2 up to n = 12.8 Mi), and
+ * never calls cudaMalloc/cudaFree.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it: make that call
+ * before any stream capture.  All calls share the one array: calls whose work
+ * overlaps on the GPU race on it and must be serialised by the caller. */
+lpar_status_t lpar_allreduce_static(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                                    void *const *out, const lpar_options_t *opts, cudaStream_t stream);
+
 /* The codec lpar_allreduce runs for these arguments after the threshold. */
 lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts);
 

@@ -1,0 +1,58 @@
+// lpar_static_ws.cu -- lpar_allreduce_static: the all-reduce with a workspace
+// that lives inside the library, for callers that cannot allocate device
+// memory themselves.
+//
+// Who needs it: code that runs where device allocation is not available or not
+// allowed -- for example a plugin or extension whose host application owns all
+// device memory and exposes no allocator to it, or a serving loop that runs
+// under a fixed memory budget and must not grow its footprint (or pay for an
+// allocation) on the communication path.  Such callers still own and pass
+// their input and output buffers; only the scratch space is provided here.
+//
+// The scratch is one file-scope __device__ array of LPAR_STATIC_WORKSPACE_BYTES.
+// Every GPU on which the library's code is loaded holds it until the process
+// exits.  Host code cannot use the array's name as a device address, so the
+// first call on each device looks the address up with cudaGetSymbolAddress
+// (with that device current) and caches it; make that first call before any
+// stream capture.  All calls share the array and it keeps the last call's
+// contents: nothing in it needs to start at zero (every byte the all-reduce
+// reads there it has written first in the same call), but calls whose work
+// overlaps on the GPU -- on different streams, or on different host threads
+// without ordering -- race on it and must be serialised by the caller.
+#include "lpar.h"
+
+#include <atomic>
+#include <cuda_runtime.h>
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_workspace[LPAR_STATIC_WORKSPACE_BYTES];
+
+// Device address of g_static_workspace on the current device (cached per device).
+lpar_status_t static_workspace(void **ptr) {
+    static std::atomic<void *> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LPAR_ERR_CUDA;
+    void *p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return LPAR_ERR_CUDA;
+        cache[dev].store(p, std::memory_order_release);
+    }
+    *ptr = p;
+    return LPAR_OK;
+}
+
+}  // namespace
+
+extern "C" __attribute__((visibility("default"))) lpar_status_t
+lpar_allreduce_static(const void *const *inputs, int N, size_t n, lpar_codec_t codec, void *const *out,
+                      const lpar_options_t *opts, cudaStream_t stream) {
+    const size_t need = lpar_workspace_bytes(N, n, lpar_effective_codec(n, codec, opts));
+    if (need > LPAR_STATIC_WORKSPACE_BYTES) return LPAR_ERR_WORKSPACE_TOO_SMALL;
+    void *ws = nullptr;
+    const lpar_status_t st = static_workspace(&ws);
+    if (st != LPAR_OK) return st;
+    return lpar_allreduce(inputs, N, n, codec, out, ws, LPAR_STATIC_WORKSPACE_BYTES, opts, stream);
+}

@@ -27,7 +27,8 @@ TILE_ELEMS = 2048
 MAX_RANKS = 8
 
 EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
-           "lpar_decode", "lpar_allreduce", "lpar_effective_codec", "lpar_status_string")
+           "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string")
+LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 class LparError(RuntimeError):
@@ -53,6 +54,7 @@ def _load():
         "lpar_reduce": (i32, [vpp, i32, sz, sz, i32, vp, vp]),
         "lpar_decode": (i32, [vp, sz, i32, vp, vp]),
         "lpar_allreduce": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_allreduce_static": (i32, [vpp, i32, sz, i32, vpp, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_effective_codec": (i32, [sz, i32, ctypes.POINTER(lpar_options_t)]),
         "lpar_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -159,6 +161,16 @@ def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_
     _check(_lib.lpar_allreduce(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
                                _ptr(workspace), workspace_bytes, ctypes.byref(opts), _stream(stream)),
            "lpar_allreduce")
+
+
+def lpar_allreduce_static(inputs, n, codec, out, min_quant_bytes=0, schedule="fused", stream=None, N=None):
+    """lpar_allreduce with the library's own 16 MiB workspace (no allocation)."""
+    ins = _ptr_array(inputs)
+    outs = _ptr_array(out)
+    N = len(inputs) if N is None else N
+    opts = _options(min_quant_bytes, schedule)
+    _check(_lib.lpar_allreduce_static(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+                                      ctypes.byref(opts), _stream(stream)), "lpar_allreduce_static")
 
 
 def lpar_status_string(status):

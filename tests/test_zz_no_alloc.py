@@ -1,0 +1,52 @@
+"""lpar_allreduce_static: the all-reduce for callers that cannot allocate device
+memory (for example a plugin whose host application owns all device memory),
+using the workspace the library keeps for itself.
+
+Its results must equal those of lpar_allreduce with a caller-provided workspace,
+on two calls in a row (the shared workspace keeps the previous call's contents).
+This file is named to be collected last, and must pass both alone in a fresh
+process and after the other tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_precision_all_b200 import build
+    build.build()
+    from quantized_precision_all_b200 import lpar
+    return lpar
+
+
+@pytest.mark.parametrize("codec,N", [("int3", 2), ("int4", 2), ("fp8", 8), ("bf16", 3)])
+def test_static_workspace_equals_caller_workspace_on_two_calls(L, codec, N):
+    n = 2048 * 37
+    g = torch.Generator(device="cuda").manual_seed(900 + N)
+    ref_out = None
+    for call in range(2):
+        xs = [(torch.randn(n, generator=g, device="cuda") * 10.0 ** (r - 1)).to(torch.bfloat16) for r in range(N)]
+        ws = torch.empty(L.lpar_workspace_bytes(N, n, codec), dtype=torch.uint8, device="cuda")
+        ref_out = [torch.empty_like(x) for x in xs]
+        L.lpar_allreduce(xs, n, codec, ref_out, ws, ws.numel())
+        out = [torch.full_like(x, float("nan")) for x in xs]
+        L.lpar_allreduce_static(xs, n, codec, out)
+        torch.cuda.synchronize()
+        for o, r in zip(out, ref_out):
+            assert torch.equal(o.view(torch.int16), r.view(torch.int16)), (codec, call)
+
+
+def test_static_workspace_rejects_messages_beyond_its_size(L):
+    n = 2048 * 4096                                   # INT3, N = 2: 3 * 3.5 MiB fits
+    xs = [torch.zeros(n, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    out = [torch.empty_like(x) for x in xs]
+    L.lpar_allreduce_static(xs, n, "int3", out)
+    big = L.LPAR_STATIC_WORKSPACE_BYTES // 2 + 2048    # BF16 needs 2n bytes > the array
+    ys = [torch.zeros(big - big % 2048 + 2048, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    with pytest.raises(L.LparError) as e:
+        L.lpar_allreduce_static(ys, ys[0].numel(), "bf16", [torch.empty_like(y) for y in ys])
+    assert e.value.status == 3
+    torch.cuda.synchronize()
