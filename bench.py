@@ -326,6 +326,47 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_sweep(args, device):
+    """One JSON line per sweep point (N, message size, codec): GB/s and the
+    fraction of measured HBM peak the whole call reaches (its algorithmic
+    bytes over its time)."""
+    from quantized_precision_all_b200 import lpar as L
+    peak, peak_src = measured_peaks()
+    stream = torch.cuda.current_stream(device)
+    for N in W.SWEEP_RANKS:
+        for mb in W.SWEEP_SIZES_BYTES:
+            w = W.sweep_workload(N, mb, "bf16")
+            xs = W.make_inputs(w, device)
+            outs = [torch.empty_like(x) for x in xs]
+            wsb = max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=device)
+            flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # > L2, rewritten between calls
+            for codec in W.SWEEP_CODECS:
+                iters = max(3, min(50, int(2e9 / (N * mb))))
+                for _ in range(3):
+                    L.lpar_allreduce(xs, w.n, codec, outs, ws, wsb, schedule=args.schedule, stream=stream)
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(iters)]
+                for e0, e1 in evs:
+                    flush.fill_(1)
+                    e0.record(stream)
+                    L.lpar_allreduce(xs, w.n, codec, outs, ws, wsb, schedule=args.schedule, stream=stream)
+                    e1.record(stream)
+                torch.cuda.synchronize(device)
+                ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+                names = kernel_names(codec, args.schedule, N)
+                alg = sum(algorithmic_bytes(k, codec, N, w.n) for k in names)
+                print(json.dumps({"sweep": True, "N": N, "message_bytes": mb, "codec": codec,
+                                  "schedule": args.schedule, "ms": ms,
+                                  "GBps": N * mb / (ms * 1e-3) / 1e9,
+                                  "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
+                                  "l2": "256 MiB buffer rewritten before every timed call",
+                                  "note": "L2-resident / launch-bound" if N * mb < (16 << 20) else "",
+                                  "peak": peak}), flush=True)
+            del xs, outs, ws, flush
+            torch.cuda.empty_cache()
+
+
 def workload_config(w, args):
     return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n,
             "message_bytes_per_rank": 2 * w.n, "codecs": list(w.codecs), "schedule": args.schedule,
@@ -345,6 +386,7 @@ def main():
     ap.add_argument("--schedule", default="fused", choices=["fused", "three_stage"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -359,6 +401,9 @@ def main():
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    if args.sweep:
+        run_sweep(args, device)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

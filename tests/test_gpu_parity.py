@@ -468,3 +468,36 @@ def test_workload_large_sampled_tiles(L):
             assert np.array_equal(got, ref[0])
         del outs, ws
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# The sweep: 128 KiB ... 1 GiB per rank, N in {2, 4, 8}, every codec, Student-t
+# (nu = 3).  Each point runs at full size on the GPU; the oracle checks the
+# first and last tile plus 62 seeded random tiles (a tile's result depends only
+# on that tile of every rank).  Points up to 1 MiB are checked in full.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N", list(W.SWEEP_RANKS))
+def test_sweep_sampled_tiles(L, N):
+    rng = np.random.default_rng(5000 + N)
+    for mb in W.SWEEP_SIZES_BYTES:
+        w = W.sweep_workload(N, mb, "bf16")
+        xs = W.make_inputs(w, "cuda")
+        T = w.n // 2048
+        if mb <= (1 << 20):
+            tiles = np.arange(T)
+        else:
+            tiles = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 62, replace=False)]))
+        idx = torch.from_numpy((tiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
+        sample_in = [x[idx].view(torch.int16).cpu().numpy().view(np.uint16) for x in xs]
+        outs = [torch.empty_like(x) for x in xs]
+        ws = torch.empty(max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS), dtype=torch.uint8,
+                         device="cuda")
+        for codec in W.SWEEP_CODECS:
+            L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel())
+            torch.cuda.synchronize()
+            ref, _ = O.allreduce(sample_in, codec)
+            got = [o[idx].view(torch.int16).cpu().numpy().view(np.uint16) for o in outs]
+            for g in got:
+                assert np.array_equal(g, ref[0]), (N, mb, codec)
+        del xs, outs, ws
+        torch.cuda.empty_cache()
