@@ -520,19 +520,40 @@ __device__ __forceinline__ void int4_word_to_h2(uint32_t w, uint32_t (&h)[4]) {
     h[3] = hsub2(__byte_perm(hi, 0x64646464u, 0x4342), bias);
 }
 
-// INT3 group g (elements 4g..4g+3) -> two packed binary16 pairs of q: (e0, e1), (e2, e3).
-__device__ __forceinline__ void int3_group_to_h2(const Packed<kINT3> &p, int g, uint32_t (&h)[2]) {
-    const uint32_t q2 = (p.q2w[g >> 2] >> (8 * (g & 3))) & 0xFFu;     // 4 x 2 bits
-    const uint32_t nib = (p.q1w >> (4 * g)) & 0xFu;                   // 4 x 1 bit
-    // low two bits: element 4g (bits 0..1) -> bits 0..1, 4g+1 (bits 2..3) -> bits 16..17
-    const uint32_t l01 = (q2 * 0x4001u) & 0x00030003u;
-    const uint32_t l23 = ((q2 >> 4) * 0x4001u) & 0x00030003u;
-    // high bit: element 4g (bit 0) -> bit 2, 4g+1 (bit 1) -> bit 18
-    const uint32_t h01 = (nib * 0x20004u) & 0x00040004u;
-    const uint32_t h23 = ((nib >> 2) * 0x20004u) & 0x00040004u;
-    const uint32_t bias = 0x64046404u;                 // (1028, 1028) in binary16
-    h[0] = hsub2(l01 | h01 | 0x64006400u, bias);
-    h[1] = hsub2(l23 | h23 | 0x64006400u, bias);
+// INT3 half-block (elements 16*half .. 16*half+15) -> eight packed binary16
+// pairs of q.  Codes are assembled one per nibble: the low two bits of the
+// even (odd) elements are q2w & 0x33333333 ((q2w >> 2) & 0x33333333), and the
+// q1w bits of the same elements are deposited at bit 2 of each nibble.  A
+// nibble code c (0..7) then indexes an 8-byte table with one PRMT: the binary16
+// value of q = c - 4 is -4, -3, ..., 3, whose low byte is always 0, so the
+// table holds only the high bytes and two more PRMTs interleave zero bytes.
+// h[0..3] = (e0,e2) (e4,e6) (e8,e10) (e12,e14); h[4..7] = (e1,e3) (e5,e7)
+// (e9,e11) (e13,e15), indices relative to 16*half.
+__device__ __forceinline__ uint32_t deposit_even_bits(uint32_t x) {   // bit 2k of x (k < 8) -> bit 4k+2
+    uint32_t t = x & 0x5555u;
+    t = (t | (t << 8)) & 0x00550055u;
+    t = (t | (t << 4)) & 0x05050505u;
+    t = (t | (t << 2)) & 0x11111111u;
+    return t << 2;
+}
+
+__device__ __forceinline__ void int3_half_to_h2(const Packed<kINT3> &p, int half, uint32_t (&h)[8]) {
+    const uint32_t w = p.q2w[half];
+    const uint32_t q1 = p.q1w >> (16 * half);
+    const uint32_t ce = (w & 0x33333333u) | deposit_even_bits(q1);          // even elements
+    const uint32_t co = ((w >> 2) & 0x33333333u) | deposit_even_bits(q1 >> 1);   // odd elements
+    const uint32_t T0 = 0xBCC0C2C4u;       // high bytes of -1, -2, -3, -4 (codes 3..0)
+    const uint32_t T1 = 0x42403C00u;       // high bytes of  3,  2,  1,  0 (codes 7..4)
+    const uint32_t e0 = __byte_perm(T0, T1, ce), e1 = __byte_perm(T0, T1, ce >> 16);
+    const uint32_t o0 = __byte_perm(T0, T1, co), o1 = __byte_perm(T0, T1, co >> 16);
+    h[0] = __byte_perm(e0, 0u, 0x1404);
+    h[1] = __byte_perm(e0, 0u, 0x3424);
+    h[2] = __byte_perm(e1, 0u, 0x1404);
+    h[3] = __byte_perm(e1, 0u, 0x3424);
+    h[4] = __byte_perm(o0, 0u, 0x1404);
+    h[5] = __byte_perm(o0, 0u, 0x3424);
+    h[6] = __byte_perm(o1, 0u, 0x1404);
+    h[7] = __byte_perm(o1, 0u, 0x3424);
 }
 
 __device__ __forceinline__ void accumulate_int4(const Packed<kINT4> &p, float (&acc)[32]) {
@@ -553,13 +574,17 @@ __device__ __forceinline__ void accumulate_int4(const Packed<kINT4> &p, float (&
 
 __device__ __forceinline__ void accumulate_int3(const Packed<kINT3> &p, float (&acc)[32]) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        uint32_t h[2];
-        int3_group_to_h2(p, g, h);
-        acc[4 * g + 0] = fma_h(h[0], 0, p.scale, acc[4 * g + 0]);
-        acc[4 * g + 1] = fma_h(h[0], 1, p.scale, acc[4 * g + 1]);
-        acc[4 * g + 2] = fma_h(h[1], 0, p.scale, acc[4 * g + 2]);
-        acc[4 * g + 3] = fma_h(h[1], 1, p.scale, acc[4 * g + 3]);
+    for (int half = 0; half < 2; ++half) {
+        uint32_t h[8];
+        int3_half_to_h2(p, half, h);
+        float *a = acc + 16 * half;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            a[4 * g + 0] = fma_h(h[g], 0, p.scale, a[4 * g + 0]);
+            a[4 * g + 2] = fma_h(h[g], 1, p.scale, a[4 * g + 2]);
+            a[4 * g + 1] = fma_h(h[4 + g], 0, p.scale, a[4 * g + 1]);
+            a[4 * g + 3] = fma_h(h[4 + g], 1, p.scale, a[4 * g + 3]);
+        }
     }
 }
 
@@ -602,11 +627,14 @@ __device__ __forceinline__ void decode_int4(const Packed<kINT4> &p, uint32_t (&o
 
 __device__ __forceinline__ void decode_int3(const Packed<kINT3> &p, uint32_t (&o)[16]) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        uint32_t h[2];
-        int3_group_to_h2(p, g, h);
-        o[2 * g] = pack_bf16x2(fma_h(h[0], 0, p.scale, -0.0f), fma_h(h[0], 1, p.scale, -0.0f));
-        o[2 * g + 1] = pack_bf16x2(fma_h(h[1], 0, p.scale, -0.0f), fma_h(h[1], 1, p.scale, -0.0f));
+    for (int half = 0; half < 2; ++half) {
+        uint32_t h[8];
+        int3_half_to_h2(p, half, h);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            o[8 * half + 2 * g] = pack_bf16x2(fma_h(h[g], 0, p.scale, -0.0f), fma_h(h[4 + g], 0, p.scale, -0.0f));
+            o[8 * half + 2 * g + 1] = pack_bf16x2(fma_h(h[g], 1, p.scale, -0.0f), fma_h(h[4 + g], 1, p.scale, -0.0f));
+        }
     }
 }
 
