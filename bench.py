@@ -66,8 +66,10 @@ def measured_peaks():
 # ---- algorithmic bytes per launch (reads + writes the definition requires) ------
 def kernel_names(codec, schedule, N):
     if codec == "bf16":
-        return ["k_bf16_reduce<N=%d,fused>" % N] if schedule == "fused" else \
+        return ["k_bf16_reduce<N=%d,fused>" % N] if schedule != "three_stage" else \
             ["k_bf16_reduce<N=%d>" % N, "k_broadcast"]
+    if schedule == "single_pass":
+        return ["k_allreduce_single<%s,N=%d>" % (codec, N)]
     if schedule == "fused":
         return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d,fused>" % (codec, N)]
     return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d>" % (codec, N), "k_decode<%s>" % codec]
@@ -75,6 +77,9 @@ def kernel_names(codec, schedule, N):
 
 def algorithmic_bytes(kernel, codec, N, n):
     c = CODEC_C[codec]
+    if kernel.startswith("k_allreduce_single"):
+        # N BF16 messages in, N wires out and back in, gathered wire out, N outputs out
+        return N * n * (2 + c) + n * (N * c + c + 2 * N)
     if kernel.startswith("k_quantize"):
         return N * n * (2 + c)                        # read N BF16 messages, write N wires
     if kernel.startswith("k_reduce") and kernel.endswith("fused>"):
@@ -228,7 +233,12 @@ def run_ours(args, rank, world, device):
     for ci, codec in enumerate(w.codecs):
         eff = L.lpar_effective_codec(n, codec, w.min_quant_bytes)
         names = kernel_names(eff, args.schedule, N)
-        bounds = [(0, 1), (1, 2), (2, 3)] if eff != "bf16" else [(1, 2), (2, 3)]
+        if eff == "bf16":
+            bounds = [(1, 2), (2, 3)]
+        elif args.schedule == "single_pass":
+            bounds = [(0, 1)]
+        else:
+            bounds = [(0, 1), (1, 2), (2, 3)]
         for name, (a, b) in zip(names, bounds):
             tot = sum(evs[s][ci][a].elapsed_time(evs[s][ci][b]) for s in range(ksteps))
             d = kern.setdefault(name, {"codec": eff, "ms_total": 0.0, "launches": 0})
@@ -383,12 +393,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_int3_int4", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--schedule", default="fused", choices=["fused", "three_stage"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_stage", "single_pass"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.schedule == "auto":                # what the library picks for LPAR_SCHEDULE_AUTO
+        args.schedule = "single_pass"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

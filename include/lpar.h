@@ -88,8 +88,12 @@ typedef enum {
 } lpar_status_t;
 
 typedef enum {
-    LPAR_SCHEDULE_FUSED = 0,       /* quantise; reduce + requantise + decode in one kernel */
-    LPAR_SCHEDULE_THREE_STAGE = 1  /* quantise; reduce + requantise; decode (three kernels) */
+    LPAR_SCHEDULE_AUTO = 0,        /* the library's choice (currently LPAR_SCHEDULE_SINGLE_PASS) */
+    LPAR_SCHEDULE_FUSED = 1,       /* quantise; reduce + requantise + decode in one kernel */
+    LPAR_SCHEDULE_THREE_STAGE = 2, /* quantise; reduce + requantise; decode (three kernels) */
+    LPAR_SCHEDULE_SINGLE_PASS = 3  /* one kernel: each CTA quantises a chunk of every rank, then
+                                      reduces, requantises and decodes that chunk from the wires
+                                      it has just written (same results, one launch) */
 } lpar_schedule_t;
 
 typedef struct {
@@ -97,12 +101,14 @@ typedef struct {
      * least this many bytes; smaller messages take the BF16 passthrough.
      * 0 = always quantise.  The INT3 page recommends 1 MB (1 << 20). */
     size_t min_quant_bytes;
-    lpar_schedule_t schedule;      /* 0 (LPAR_SCHEDULE_FUSED) is the default */
+    lpar_schedule_t schedule;      /* 0 (LPAR_SCHEDULE_AUTO) is the default */
     /* Optional tracing: events recorded on `stream` at the stage boundaries --
      * [0] before stage 1, [1] after stage 1, [2] after stage 2 (after the
      * fused reduce+decode in the fused schedule), [3] after stage 3 (three-
-     * stage schedule only).  NULL entries are skipped.  The BF16 passthrough
-     * has no stage 1: [0] and [1] are recorded back to back. */
+     * stage schedule only).  The single-pass schedule records [0] before and
+     * [1] after its one kernel.  NULL entries are skipped.  The BF16
+     * passthrough has no stage 1: [0] and [1] are recorded back to back, then
+     * [2] after its (fused, or single-pass) kernel. */
     cudaEvent_t stage_events[4];
 } lpar_options_t;
 
@@ -141,7 +147,8 @@ lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec,
  * (in place); out buffers must not overlap each other or the workspace.
  * workspace: device memory of at least lpar_workspace_bytes(N, n, effective
  * codec) bytes, 16-byte aligned, contents ignored and overwritten.
- * opts may be NULL (always quantise, fused schedule). */
+ * opts may be NULL (always quantise, LPAR_SCHEDULE_AUTO).  Every schedule
+ * gives the same bits. */
 lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                              void *const *out, void *workspace, size_t workspace_bytes,
                              const lpar_options_t *opts, cudaStream_t stream);

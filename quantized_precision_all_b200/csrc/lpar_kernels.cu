@@ -252,6 +252,37 @@ __global__ void __launch_bounds__(kThreads, 5) k_quantize(const __grid_constant_
 // K2 / K23: tiles [tile_begin, tile_end) of N wires -> gathered wire (and,
 // when FUSED, the decoded BF16 result into every out[r]).
 // ---------------------------------------------------------------------------
+// Stage 2 for one block: thread-owned block b of `tile`, N wires -> gathered
+// wire (and the decoded BF16 words into `sink`).
+template <int C, int N, bool WANT_V, class Sink>
+__device__ __forceinline__ void reduce_block(const uint8_t *const *wp, size_t tile, int b, uint8_t *gather,
+                                             const Sink &sink) {
+    Packed<C> p[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) load_block(wp[r] + tile * Layout<C>::kTileBytes, b, p[r]);
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;          // +0.0f, then ranks in ascending order
+#pragma unroll
+    for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
+    const float a = absmax_f32x32(acc);
+    Packed<C> g;
+    if constexpr (C == kFP8) {
+        encode_fp8<WANT_V>(acc, a, g, sink);
+    } else {
+        const IntScale k = int_scale<Layout<C>::kBits>(a);
+        g.scale = k.bits;
+        bool ok = k.fast;
+        if constexpr (C == kINT4) {
+            if (ok) ok = int4_fast<true, WANT_V>(acc, k, g.w, sink);
+        } else {
+            if (ok) ok = int3_fast<true, WANT_V>(acc, k, g.q2w, g.q1w, sink);
+        }
+        if (!ok) reduce_block_exact<C, WANT_V>(wp, N, tile, b, &g, sink);
+    }
+    store_block(gather + tile * Layout<C>::kTileBytes, b, g);
+}
+
 template <int C, int N, bool FUSED>
 __global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InPtrs wires, uint8_t *gather,
                                                      const __grid_constant__ OutPtrs out, size_t tile_begin,
@@ -263,38 +294,78 @@ __global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InP
     if (t < ntiles * kBlocksPerTile) {
         const size_t tile = tile0 + t / kBlocksPerTile;
         const int b = t % kBlocksPerTile;
-        Packed<C> p[N];
-#pragma unroll
-        for (int r = 0; r < N; ++r) load_block(wires.p[r] + tile * Layout<C>::kTileBytes, b, p[r]);
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.0f;     // +0.0f, then ranks in ascending order
-#pragma unroll
-        for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
-        const float a = absmax_f32x32(acc);
-        Packed<C> g;
-        const auto sink = [&]() {
-            if constexpr (FUSED) return StageSink{stage, t};
-            else return NoSink{};
-        }();
-        if constexpr (C == kFP8) {
-            encode_fp8<FUSED>(acc, a, g, sink);
-        } else {
-            const IntScale k = int_scale<Layout<C>::kBits>(a);
-            g.scale = k.bits;
-            bool ok = k.fast;
-            if constexpr (C == kINT4) {
-                if (ok) ok = int4_fast<true, FUSED>(acc, k, g.w, sink);
-            } else {
-                if (ok) ok = int3_fast<true, FUSED>(acc, k, g.q2w, g.q1w, sink);
-            }
-            if (!ok) reduce_block_exact<C, FUSED>(wires.p, N, tile, b, &g, sink);
-        }
-        store_block(gather + tile * Layout<C>::kTileBytes, b, g);
+        if constexpr (FUSED) reduce_block<C, N, true>(wires.p, tile, b, gather, StageSink{stage, t});
+        else reduce_block<C, N, false>(wires.p, tile, b, gather, NoSink{});
     }
     if (FUSED) {
         __syncthreads();
         stage_to_outputs(stage, out, N, tile0 * (kTileElems * 2), ntiles);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K123 (single-pass schedule): one persistent kernel.  For each chunk of 4
+// tiles a CTA quantises the chunk of every rank into that rank's wire (stage
+// 1), then reduces the chunk from the wires it has just written, requantises
+// it into the gathered wire and decodes it into every rank's output (stages 2
+// and 3).  A tile's result depends only on the same tile of every rank, so no
+// CTA waits for another; each thread reads back only wire blocks it wrote
+// itself (same thread, program order).  The next rank's BF16 chunk is
+// prefetched with cp.async while the current one is processed.
+// ---------------------------------------------------------------------------
+template <int C, int N>
+__global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_constant__ InPtrs in,
+                                                                  const __grid_constant__ OutPtrs wire,
+                                                                  uint8_t *gather,
+                                                                  const __grid_constant__ OutPtrs out,
+                                                                  size_t tiles, unsigned chunks) {
+    __shared__ __align__(128) uint8_t stage_in[2][kStageBytes];
+    __shared__ __align__(128) uint8_t stage_out[kStageBytes];
+    const int t = threadIdx.x;
+    unsigned c = blockIdx.x;
+    if (c < chunks) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        stage_load_chunk(stage_in[0], in.p[0] + tile0 * (kTileElems * 2),
+                         (int)min((size_t)kTilesPerCta, tiles - tile0));
+    }
+    cp_async_commit();
+    int buf = 0;
+    for (; c < chunks; c += gridDim.x) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+        const bool active = t < ntiles * kBlocksPerTile;
+        const size_t tile = tile0 + t / kBlocksPerTile;
+        const int b = t % kBlocksPerTile;
+#pragma unroll 1
+        for (int r = 0; r < N; ++r) {
+            // prefetch the next item: rank r+1 of this chunk, or rank 0 of the next chunk
+            const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
+            if (cn < chunks) {
+                const size_t tn = (size_t)cn * kTilesPerCta;
+                stage_load_chunk(stage_in[buf ^ 1], in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
+                                 (int)min((size_t)kTilesPerCta, tiles - tn));
+            }
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncthreads();
+            if (active) {
+                uint32_t x16[16];
+                stage_read(stage_in[buf], t, x16);
+                float x[32];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
+                const float a = absmax_bf16x32(x16);
+                Packed<C> p;
+                encode<C, false, false>(x, a, p, NoSink{});
+                store_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
+            }
+            __syncthreads();                           // stage_in[buf] is refilled next
+            buf ^= 1;
+        }
+        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{stage_out, t});
+        __syncthreads();
+        stage_to_outputs(stage_out, out, N, tile0 * (kTileElems * 2), ntiles);
+        __syncthreads();                               // stage_out is rewritten next chunk
     }
 }
 
@@ -444,6 +515,41 @@ static void launch_bf16_reduce(const InPtrs &in, int N, uint8_t *g, const OutPtr
     }
 }
 
+template <int C, int N>
+static void launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
+                             cudaStream_t st) {
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned res = resident_ctas(k_allreduce_single<C, N>);
+    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 4u));
+    k_allreduce_single<C, N><<<grid, kThreads, 0, st>>>(in, wire, g, o, tiles, chunks);
+}
+
+template <int C>
+static void launch_single_c(const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
+                            size_t tiles, cudaStream_t st) {
+    switch (N) {
+    case 1: launch_single_cn<C, 1>(in, wire, g, o, tiles, st); break;
+    case 2: launch_single_cn<C, 2>(in, wire, g, o, tiles, st); break;
+    case 3: launch_single_cn<C, 3>(in, wire, g, o, tiles, st); break;
+    case 4: launch_single_cn<C, 4>(in, wire, g, o, tiles, st); break;
+    case 5: launch_single_cn<C, 5>(in, wire, g, o, tiles, st); break;
+    case 6: launch_single_cn<C, 6>(in, wire, g, o, tiles, st); break;
+    case 7: launch_single_cn<C, 7>(in, wire, g, o, tiles, st); break;
+    case 8: launch_single_cn<C, 8>(in, wire, g, o, tiles, st); break;
+    default: break;
+    }
+}
+
+static void launch_single(int codec, const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
+                          size_t tiles, cudaStream_t st) {
+    switch (codec) {
+    case kINT4: launch_single_c<kINT4>(in, wire, N, g, o, tiles, st); break;
+    case kINT3: launch_single_c<kINT3>(in, wire, N, g, o, tiles, st); break;
+    case kFP8: launch_single_c<kFP8>(in, wire, N, g, o, tiles, st); break;
+    default: break;
+    }
+}
+
 static void launch_decode(int codec, const uint8_t *wire, const OutPtrs &o, int N, size_t tiles, cudaStream_t st) {
     const unsigned grid = grid_for_tiles(tiles);
     switch (codec) {
@@ -576,8 +682,11 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
                                       void *const *out, void *workspace, size_t workspace_bytes,
                                       const lpar_options_t *opts, cudaStream_t stream) {
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
-    const int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_FUSED;
-    if (schedule != LPAR_SCHEDULE_FUSED && schedule != LPAR_SCHEDULE_THREE_STAGE) return LPAR_ERR_UNSUPPORTED;
+    int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_AUTO;
+    if (schedule != LPAR_SCHEDULE_AUTO && schedule != LPAR_SCHEDULE_FUSED &&
+        schedule != LPAR_SCHEDULE_THREE_STAGE && schedule != LPAR_SCHEDULE_SINGLE_PASS)
+        return LPAR_ERR_UNSUPPORTED;
+    if (schedule == LPAR_SCHEDULE_AUTO) schedule = LPAR_SCHEDULE_SINGLE_PASS;
     if (N < 1 || N > kMaxRanks || n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
     if (!inputs || !out || !workspace) return LPAR_ERR_INVALID_ARG;
@@ -594,7 +703,7 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
     if (workspace_bytes < lpar_workspace_bytes(N, n, eff)) return LPAR_ERR_WORKSPACE_TOO_SMALL;
     const size_t tiles = n / kTileElems;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    const bool fused = schedule == LPAR_SCHEDULE_FUSED;
+    const bool fused = schedule != LPAR_SCHEDULE_THREE_STAGE;   // BF16: fused and single-pass coincide
     auto mark = [&](int i) {
         if (opts && opts->stage_events[i]) cudaEventRecord(opts->stage_events[i], stream);
     };
@@ -626,6 +735,11 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
     }
     uint8_t *gather = ws + (size_t)N * wb;
     mark(0);
+    if (schedule == LPAR_SCHEDULE_SINGLE_PASS) {
+        launch_single(eff, in, wires, N, gather, o, tiles, stream);
+        mark(1);
+        return launch_status();
+    }
     launch_quantize(eff, in, wires, N, tiles, stream);
     if (cudaGetLastError() != cudaSuccess) return LPAR_ERR_CUDA;
     mark(1);

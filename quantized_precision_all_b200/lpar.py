@@ -19,8 +19,9 @@ LIB_PATH = os.path.join(HERE, "liblpar.so")
 LPAR_CODEC_BF16, LPAR_CODEC_FP8_E4M3, LPAR_CODEC_INT4, LPAR_CODEC_INT3 = 0, 1, 2, 3
 CODECS = {"bf16": LPAR_CODEC_BF16, "fp8": LPAR_CODEC_FP8_E4M3, "int4": LPAR_CODEC_INT4, "int3": LPAR_CODEC_INT3}
 CODEC_NAMES = {v: k for k, v in CODECS.items()}
-LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE = 0, 1
-SCHEDULES = {"fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE}
+LPAR_SCHEDULE_AUTO, LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE, LPAR_SCHEDULE_SINGLE_PASS = 0, 1, 2, 3
+SCHEDULES = {"auto": LPAR_SCHEDULE_AUTO, "fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE,
+             "single_pass": LPAR_SCHEDULE_SINGLE_PASS}
 STATUS = {0: "LPAR_OK", 1: "LPAR_ERR_INVALID_ARG", 2: "LPAR_ERR_MISALIGNED",
           3: "LPAR_ERR_WORKSPACE_TOO_SMALL", 4: "LPAR_ERR_UNSUPPORTED", 5: "LPAR_ERR_CUDA"}
 TILE_ELEMS = 2048
@@ -106,7 +107,7 @@ def _stream(stream):
     return stream.cuda_stream
 
 
-def _options(min_quant_bytes=0, schedule="fused", stage_events=None):
+def _options(min_quant_bytes=0, schedule="auto", stage_events=None):
     sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
     opts = lpar_options_t(min_quant_bytes, sched)
     for i, ev in enumerate(stage_events or ()):
@@ -152,7 +153,7 @@ def lpar_decode(wire, n, codec, out_bf16, stream=None):
     _check(_lib.lpar_decode(_ptr(wire), n, _codec(codec), _ptr(out_bf16), _stream(stream)), "lpar_decode")
 
 
-def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_bytes=0, schedule="fused",
+def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_bytes=0, schedule="auto",
                    stream=None, N=None, stage_events=None):
     ins = _ptr_array(inputs)
     outs = _ptr_array(out)
@@ -163,7 +164,7 @@ def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_
            "lpar_allreduce")
 
 
-def lpar_allreduce_static(inputs, n, codec, out, min_quant_bytes=0, schedule="fused", stream=None, N=None):
+def lpar_allreduce_static(inputs, n, codec, out, min_quant_bytes=0, schedule="auto", stream=None, N=None):
     """lpar_allreduce with the library's own 16 MiB workspace (no allocation)."""
     ins = _ptr_array(inputs)
     outs = _ptr_array(out)
@@ -178,7 +179,7 @@ def lpar_status_string(status):
 
 
 # ---- convenience: allocate with torch, then call the C ABI -----------------------
-def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedule="fused", stream=None):
+def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedule="auto", stream=None):
     """All-reduce a list of N equal-size BF16 CUDA tensors; returns the N outputs."""
     import torch
     n = inputs[0].numel()

@@ -116,7 +116,7 @@ def test_argument_errors_allreduce(L):
     st = 0
     n = 2048 * 4
     ws = L.lpar_workspace_bytes(2, n, "int4")
-    ok = dict(min_quant_bytes=0, schedule="fused", stream=st)
+    ok = dict(min_quant_bytes=0, schedule="auto", stream=st)
     assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws - 16, **ok) == 3
     assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, M], A, ws, **ok) == 2
     assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], M, ws, **ok) == 2

@@ -342,7 +342,7 @@ def test_reduce_bf16_rounding_ties(L):
 # ---------------------------------------------------------------------------
 # The whole all-reduce
 # ---------------------------------------------------------------------------
-def run_allreduce(L, xs, codec, schedule="fused", min_quant_bytes=0, inplace=False):
+def run_allreduce(L, xs, codec, schedule="auto", min_quant_bytes=0, inplace=False):
     N, n = len(xs), xs[0].size
     ins = [to_device(x) for x in xs]
     outs = ins if inplace else [Guarded(2 * n, fill=0x00) for _ in range(N)]
@@ -357,7 +357,7 @@ def run_allreduce(L, xs, codec, schedule="fused", min_quant_bytes=0, inplace=Fal
 
 @pytest.mark.parametrize("codec", CODECS)
 @pytest.mark.parametrize("N", [1, 2, 3, 8])
-@pytest.mark.parametrize("schedule", ["fused", "three_stage"])
+@pytest.mark.parametrize("schedule", ["auto", "fused", "three_stage", "single_pass"])
 def test_allreduce_matches_oracle(L, codec, N, schedule):
     tiles = 9                                          # 2 CTAs + a ragged one per rank
     n = tiles * 2048
@@ -420,7 +420,7 @@ def test_workload_full_oracle(L, name):
     w = W.WORKLOADS[name]
     xs = workload_bits(w)
     for codec in w.codecs:
-        for schedule in ("fused", "three_stage"):
+        for schedule in ("fused", "three_stage", "single_pass"):
             outs, _ = run_allreduce(L, xs, codec, schedule, min_quant_bytes=w.min_quant_bytes)
             ref, used = O.allreduce(xs, codec, min_quant_bytes=w.min_quant_bytes)
             assert used == codec
@@ -460,12 +460,13 @@ def test_workload_large_sampled_tiles(L):
     for codec in w.codecs:
         outs = [torch.empty_like(x) for x in xs]
         ws = torch.empty(L.lpar_workspace_bytes(w.N, w.n, codec), dtype=torch.uint8, device="cuda")
-        L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel())
-        torch.cuda.synchronize()
         ref, _ = O.allreduce(sample_in, codec)
-        for o in outs:
-            got = o[idx].view(torch.int16).cpu().numpy().view(np.uint16)
-            assert np.array_equal(got, ref[0])
+        for schedule in ("fused", "single_pass"):
+            L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel(), schedule=schedule)
+            torch.cuda.synchronize()
+            for o in outs:
+                got = o[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+                assert np.array_equal(got, ref[0]), (codec, schedule)
         del outs, ws
     torch.cuda.empty_cache()
 
@@ -493,11 +494,12 @@ def test_sweep_sampled_tiles(L, N):
         ws = torch.empty(max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS), dtype=torch.uint8,
                          device="cuda")
         for codec in W.SWEEP_CODECS:
-            L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel())
-            torch.cuda.synchronize()
             ref, _ = O.allreduce(sample_in, codec)
-            got = [o[idx].view(torch.int16).cpu().numpy().view(np.uint16) for o in outs]
-            for g in got:
-                assert np.array_equal(g, ref[0]), (N, mb, codec)
+            for schedule in ("fused", "single_pass"):
+                L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel(), schedule=schedule)
+                torch.cuda.synchronize()
+                got = [o[idx].view(torch.int16).cpu().numpy().view(np.uint16) for o in outs]
+                for g in got:
+                    assert np.array_equal(g, ref[0]), (N, mb, codec, schedule)
         del xs, outs, ws
         torch.cuda.empty_cache()
