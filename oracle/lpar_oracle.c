@@ -25,6 +25,9 @@
  *         reduce-scatter then all-gather).
  *  [FP8]  "FP8 Formats for Deep Learning", abstract (E4M3: 4 exponent bits,
  *         3 mantissa bits, no infinities, a single NaN mantissa pattern).
+ *  [MX]   "Microscaling Data Formats for Deep Learning", abstract (a scale
+ *         shared by a block of narrow floating-point elements); [QR] Summary
+ *         ("INT4 and FP4" modes of the same all-reduce).
  *
  * Readings where the pages are silent (each one is listed with its reason in
  * the design notes): 32-element blocks in 2048-element tiles (the only split
@@ -36,6 +39,10 @@
  * encoded by multiplying with fl32(1 / s), flushed to zero below 2^-126;
  * requantisation with the same codec after the FP32 sum (the "transmitted
  * tile" of the all-gather); sum in ascending rank order from +0.0f.
+ * MXFP4 (the FP4 codec): E2M1 elements, one E8M0 power-of-two scale per 32
+ * elements, shared exponent floor(log2(absmax)) - 2 (2 = the largest E2M1
+ * exponent) clamped to [-127, 127], elements RNE(x / 2^E) saturated at +-6;
+ * tile = 1024 B of nibbles (element 2k low) then 64 scale bytes.
  */
 #include "lpar_oracle.h"
 
@@ -158,6 +165,34 @@ uint8_t orc_f32_to_e4m3_rne_satfinite(float x)
     return (uint8_t)(sign | encode_on_grid(r, 4, -6, 7));
 }
 
+/*
+ * E2M1 (the MX FP4 element): 1 sign, 2 exponent (bias 1), 1 mantissa bit; no
+ * infinities or NaN.  Exponent field 0 holds the subnormal 0.m * 2^0, so the
+ * magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4 and 6.
+ */
+float orc_e2m1_to_f32(uint8_t c)
+{
+    int sign = (c >> 3) & 1;
+    int ef = (c >> 1) & 3;
+    int mf = c & 1;
+    double v = (ef == 0) ? 0.5 * mf : ldexp(1.0 + 0.5 * mf, ef - 1);
+    return (float)(sign ? -v : v);
+}
+
+/* A real value (binary64, exact) -> E2M1, round to nearest even, magnitudes
+ * above 6 saturate to 6; the sign is kept (a negative value that rounds to
+ * zero gives the negative-zero code 0x8). */
+uint8_t orc_e2m1_rne_satfinite(double y)
+{
+    uint8_t sign = signbit(y) ? 0x8 : 0x0;
+    double r = round_to_format(fabs(y), 2, 0);
+    if (r > 6.0) r = 6.0;
+    return (uint8_t)(sign | encode_on_grid(r, 2, 0, 1));
+}
+
+/* E8M0 scale code -> 2^(code - 127) (code 255, the NaN pattern, is never produced). */
+double orc_e8m0_to_f64(uint8_t code) { return ldexp(1.0, (int)code - 127); }
+
 /* ------------------------------------------------------------------------- */
 /* Tile geometry ([QR] Summary: 1152 B INT4, 896 B INT3 per transmitted tile). */
 /* ------------------------------------------------------------------------- */
@@ -170,6 +205,7 @@ size_t orc_tile_bytes(int codec)
     case ORC_INT4: return ORC_TILE_ELEMS / 2 + ORC_BLOCKS_PER_TILE * 2;       /* 1024 + 128 = 1152 */
     case ORC_INT3: return ORC_TILE_ELEMS / 4 + ORC_TILE_ELEMS / 8
                         + ORC_BLOCKS_PER_TILE * 2;                   /* 512 + 256 + 128 = 896 */
+    case ORC_MXFP4: return ORC_TILE_ELEMS / 2 + ORC_BLOCKS_PER_TILE;  /* 1024 + 64 = 1088 */
     default: return 0;
     }
 }
@@ -242,6 +278,38 @@ float orc_dequant_fp8(uint8_t code, float scale)
     return orc_e4m3_to_f32(code) * scale;        /* one binary32 multiply */
 }
 
+/*
+ * MXFP4 block ([MX]): the shared exponent E is the largest power of two that
+ * the block's absmax reaches, minus the largest E2M1 exponent (2), so the
+ * absmax lands in [4, 8) after scaling; E is clamped to the E8M0 range
+ * [-127, 127] (an all-zero block takes the bottom of the range).  Each element
+ * is x / 2^E (exact in binary64) rounded to E2M1.
+ */
+void orc_quant_block_mxfp4(const float *x, uint8_t *scale_code, uint8_t *codes)
+{
+    float a = 0.0f;
+    for (int j = 0; j < ORC_BLOCK; ++j) {
+        float m = fabsf(x[j]);
+        if (m > a) a = m;
+    }
+    int E = -127;
+    if (a > 0.0f) {
+        int F;
+        frexp((double)a, &F);                    /* a = m * 2^F, m in [0.5, 1): floor(log2 a) = F - 1 */
+        E = (F - 1) - 2;
+        if (E < -127) E = -127;
+        if (E > 127) E = 127;
+    }
+    for (int j = 0; j < ORC_BLOCK; ++j) codes[j] = orc_e2m1_rne_satfinite(ldexp((double)x[j], -E));
+    *scale_code = (uint8_t)(E + 127);
+}
+
+float orc_dequant_mxfp4(uint8_t code, uint8_t scale_code)
+{
+    /* exact: a 2-bit significand times a power of two in [2^-127, 2^125] */
+    return (float)((double)orc_e2m1_to_f32(code) * orc_e8m0_to_f64(scale_code));
+}
+
 /* ------------------------------------------------------------------------- */
 /* Tile packing (byte layout is a reading: codes/planes first, scales last).  */
 /* ------------------------------------------------------------------------- */
@@ -274,6 +342,14 @@ void orc_quant_tile(const float *x, int codec, uint8_t *tile)
             orc_quant_block_fp8(xb, &s, codes);
             for (int j = 0; j < ORC_BLOCK; ++j) tile[b * ORC_BLOCK + j] = codes[j];
             put_f32_le(tile + ORC_TILE_ELEMS + 4 * b, s);
+        } else if (codec == ORC_MXFP4) {
+            uint8_t sc;
+            orc_quant_block_mxfp4(xb, &sc, codes);
+            for (int j = 0; j < ORC_BLOCK; ++j) {
+                int i = b * ORC_BLOCK + j;
+                tile[i / 2] |= (uint8_t)(codes[j] << (4 * (i % 2)));
+            }
+            tile[ORC_TILE_ELEMS / 2 + b] = sc;
         } else if (codec == ORC_INT4) {
             uint16_t sb;
             orc_quant_block_int(xb, 4, &sb, codes);
@@ -302,7 +378,8 @@ uint8_t orc_tile_code(const uint8_t *tile, int codec, int i)
 {
     switch (codec) {
     case ORC_FP8:  return tile[i];
-    case ORC_INT4: return (uint8_t)((tile[i / 2] >> (4 * (i % 2))) & 0xF);
+    case ORC_INT4:
+    case ORC_MXFP4: return (uint8_t)((tile[i / 2] >> (4 * (i % 2))) & 0xF);
     case ORC_INT3: {
         uint8_t lo = (uint8_t)((tile[i / 4] >> (2 * (i % 4))) & 3);
         uint8_t hi = (uint8_t)((tile[ORC_TILE_ELEMS / 4 + i / 8] >> (i % 8)) & 1);
@@ -331,6 +408,9 @@ void orc_dequant_tile(const uint8_t *tile, int codec, float *v)
         case ORC_INT3:
             v[i] = orc_dequant_int(orc_tile_code(tile, codec, i), 3,
                                    get_u16_le(tile + ORC_TILE_ELEMS / 4 + ORC_TILE_ELEMS / 8 + 2 * b));
+            break;
+        case ORC_MXFP4:
+            v[i] = orc_dequant_mxfp4(orc_tile_code(tile, codec, i), tile[ORC_TILE_ELEMS / 2 + b]);
             break;
         }
     }
@@ -394,6 +474,7 @@ int orc_allreduce(const uint16_t *const *in_bf16, int N, size_t n, int codec,
                   uint16_t *const *out_bf16, size_t min_quant_bytes)
 {
     if (N < 1 || N > ORC_MAX_RANKS || n % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
     if (codec != ORC_BF16 && 2 * n < min_quant_bytes) codec = ORC_BF16;
     size_t wb = orc_wire_bytes(codec, n);
     size_t tiles = n / ORC_TILE_ELEMS;

@@ -18,7 +18,7 @@
 extern "C" {
 #endif
 
-enum { ORC_BF16 = 0, ORC_FP8 = 1, ORC_INT4 = 2, ORC_INT3 = 3 };
+enum { ORC_BF16 = 0, ORC_FP8 = 1, ORC_INT4 = 2, ORC_INT3 = 3, ORC_MXFP4 = 4 };
 enum { ORC_BLOCK = 32, ORC_TILE_ELEMS = 2048, ORC_BLOCKS_PER_TILE = 64, ORC_MAX_RANKS = 8 };
 
 /* number formats */
@@ -28,6 +28,9 @@ uint16_t orc_f32_to_f16_rne(float x);
 float    orc_f16_to_f32(uint16_t h);
 float    orc_e4m3_to_f32(uint8_t e);
 uint8_t  orc_f32_to_e4m3_rne_satfinite(float x);
+float    orc_e2m1_to_f32(uint8_t c);
+uint8_t  orc_e2m1_rne_satfinite(double y);
+double   orc_e8m0_to_f64(uint8_t code);
 
 /* geometry */
 size_t orc_tile_bytes(int codec);
@@ -38,6 +41,8 @@ void  orc_quant_block_int(const float *x, int bits, uint16_t *scale_bits, uint8_
 float orc_dequant_int(uint8_t code, int bits, uint16_t scale_bits);
 void  orc_quant_block_fp8(const float *x, float *scale, uint8_t *codes);
 float orc_dequant_fp8(uint8_t code, float scale);
+void  orc_quant_block_mxfp4(const float *x, uint8_t *scale_code, uint8_t *codes);
+float orc_dequant_mxfp4(uint8_t code, uint8_t scale_code);
 
 /* one 2048-element tile */
 void    orc_quant_tile(const float *x, int codec, uint8_t *tile);

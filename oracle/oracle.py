@@ -4,7 +4,8 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this module.  It never touches the CUDA library.
 
 Arrays are numpy: BF16 data travels as ``uint16`` bit patterns, wires as
-``uint8``.  Codecs are named by string: ``bf16``, ``fp8``, ``int4``, ``int3``.
+``uint8``.  Codecs are named by string: ``bf16``, ``fp8``, ``int4``, ``int3``,
+``mxfp4``.
 """
 import ctypes
 import os
@@ -13,7 +14,7 @@ import numpy as np
 
 from . import build_oracle
 
-CODECS = {"bf16": 0, "fp8": 1, "int4": 2, "int3": 3}
+CODECS = {"bf16": 0, "fp8": 1, "int4": 2, "int3": 3, "mxfp4": 4}
 TILE_ELEMS = 2048
 BLOCK = 32
 MAX_RANKS = 8
@@ -38,12 +39,17 @@ def lib():
             "orc_f16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
             "orc_e4m3_to_f32": (ctypes.c_float, [ctypes.c_uint8]),
             "orc_f32_to_e4m3_rne_satfinite": (ctypes.c_uint8, [ctypes.c_float]),
+            "orc_e2m1_to_f32": (ctypes.c_float, [ctypes.c_uint8]),
+            "orc_e2m1_rne_satfinite": (ctypes.c_uint8, [ctypes.c_double]),
+            "orc_e8m0_to_f64": (ctypes.c_double, [ctypes.c_uint8]),
             "orc_tile_bytes": (sz, [ctypes.c_int]),
             "orc_wire_bytes": (sz, [ctypes.c_int, sz]),
             "orc_quant_block_int": (None, [f32p, ctypes.c_int, u16p, u8p]),
             "orc_dequant_int": (ctypes.c_float, [ctypes.c_uint8, ctypes.c_int, ctypes.c_uint16]),
             "orc_quant_block_fp8": (None, [f32p, f32p, u8p]),
             "orc_dequant_fp8": (ctypes.c_float, [ctypes.c_uint8, ctypes.c_float]),
+            "orc_quant_block_mxfp4": (None, [f32p, u8p, u8p]),
+            "orc_dequant_mxfp4": (ctypes.c_float, [ctypes.c_uint8, ctypes.c_uint8]),
             "orc_quant_tile": (None, [f32p, ctypes.c_int, u8p]),
             "orc_tile_code": (ctypes.c_uint8, [u8p, ctypes.c_int, ctypes.c_int]),
             "orc_dequant_tile": (None, [u8p, ctypes.c_int, f32p]),
@@ -95,6 +101,19 @@ def f32_to_e4m3(x):
     return lib().orc_f32_to_e4m3_rne_satfinite(float(np.float32(x)))
 
 
+def e2m1_to_f32(c):
+    return lib().orc_e2m1_to_f32(int(c))
+
+
+def e2m1_rne(y):
+    """A real value (Python float, binary64) -> E2M1 code."""
+    return lib().orc_e2m1_rne_satfinite(float(y))
+
+
+def e8m0_value(code):
+    return lib().orc_e8m0_to_f64(int(code))
+
+
 # ---- geometry --------------------------------------------------------------
 def tile_bytes(codec):
     return lib().orc_tile_bytes(_codec(codec))
@@ -129,6 +148,19 @@ def quant_block_fp8(x):
 
 def dequant_fp8(code, scale):
     return lib().orc_dequant_fp8(int(code), float(np.float32(scale)))
+
+
+def quant_block_mxfp4(x):
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    assert x.size == BLOCK
+    sc = ctypes.c_uint8()
+    codes = np.zeros(BLOCK, np.uint8)
+    lib().orc_quant_block_mxfp4(_ptr(x, ctypes.c_float), ctypes.byref(sc), _ptr(codes, ctypes.c_uint8))
+    return sc.value, codes
+
+
+def dequant_mxfp4(code, scale_code):
+    return lib().orc_dequant_mxfp4(int(code), int(scale_code))
 
 
 def quant_tile(x, codec):

@@ -126,3 +126,43 @@ def quant_block_fp8(xs):
         return Fraction(0), [0] * len(xs)
     inv = rn32(1 / s)
     return s, [e4m3_rne_satfinite(rn32(x * inv)) for x in xs]
+
+
+# ---- MXFP4: E2M1 elements with one power-of-two (E8M0) scale per block -------
+# The eight E2M1 magnitudes, listed in code order 0..7 (1 sign bit above them).
+E2M1_MAGNITUDES = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2),
+                   Fraction(2), Fraction(3), Fraction(4), Fraction(6)]
+
+
+def e2m1_rne_satfinite(fr: Fraction, negative: bool) -> int:
+    """Nearest E2M1 code to a real value by search over the eight magnitudes:
+    ties go to the code with an even mantissa bit (code & 1 == 0), magnitudes
+    above 6 saturate, and the sign bit follows `negative` (so -0 keeps it)."""
+    a = abs(fr)
+    best = None
+    for c, v in enumerate(E2M1_MAGNITUDES):
+        d = abs(v - a)
+        if best is None or d < best[0] or (d == best[0] and (c & 1) == 0):
+            best = (d, c)
+    code = best[1] if a <= 6 else 7
+    return code | (0x8 if negative else 0)
+
+
+def mx_shared_exponent(a: Fraction) -> int:
+    """The integer E with 4 * 2^E <= a < 8 * 2^E (the absmax scaled into the
+    top binade of E2M1), clamped to the E8M0 range; -127 for a == 0.  Found by
+    search from a bracket, not by a logarithm formula."""
+    if a == 0:
+        return -127
+    E = 0
+    while Fraction(4) * Fraction(2) ** E > a:
+        E -= 1
+    while Fraction(8) * Fraction(2) ** E <= a:
+        E += 1
+    return max(-127, min(127, E))
+
+
+def quant_block_mxfp4(xs, negs):
+    """xs: exact values, negs: their sign bits.  Returns (E, codes)."""
+    E = mx_shared_exponent(max(abs(x) for x in xs))
+    return E, [e2m1_rne_satfinite(x / Fraction(2) ** E, n) for x, n in zip(xs, negs)]
