@@ -35,7 +35,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "quantized all-reduce GB/s (N x input bytes/s) and % of HBM peak on 1 B200"
 TILE = 2048
-CODEC_C = {"bf16": 2.0, "fp8": 2304 / 2048, "int4": 1152 / 2048, "int3": 896 / 2048}
+CODEC_C = {"bf16": 2.0, "fp8": 2304 / 2048, "int4": 1152 / 2048, "int3": 896 / 2048, "mxfp4": 1088 / 2048}
 KERNEL_SOURCES = ("quantized_precision_all_b200/csrc/lpar_kernels.cu", "quantized_precision_all_b200/csrc/lpar_codec.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 REF_TILES_PER_STEP = 256            # reference arm: 0.5 Mi elements per rank per step

@@ -21,6 +21,9 @@
  *    (tree all-reduce = reduce-scatter followed by all-gather).
  *  - "FP8 Formats for Deep Learning", abstract (E4M3: no infinities, one NaN
  *    pattern, so 448 is the largest finite value).
+ *  - "Microscaling Data Formats for Deep Learning", abstract (narrow
+ *    floating-point elements sharing one per-block scale), with the INT3
+ *    page's Summary naming the FP4 mode of the same all-reduce.
  *
  * Formats (readings where the pages are silent are marked "reading"):
  *  - A tile is 2048 consecutive elements made of 64 blocks of 32 (reading,
@@ -36,9 +39,17 @@
  *  - FP8 tile (2304 B): 2048 E4M3 codes, then 64 little-endian binary32 scales
  *    s = fl32(absmax / 448); a block with s < 2^-126 is stored as s = 0 and
  *    codes 0; otherwise code = e4m3_rne_satfinite(fl32(x * fl32(1 / s))).
+ *  - MXFP4 tile (1088 B): 1024 B of E2M1 codes (element i in byte i/2, low
+ *    nibble for even i; 1 sign, 2 exponent bits with bias 1, 1 mantissa bit:
+ *    magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), then 64 E8M0 scale bytes
+ *    (value 2^(byte - 127)).  E = clamp(floor(log2(absmax)) - 2, -127, 127)
+ *    (-127 for an all-zero block), code = e2m1_rne(x / 2^E) with magnitudes
+ *    above 6 saturating to 6 and the sign kept (a negative value that rounds
+ *    to zero gives code 0x8).
  *  - BF16 "tile" (4096 B): the BF16 values themselves (no compression).
  *  - Dequantised value: (float)q * s for INT (exact), fl32(e4m3(code) * s) for
- *    FP8.  Final output: bf16_rne of the dequantised gathered value.
+ *    FP8, e2m1(code) * 2^E for MXFP4 (exact).  Final output: bf16_rne of the
+ *    dequantised gathered value.
  *
  * Conventions for every call:
  *  - All data pointers are DEVICE pointers on the current CUDA device; the
@@ -75,7 +86,8 @@ typedef enum {
     LPAR_CODEC_BF16 = 0,      /* uncompressed passthrough, 4096 B per tile */
     LPAR_CODEC_FP8_E4M3 = 1,  /* E4M3 codes + binary32 scale per 32 elements, 2304 B per tile */
     LPAR_CODEC_INT4 = 2,      /* 4-bit codes + binary16 scale per 32 elements, 1152 B per tile */
-    LPAR_CODEC_INT3 = 3       /* q2w + q1w planes + binary16 scale per 32, 896 B per tile */
+    LPAR_CODEC_INT3 = 3,      /* q2w + q1w planes + binary16 scale per 32, 896 B per tile */
+    LPAR_CODEC_MXFP4 = 4      /* E2M1 codes + E8M0 (power of two) scale per 32, 1088 B per tile */
 } lpar_codec_t;
 
 typedef enum {
@@ -113,7 +125,7 @@ typedef struct {
 } lpar_options_t;
 
 /* Bytes of one 2048-element tile: 4096 (BF16), 2304 (FP8), 1152 (INT4), 896
- * (INT3); 0 for an unknown codec. */
+ * (INT3), 1088 (MXFP4); 0 for an unknown codec. */
 size_t lpar_tile_bytes(lpar_codec_t codec);
 
 /* Bytes of the wire of an n-element message: (n / 2048) * lpar_tile_bytes(codec). */

@@ -11,6 +11,10 @@
 //              q = clamp(RNE(x / s)) of the exact quotient, code = q + 2^(b-1).
 //   FP8 E4M3:  s = fl32(absmax / 448), zero block when s < 2^-126,
 //              code = e4m3_rne_satfinite(fl32(x * fl32(1 / s))).
+//   MXFP4:     ("Microscaling Data Formats for Deep Learning", abstract: a
+//              scale shared by a block of narrow floating-point elements)
+//              E = clamp(floor(log2(absmax)) - 2, -127, 127) stored as the E8M0
+//              byte E + 127; code = e2m1_rne_satfinite(x / 2^E), sign kept.
 //
 // Exact RNE(x / s) without a per-element division
 // -----------------------------------------------
@@ -60,7 +64,7 @@ constexpr int kBlock = 32;
 constexpr int kTileElems = 2048;
 constexpr int kBlocksPerTile = 64;
 
-enum CodecId : int { kBF16 = 0, kFP8 = 1, kINT4 = 2, kINT3 = 3 };
+enum CodecId : int { kBF16 = 0, kFP8 = 1, kINT4 = 2, kINT3 = 3, kMXFP4 = 4 };
 
 // Byte layout of one 2048-element tile.
 template <int C> struct Layout;
@@ -73,6 +77,9 @@ template <> struct Layout<kINT3> {
 template <> struct Layout<kFP8> {
     static constexpr int kTileBytes = 2304, kScaleOff = 2048;
 };
+template <> struct Layout<kMXFP4> {
+    static constexpr int kTileBytes = 1088, kScaleOff = 1024;
+};
 template <> struct Layout<kBF16> {
     static constexpr int kTileBytes = 4096;
 };
@@ -82,6 +89,7 @@ template <int C> struct Packed;
 template <> struct Packed<kINT4> { uint32_t w[4]; uint16_t scale; };          // 16 B codes
 template <> struct Packed<kINT3> { uint32_t q2w[2]; uint32_t q1w; uint16_t scale; };
 template <> struct Packed<kFP8> { uint32_t w[8]; float scale; };              // 32 B codes
+template <> struct Packed<kMXFP4> { uint32_t w[4]; uint32_t scale; };         // 16 B codes, E8M0 byte
 
 constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23: ulp 1, bits 0x4B400000
 constexpr float kMagic2 = 25165824.0f;                // 3 * 2^23 = 1.5 * 2^24: ulp 2
@@ -177,6 +185,40 @@ __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two));
     return h2;
+}
+
+// Two binary32 -> one byte of two E2M1 codes (RNE, finite saturation at +-6),
+// `lo` in bits 0..3, zero-extended to 32 bits.
+__device__ __forceinline__ uint32_t pack_e2m1x2(float lo, float hi) {
+    uint32_t d;
+    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}"
+        : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// Eight binary32 -> eight E2M1 codes, element k in nibble k.
+__device__ __forceinline__ uint32_t pack_e2m1x8(float a0, float a1, float a2, float a3, float a4, float a5,
+                                                float a6, float a7) {
+    const uint32_t b01 = __byte_perm(pack_e2m1x2(a0, a1), pack_e2m1x2(a2, a3), 0x0040);
+    const uint32_t b23 = __byte_perm(pack_e2m1x2(a4, a5), pack_e2m1x2(a6, a7), 0x0040);
+    return __byte_perm(b01, b23, 0x5410);
+}
+
+// Byte k of w (two E2M1 codes) -> packed binary16 pair (exact: E2M1 is a
+// subset of binary16), the low nibble's element in the low half.  The byte is
+// isolated first, so no other bits of the register reach the conversion.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t w, int k) {
+    const uint32_t two = __byte_perm(w, 0u, 0x4440u + (uint32_t)k);
+    uint32_t h;
+    asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h) : "r"(two));
+    return h;
+}
+
+// Eight E2M1 codes -> four packed binary16 pairs; pair j holds elements
+// (2j, 2j + 1) in (low, high).
+__device__ __forceinline__ void e2m1x8_to_h2(uint32_t w, uint32_t (&h)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) h[k] = e2m1x2_to_h2(w, k);
 }
 
 // Maximum of |bf16| over a packed pair, as a packed pair; the sign bits are
@@ -502,6 +544,42 @@ __device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed
     p.scale = s;
 }
 
+// MXFP4.  E8M0 scale byte ec = max(biased exponent of absmax - 2, 0): for a
+// normal absmax the biased exponent is floor(log2 a) + 127, so ec = E + 127
+// with E = floor(log2 a) - 2, and the clamp at 0 is E >= -127 (absmax zero or
+// below 2^-125).  x / 2^E is the product with 2^-E = 2^(127 - ec), whose
+// biased exponent 254 - ec is in [1, 254], so it is exact unless it falls
+// below 2^-126, where every value rounds to a signed zero either way.  Scalar IEEE products keep
+// subnormal inputs (stage-2 sums can be subnormal).
+__device__ __forceinline__ uint32_t mx_scale_code(float a) {
+    const int ef = (int)(__float_as_uint(a) >> 23);
+    return (uint32_t)max(ef - 2, 0);
+}
+__device__ __forceinline__ float mx_scale_value(uint32_t ec) {       // 2^(ec - 127), exact
+    return __uint_as_float(ec ? (ec << 23) : 0x00400000u);
+}
+
+template <bool WANT_V, class Sink>
+__device__ __forceinline__ void encode_mxfp4(const float (&x)[32], float a, Packed<kMXFP4> &p, const Sink &sink) {
+    const uint32_t ec = mx_scale_code(a);
+    const float m = __uint_as_float((254u - ec) << 23);          // 2^-E
+    p.scale = ec;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float *xi = x + 8 * i;
+        p.w[i] = pack_e2m1x8(__fmul_rn(xi[0], m), __fmul_rn(xi[1], m), __fmul_rn(xi[2], m), __fmul_rn(xi[3], m),
+                             __fmul_rn(xi[4], m), __fmul_rn(xi[5], m), __fmul_rn(xi[6], m), __fmul_rn(xi[7], m));
+        if (WANT_V) {                                             // E2M1 value * 2^E: exact, so is its BF16
+            const float sv = mx_scale_value(ec);
+            uint32_t h[4], o[4];
+            e2m1x8_to_h2(p.w[i], h);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] = pack_bf16x2(__fmul_rn(h2f(h[k], 0), sv), __fmul_rn(h2f(h[k], 1), sv));
+            sink.put(i, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Dequantisation.  INT codes become exact binary16 integers q (magic 1024 +
 // code, minus 1024 + bias), and acc = fl32(acc + q*s) is one mixed-precision
@@ -604,6 +682,24 @@ __device__ __forceinline__ void accumulate_fp8(const Packed<kFP8> &p, float (&ac
     }
 }
 
+// MXFP4: acc = fl32(acc + e * 2^E) in one FMA; the product has at most two
+// significant bits and is at least 2^-128, so it is exact and the FMA rounds
+// once, like the definition's acc + v.  Scalar: the product can be subnormal.
+__device__ __forceinline__ void accumulate_mxfp4(const Packed<kMXFP4> &p, float (&acc)[32]) {
+    const float sv = mx_scale_value(p.scale);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h[4];
+        e2m1x8_to_h2(p.w[i], h);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = 8 * i + 2 * k;
+            acc[j] = __fmaf_rn(h2f(h[k], 0), sv, acc[j]);
+            acc[j + 1] = __fmaf_rn(h2f(h[k], 1), sv, acc[j + 1]);
+        }
+    }
+}
+
 // Decode one block to BF16 (RNE), 16 packed words (element 2k in the low half).
 // The value is q * s (one exact product; -0 addend keeps the product's zero sign).
 __device__ __forceinline__ void decode_int4(const Packed<kINT4> &p, uint32_t (&o)[16]) {
@@ -646,6 +742,18 @@ __device__ __forceinline__ void decode_fp8(const Packed<kFP8> &p, uint32_t (&o)[
             const uint32_t e = e4m3x2_to_h2(p.w[i] >> (16 * h));
             o[2 * i + h] = pack_bf16x2(__fmul_rn(h2f(e, 0), p.scale), __fmul_rn(h2f(e, 1), p.scale));
         }
+    }
+}
+
+__device__ __forceinline__ void decode_mxfp4(const Packed<kMXFP4> &p, uint32_t (&o)[16]) {
+    const float sv = mx_scale_value(p.scale);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h[4];
+        e2m1x8_to_h2(p.w[i], h);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o[4 * i + k] = pack_bf16x2(__fmul_rn(h2f(h[k], 0), sv), __fmul_rn(h2f(h[k], 1), sv));
     }
 }
 

@@ -85,6 +85,16 @@ __device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<k
     *reinterpret_cast<float *>(tile + Layout<kFP8>::kScaleOff + 4 * b) = p.scale;
 }
 
+__device__ __forceinline__ void load_block(const uint8_t *tile, int b, Packed<kMXFP4> &p) {
+    const uint4 c = *reinterpret_cast<const uint4 *>(tile + 16 * b);
+    p.w[0] = c.x; p.w[1] = c.y; p.w[2] = c.z; p.w[3] = c.w;
+    p.scale = tile[Layout<kMXFP4>::kScaleOff + b];
+}
+__device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<kMXFP4> &p) {
+    *reinterpret_cast<uint4 *>(tile + 16 * b) = make_uint4(p.w[0], p.w[1], p.w[2], p.w[3]);
+    tile[Layout<kMXFP4>::kScaleOff + b] = (uint8_t)p.scale;
+}
+
 // Destinations for the decoded BF16 words of a block (piece j = 16 B).
 struct NoSink {
     __device__ __forceinline__ void put(int, uint4) const {}
@@ -136,6 +146,7 @@ __device__ __noinline__ void reduce_block_exact(const uint8_t *const *wp, int N,
 template <int C, bool STAGE2, bool WANT_V, class Sink>
 __device__ __forceinline__ void encode(const float (&x)[32], float a, Packed<C> &p, const Sink &sink) {
     if constexpr (C == kFP8) encode_fp8<WANT_V>(x, a, p, sink);
+    else if constexpr (C == kMXFP4) encode_mxfp4<WANT_V>(x, a, p, sink);
     else encode_int<C, STAGE2, WANT_V>(x, a, p, sink);
 }
 
@@ -143,6 +154,7 @@ template <int C>
 __device__ __forceinline__ void accumulate(const Packed<C> &p, float (&acc)[32]) {
     if constexpr (C == kINT4) accumulate_int4(p, acc);
     else if constexpr (C == kINT3) accumulate_int3(p, acc);
+    else if constexpr (C == kMXFP4) accumulate_mxfp4(p, acc);
     else accumulate_fp8(p, acc);
 }
 
@@ -150,6 +162,7 @@ template <int C>
 __device__ __forceinline__ void decode(const Packed<C> &p, uint32_t (&o)[16]) {
     if constexpr (C == kINT4) decode_int4(p, o);
     else if constexpr (C == kINT3) decode_int3(p, o);
+    else if constexpr (C == kMXFP4) decode_mxfp4(p, o);
     else decode_fp8(p, o);
 }
 
@@ -269,6 +282,8 @@ __device__ __forceinline__ void reduce_block(const uint8_t *const *wp, size_t ti
     Packed<C> g;
     if constexpr (C == kFP8) {
         encode_fp8<WANT_V>(acc, a, g, sink);
+    } else if constexpr (C == kMXFP4) {
+        encode_mxfp4<WANT_V>(acc, a, g, sink);
     } else {
         const IntScale k = int_scale<Layout<C>::kBits>(a);
         g.scale = k.bits;
@@ -467,6 +482,7 @@ static void launch_quantize(int codec, const InPtrs &in, const OutPtrs &wire, in
     case kINT4: launch_quantize_c<kINT4>(in, wire, N, tiles, st); break;
     case kINT3: launch_quantize_c<kINT3>(in, wire, N, tiles, st); break;
     case kFP8: launch_quantize_c<kFP8>(in, wire, N, tiles, st); break;
+    case kMXFP4: launch_quantize_c<kMXFP4>(in, wire, N, tiles, st); break;
     default: break;
     }
 }
@@ -494,6 +510,7 @@ static void launch_reduce(int codec, const InPtrs &w, int N, uint8_t *g, const O
     case kINT4: launch_reduce_c<kINT4, FUSED>(w, N, g, o, t0, t1, st); break;
     case kINT3: launch_reduce_c<kINT3, FUSED>(w, N, g, o, t0, t1, st); break;
     case kFP8: launch_reduce_c<kFP8, FUSED>(w, N, g, o, t0, t1, st); break;
+    case kMXFP4: launch_reduce_c<kMXFP4, FUSED>(w, N, g, o, t0, t1, st); break;
     default: break;
     }
 }
@@ -546,6 +563,7 @@ static void launch_single(int codec, const InPtrs &in, const OutPtrs &wire, int 
     case kINT4: launch_single_c<kINT4>(in, wire, N, g, o, tiles, st); break;
     case kINT3: launch_single_c<kINT3>(in, wire, N, g, o, tiles, st); break;
     case kFP8: launch_single_c<kFP8>(in, wire, N, g, o, tiles, st); break;
+    case kMXFP4: launch_single_c<kMXFP4>(in, wire, N, g, o, tiles, st); break;
     default: break;
     }
 }
@@ -556,6 +574,7 @@ static void launch_decode(int codec, const uint8_t *wire, const OutPtrs &o, int 
     case kINT4: k_decode<kINT4><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
     case kINT3: k_decode<kINT3><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
     case kFP8: k_decode<kFP8><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
+    case kMXFP4: k_decode<kMXFP4><<<grid, kThreads, 0, st>>>(wire, o, N, tiles); break;
     default: break;
     }
 }
@@ -569,7 +588,7 @@ static void launch_broadcast(const uint8_t *src, const OutPtrs &o, int N, size_t
 // ---------------------------------------------------------------------------
 // Validation helpers.
 // ---------------------------------------------------------------------------
-static inline bool codec_ok(int c) { return c >= LPAR_CODEC_BF16 && c <= LPAR_CODEC_INT3; }
+static inline bool codec_ok(int c) { return c >= LPAR_CODEC_BF16 && c <= LPAR_CODEC_MXFP4; }
 static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static inline lpar_status_t launch_status() {
@@ -588,6 +607,7 @@ LPAR_API size_t lpar_tile_bytes(lpar_codec_t codec) {
     case LPAR_CODEC_FP8_E4M3: return Layout<kFP8>::kTileBytes;
     case LPAR_CODEC_INT4: return Layout<kINT4>::kTileBytes;
     case LPAR_CODEC_INT3: return Layout<kINT3>::kTileBytes;
+    case LPAR_CODEC_MXFP4: return Layout<kMXFP4>::kTileBytes;
     default: return 0;
     }
 }

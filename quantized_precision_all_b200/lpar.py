@@ -16,8 +16,9 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblpar.so")
 
-LPAR_CODEC_BF16, LPAR_CODEC_FP8_E4M3, LPAR_CODEC_INT4, LPAR_CODEC_INT3 = 0, 1, 2, 3
-CODECS = {"bf16": LPAR_CODEC_BF16, "fp8": LPAR_CODEC_FP8_E4M3, "int4": LPAR_CODEC_INT4, "int3": LPAR_CODEC_INT3}
+LPAR_CODEC_BF16, LPAR_CODEC_FP8_E4M3, LPAR_CODEC_INT4, LPAR_CODEC_INT3, LPAR_CODEC_MXFP4 = 0, 1, 2, 3, 4
+CODECS = {"bf16": LPAR_CODEC_BF16, "fp8": LPAR_CODEC_FP8_E4M3, "int4": LPAR_CODEC_INT4, "int3": LPAR_CODEC_INT3,
+          "mxfp4": LPAR_CODEC_MXFP4}
 CODEC_NAMES = {v: k for k, v in CODECS.items()}
 LPAR_SCHEDULE_AUTO, LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE, LPAR_SCHEDULE_SINGLE_PASS = 0, 1, 2, 3
 SCHEDULES = {"auto": LPAR_SCHEDULE_AUTO, "fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE,

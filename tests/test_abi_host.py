@@ -46,6 +46,7 @@ def test_tile_and_wire_sizes(L):
     assert L.lpar_tile_bytes("int3") == 896
     assert L.lpar_tile_bytes("fp8") == 2304
     assert L.lpar_tile_bytes("bf16") == 4096
+    assert L.lpar_tile_bytes("mxfp4") == 1088
     assert L.lpar_tile_bytes(7) == 0
     assert L.lpar_wire_bytes("int3", 2048 * 3) == 3 * 896
     assert L.lpar_wire_bytes("int4", 2048 * 5 + 100) == 5 * 1152
@@ -59,6 +60,7 @@ def test_workspace_bytes(L):
     assert L.lpar_workspace_bytes(8, n, "fp8") == 9 * 10 * 2304
     assert L.lpar_workspace_bytes(2, n, "int3") == 3 * 10 * 896
     assert L.lpar_workspace_bytes(4, n, "bf16") == 2 * n
+    assert L.lpar_workspace_bytes(3, n, "mxfp4") == 4 * 10 * 1088
     assert L.lpar_workspace_bytes(0, n, "int4") == 0
     assert L.lpar_workspace_bytes(9, n, "int4") == 0
 

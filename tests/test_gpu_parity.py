@@ -17,8 +17,8 @@ pytestmark = pytest.mark.gpu
 
 GUARD = 4096
 CANARY = 0xA5
-CODECS = ("int4", "int3", "fp8", "bf16")
-QCODECS = ("int4", "int3", "fp8")
+CODECS = ("int4", "int3", "fp8", "mxfp4", "bf16")
+QCODECS = ("int4", "int3", "fp8", "mxfp4")
 
 
 @pytest.fixture(scope="module")
@@ -70,7 +70,8 @@ def f16_value(bits):
 # ---------------------------------------------------------------------------
 # Adversarial BF16 inputs (seeded): block kinds cycle through random normal at
 # random scales, all-zero, single outliers, exact ties of the INT grids,
-# saturating magnitudes, tiny magnitudes (subnormal scales), negative zeros.
+# saturating magnitudes, tiny magnitudes (subnormal scales), negative zeros,
+# E4M3 and E2M1 grid points, midpoints and saturation.
 # ---------------------------------------------------------------------------
 def bf16(x):
     return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
@@ -80,7 +81,7 @@ def adversarial_bf16(n, seed):
     rng = np.random.default_rng(seed)
     nb = n // 32
     x = np.zeros((nb, 32), np.float32)
-    kinds = rng.integers(0, 9, nb)
+    kinds = rng.integers(0, 10, nb)
     for b in range(nb):
         k = kinds[b]
         if k == 0:
@@ -104,6 +105,13 @@ def adversarial_bf16(n, seed):
         elif k == 7:
             x[b] = -0.0
             x[b, rng.integers(32)] = rng.standard_normal()
+        elif k == 9:
+            # MXFP4 ties and saturation: E2M1 grid points, midpoints and values in
+            # (6, 8) at a power-of-two scale, some with tiny (E8M0-clamped) scales
+            e = rng.integers(-20, 20) if rng.random() < 0.8 else rng.integers(-140, -126)
+            grid = np.array([0, 0.25, 0.5, 0.75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 7], np.float32)
+            x[b] = rng.choice(grid, 32) * rng.choice([-1, 1], 32) * 2.0 ** e
+            x[b, rng.integers(32)] = rng.choice([4.0, 6.0, 7.5]) * 2.0 ** e
         else:
             # FP8 ties and saturation: E4M3 grid points and midpoints at a power-of-two scale
             e = rng.integers(-20, 20)
@@ -173,14 +181,17 @@ def test_decode_matches_oracle(L, codec):
     assert np.array_equal(host_u16(out), O.decode(wire, n, codec))
 
 
-@pytest.mark.parametrize("codec", ["int4", "int3"])
+@pytest.mark.parametrize("codec", ["int4", "int3", "mxfp4"])
 def test_decode_arbitrary_code_bytes(L, codec):
-    # any code byte pattern is a valid INT code; keep scales finite
+    # any code byte pattern is a valid INT or E2M1 code; keep scales finite
     n = 2048 * 6
     rng = np.random.default_rng(32)
     wire = rng.integers(0, 256, L.lpar_wire_bytes(codec, n), dtype=np.uint8)
     tb = L.lpar_tile_bytes(codec)
     for t in range(n // 2048):
+        if codec == "mxfp4":                              # E8M0 bytes 0..254 (255 is NaN)
+            wire[t * tb + 1024:t * tb + tb] = rng.integers(0, 255, 64).astype(np.uint8)
+            continue
         sc = rng.integers(0, 0x7C00, 64).astype(np.uint16) | (rng.integers(0, 2, 64).astype(np.uint16) << 15)
         wire[t * tb + tb - 128:t * tb + tb] = sc.view(np.uint8)
     dw = Guarded(wire.size)
@@ -277,6 +288,52 @@ def test_fp8_subnormal_products_and_inputs(L, N):
     L.lpar_quantize(dx.ptr(), n, "fp8", dw.ptr())
     torch.cuda.synchronize()
     assert np.array_equal(dw.host(), wire)
+
+
+@pytest.mark.parametrize("entry", ["reduce", "allreduce"])
+def test_mxfp4_stage_two_ties_and_tiny_sums(L, entry):
+    # rank 0 sits on the E2M1 grid at 2^E with absmax 6 * 2^E; rank 1 holds
+    # 0, +-0.25, +-0.5 times 2^E (its own absmax 0.5 * 2^E, so its grid reaches
+    # 0.25 * 2^E).  The sums 0.75, 1.25, 1.75, 2.5, 3.5 (times 2^E) are E2M1
+    # midpoints of the requantisation; some blocks use scales near 2^-127 so
+    # the dequantised values and sums are subnormal.
+    rng = np.random.default_rng(61)
+    n = 2048 * 4
+    x0 = np.zeros(n, np.float32)
+    x1 = np.zeros(n, np.float32)
+    g0 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    for b in range(n // 32):
+        E = rng.integers(-12, 12) if b % 4 else rng.integers(-128, -121)
+        a = rng.choice(g0, 32) * rng.choice([-1, 1], 32)
+        c = rng.choice(np.array([0, 0.25, 0.5], np.float32), 32) * rng.choice([-1, 1], 32)
+        a[0], c[0] = 6.0, 0.0
+        c[1] = 0.5
+        x0[b * 32:(b + 1) * 32] = a * 2.0 ** E
+        x1[b * 32:(b + 1) * 32] = c * 2.0 ** E
+    xs = [bf16(x0), bf16(x1)]
+    assert all(np.array_equal(O.bf16_bits_to_f32(b16), x) for b16, x in zip(xs, (x0, x1)))
+    if entry == "reduce":
+        wires = [O.quantize(x, "mxfp4") for x in xs]
+        dws = []
+        for w in wires:
+            g = Guarded(w.size)
+            g.t.copy_(torch.from_numpy(w))
+            dws.append(g)
+        out = Guarded(wires[0].size)
+        L.lpar_reduce([g.ptr() for g in dws], 0, n // 2048, "mxfp4", out.ptr())
+        torch.cuda.synchronize()
+        assert np.array_equal(out.host(), O.reduce(wires, 0, n // 2048, "mxfp4"))
+    else:
+        outs, _ = run_allreduce(L, xs, "mxfp4")
+        ref, _ = O.allreduce(xs, "mxfp4")
+        for o in outs:
+            assert np.array_equal(o, ref[0])
+    # the construction produced midpoints of the E2M1 grid: a block's sum has
+    # absmax in [6, 6.5] * 2^E, so the requantisation divides by 2^E
+    sums = (x0 + x1).reshape(-1, 32).astype(np.float64)
+    amax = np.max(np.abs(sums), axis=1, keepdims=True)
+    scaled = np.abs(sums) / 2.0 ** (np.floor(np.log2(amax)) - 2)
+    assert np.count_nonzero(np.isin(scaled, [0.75, 1.25, 1.75, 2.5, 3.5])) > n // 10
 
 
 @pytest.mark.parametrize("bits,codec", [(4, "int4"), (3, "int3")])
@@ -446,11 +503,13 @@ def test_workload_prefill_fp8_full_oracle_and_error_report(L):
     assert errs["bf16"][1] <= errs["fp8"][1]
 
 
-def test_workload_large_sampled_tiles(L):
-    """1 GiB per rank, INT3 then INT4, in the launch configuration the bench times;
-    compared on 1024 seeded random tiles plus the first and the last (tiles are
-    independent, so a tile's result depends only on that tile of every rank)."""
-    w = W.WORKLOADS["large_int3_int4"]
+@pytest.mark.parametrize("name", ["large_int3_int4", "large_mxfp4"])
+def test_workload_large_sampled_tiles(L, name):
+    """1 GiB per rank (INT3 then INT4, or MXFP4) in the launch configuration the
+    bench times; compared on 1024 seeded random tiles plus the first and the
+    last (tiles are independent, so a tile's result depends only on that tile
+    of every rank)."""
+    w = W.WORKLOADS[name]
     xs = W.make_inputs(w, "cuda")
     T = w.n // 2048
     rng = np.random.default_rng(4)

@@ -62,6 +62,10 @@ WORKLOADS = {
              "INT3 then INT4 back to back"),
 }
 
+WORKLOADS["large_mxfp4"] = Workload(
+    "large_mxfp4", N=2, n=512 * 1024 * 1024, dist="normal", sigma=0.02, seed=4, codecs=("mxfp4",),
+    note="large message, FP4 mode: N=2 x 512 Mi BF16 (1 GiB per rank), N(0, 0.02^2), MXFP4")
+
 # A smaller case of the large workload for ncu captures: inputs (256 MiB) still
 # exceed the 126 MB L2, while the whole footprint stays under 1 GiB.
 PROFILE_WORKLOADS = {
@@ -74,7 +78,7 @@ WORKLOADS.update(PROFILE_WORKLOADS)
 
 SWEEP_SIZES_BYTES = [1 << k for k in range(17, 31)]    # 128 KiB ... 1 GiB per rank
 SWEEP_RANKS = (2, 4, 8)
-SWEEP_CODECS = ("bf16", "fp8", "int4", "int3")
+SWEEP_CODECS = ("bf16", "fp8", "int4", "int3", "mxfp4")
 
 
 def sweep_workload(N: int, message_bytes: int, codec: str) -> Workload:
