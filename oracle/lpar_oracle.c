@@ -499,3 +499,132 @@ int orc_allreduce(const uint16_t *const *in_bf16, int N, size_t n, int codec,
     free(gather);
     return codec;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Standalone low-precision collectives ([RX] Low-Precision Collectives: the   */
+/* quantised wire is used by the other collectives too) and the one-shot       */
+/* all-reduce ([RX] Direct Data Access, "flat": every rank reduces all inputs  */
+/* itself).  Each rank's message is quantised once (stage 1); the receiver     */
+/* dequantises.  A reduction sums in binary32 in ascending rank order from     */
+/* +0.0f and rounds the sum once to BF16 (no second quantisation: nothing is   */
+/* transmitted after it).                                                       */
+/* ------------------------------------------------------------------------- */
+
+/* Quantise every rank's message (or copy it for BF16) into freshly allocated
+ * wires; returns 0 on success. */
+static int quantize_all(const uint16_t *const *in_bf16, int N, size_t n, int codec, uint8_t **wires)
+{
+    size_t wb = orc_wire_bytes(codec, n);
+    for (int r = 0; r < N; ++r) {
+        wires[r] = (uint8_t *)malloc(wb ? wb : 1);
+        if (!wires[r]) { for (int k = 0; k < r; ++k) free(wires[k]); return -1; }
+        if (codec == ORC_BF16) memcpy(wires[r], in_bf16[r], wb);
+        else orc_quantize(in_bf16[r], n, codec, wires[r]);
+    }
+    return 0;
+}
+
+/* BF16 sum of tile t over the N wires (acc from +0.0f, ranks ascending). */
+static void reduce_tile_to_bf16(uint8_t *const *wires, int N, size_t t, int codec, uint16_t *dst)
+{
+    float acc[ORC_TILE_ELEMS], v[ORC_TILE_ELEMS];
+    size_t tb = orc_tile_bytes(codec);
+    for (int i = 0; i < ORC_TILE_ELEMS; ++i) acc[i] = +0.0f;
+    for (int r = 0; r < N; ++r) {
+        orc_dequant_tile(wires[r] + t * tb, codec, v);
+        for (int i = 0; i < ORC_TILE_ELEMS; ++i) acc[i] = acc[i] + v[i];
+    }
+    for (int i = 0; i < ORC_TILE_ELEMS; ++i) dst[i] = orc_f32_to_bf16_rne(acc[i]);
+}
+
+static int effective(int codec, size_t message_bytes, size_t min_quant_bytes)
+{
+    return (codec != ORC_BF16 && message_bytes < min_quant_bytes) ? ORC_BF16 : codec;
+}
+
+/*
+ * Reduce-scatter: rank j receives tiles [jT/N, (j+1)T/N) of the sum (the same
+ * floor partition as the all-reduce's shards), as BF16, in out_bf16[j] from
+ * element 0.  Threshold on the per-rank message 2n.
+ */
+int orc_reduce_scatter(const uint16_t *const *in_bf16, int N, size_t n, int codec,
+                       uint16_t *const *out_bf16, size_t min_quant_bytes)
+{
+    if (N < 1 || N > ORC_MAX_RANKS || n % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
+    codec = effective(codec, 2 * n, min_quant_bytes);
+    uint8_t *wires[ORC_MAX_RANKS];
+    if (quantize_all(in_bf16, N, n, codec, wires)) return -1;
+    size_t T = n / ORC_TILE_ELEMS;
+    for (int j = 0; j < N; ++j) {
+        size_t t0 = (size_t)j * T / (size_t)N, t1 = (size_t)(j + 1) * T / (size_t)N;
+        for (size_t t = t0; t < t1; ++t)
+            reduce_tile_to_bf16(wires, N, t, codec, out_bf16[j] + (t - t0) * ORC_TILE_ELEMS);
+    }
+    for (int r = 0; r < N; ++r) free(wires[r]);
+    return codec;
+}
+
+/* One-shot all-reduce: every rank receives the whole BF16 sum. */
+int orc_allreduce_oneshot(const uint16_t *const *in_bf16, int N, size_t n, int codec,
+                          uint16_t *const *out_bf16, size_t min_quant_bytes)
+{
+    if (N < 1 || N > ORC_MAX_RANKS || n % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
+    codec = effective(codec, 2 * n, min_quant_bytes);
+    uint8_t *wires[ORC_MAX_RANKS];
+    if (quantize_all(in_bf16, N, n, codec, wires)) return -1;
+    for (size_t t = 0; t < n / ORC_TILE_ELEMS; ++t)
+        for (int r = 0; r < N; ++r)
+            reduce_tile_to_bf16(wires, N, t, codec, out_bf16[r] + t * ORC_TILE_ELEMS);
+    for (int r = 0; r < N; ++r) free(wires[r]);
+    return codec;
+}
+
+/*
+ * All-gather: rank r contributes m elements; every rank j receives all N
+ * contributions, rank r's at elements [r*m, (r+1)*m) of out_bf16[j], each the
+ * BF16 decode of rank r's wire.  Threshold on the per-rank message 2m.
+ */
+int orc_all_gather(const uint16_t *const *in_bf16, int N, size_t m, int codec,
+                   uint16_t *const *out_bf16, size_t min_quant_bytes)
+{
+    if (N < 1 || N > ORC_MAX_RANKS || m % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
+    codec = effective(codec, 2 * m, min_quant_bytes);
+    uint8_t *wires[ORC_MAX_RANKS];
+    if (quantize_all(in_bf16, N, m, codec, wires)) return -1;
+    for (int r = 0; r < N; ++r)
+        for (int j = 0; j < N; ++j) {
+            if (codec == ORC_BF16) memcpy(out_bf16[j] + (size_t)r * m, wires[r], 2 * m);
+            else orc_decode(wires[r], m, codec, out_bf16[j] + (size_t)r * m);
+        }
+    for (int r = 0; r < N; ++r) free(wires[r]);
+    return codec;
+}
+
+/*
+ * All-to-all: rank r's message is N segments of m elements, segment j bound
+ * for rank j; rank j receives rank r's segment j at elements [r*m, (r+1)*m)
+ * of out_bf16[j], the BF16 decode of that part of rank r's wire.  Threshold
+ * on the per-rank message 2*N*m.
+ */
+int orc_all_to_all(const uint16_t *const *in_bf16, int N, size_t m, int codec,
+                   uint16_t *const *out_bf16, size_t min_quant_bytes)
+{
+    if (N < 1 || N > ORC_MAX_RANKS || m % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
+    size_t n = (size_t)N * m;
+    codec = effective(codec, 2 * n, min_quant_bytes);
+    uint8_t *wires[ORC_MAX_RANKS];
+    if (quantize_all(in_bf16, N, n, codec, wires)) return -1;
+    size_t seg_wire = orc_wire_bytes(codec, m);
+    for (int r = 0; r < N; ++r)
+        for (int j = 0; j < N; ++j) {
+            const uint8_t *seg = wires[r] + (size_t)j * seg_wire;
+            if (codec == ORC_BF16) memcpy(out_bf16[j] + (size_t)r * m, seg, 2 * m);
+            else orc_decode(seg, m, codec, out_bf16[j] + (size_t)r * m);
+        }
+    for (int r = 0; r < N; ++r) free(wires[r]);
+    return codec;
+}

@@ -57,6 +57,16 @@ void orc_decode(const uint8_t *wire, size_t n, int codec, uint16_t *out_bf16);
 int  orc_allreduce(const uint16_t *const *in_bf16, int N, size_t n, int codec,
                    uint16_t *const *out_bf16, size_t min_quant_bytes);
 
+/* standalone collectives and the one-shot all-reduce (return the codec used, or -1) */
+int orc_reduce_scatter(const uint16_t *const *in_bf16, int N, size_t n, int codec,
+                       uint16_t *const *out_bf16, size_t min_quant_bytes);
+int orc_allreduce_oneshot(const uint16_t *const *in_bf16, int N, size_t n, int codec,
+                          uint16_t *const *out_bf16, size_t min_quant_bytes);
+int orc_all_gather(const uint16_t *const *in_bf16, int N, size_t m, int codec,
+                   uint16_t *const *out_bf16, size_t min_quant_bytes);
+int orc_all_to_all(const uint16_t *const *in_bf16, int N, size_t m, int codec,
+                   uint16_t *const *out_bf16, size_t min_quant_bytes);
+
 #ifdef __cplusplus
 }
 #endif

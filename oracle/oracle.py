@@ -58,6 +58,14 @@ def lib():
             "orc_decode": (None, [u8p, sz, ctypes.c_int, u16p]),
             "orc_allreduce": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
                                              ctypes.POINTER(u16p), sz]),
+            "orc_reduce_scatter": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
+                                                  ctypes.POINTER(u16p), sz]),
+            "orc_allreduce_oneshot": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
+                                                     ctypes.POINTER(u16p), sz]),
+            "orc_all_gather": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
+                                              ctypes.POINTER(u16p), sz]),
+            "orc_all_to_all": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
+                                              ctypes.POINTER(u16p), sz]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -229,3 +237,45 @@ def allreduce(inputs_bf16, codec, min_quant_bytes=0):
 def bf16_bits_to_f32(bits):
     """Vectorised exact widening of BF16 bit patterns (numpy, no rounding)."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _collective(fn, inputs_bf16, codec, out_sizes, size_arg, min_quant_bytes):
+    ins = [np.ascontiguousarray(x, dtype=np.uint16).reshape(-1) for x in inputs_bf16]
+    outs = [np.zeros(k, np.uint16) for k in out_sizes]
+    ia = (ctypes.POINTER(ctypes.c_uint16) * len(ins))(*[_ptr(x, ctypes.c_uint16) for x in ins])
+    oa = (ctypes.POINTER(ctypes.c_uint16) * len(outs))(*[_ptr(o, ctypes.c_uint16) for o in outs])
+    used = fn(ia, len(ins), size_arg, _codec(codec), oa, min_quant_bytes)
+    if used < 0:
+        raise ValueError("oracle rejected the arguments")
+    return outs, {v: k for k, v in CODECS.items()}[used]
+
+
+def shard_tiles(N, T):
+    """Tile range [t0, t1) of shard j for j = 0..N-1 (floor partition)."""
+    return [(j * T // N, (j + 1) * T // N) for j in range(N)]
+
+
+def reduce_scatter(inputs_bf16, codec, min_quant_bytes=0):
+    """Rank j gets its shard of the BF16 sum; returns (outputs, codec used)."""
+    n = np.asarray(inputs_bf16[0]).size
+    sizes = [(t1 - t0) * TILE_ELEMS for t0, t1 in shard_tiles(len(inputs_bf16), n // TILE_ELEMS)]
+    return _collective(lib().orc_reduce_scatter, inputs_bf16, codec, sizes, n, min_quant_bytes)
+
+
+def allreduce_oneshot(inputs_bf16, codec, min_quant_bytes=0):
+    n = np.asarray(inputs_bf16[0]).size
+    return _collective(lib().orc_allreduce_oneshot, inputs_bf16, codec, [n] * len(inputs_bf16), n,
+                       min_quant_bytes)
+
+
+def all_gather(inputs_bf16, codec, min_quant_bytes=0):
+    """Each of N ranks contributes m elements; every rank gets all N * m."""
+    N, m = len(inputs_bf16), np.asarray(inputs_bf16[0]).size
+    return _collective(lib().orc_all_gather, inputs_bf16, codec, [N * m] * N, m, min_quant_bytes)
+
+
+def all_to_all(inputs_bf16, codec, min_quant_bytes=0):
+    """Each rank's N * m elements are N segments of m, segment j bound for rank j."""
+    N = len(inputs_bf16)
+    m = np.asarray(inputs_bf16[0]).size // N
+    return _collective(lib().orc_all_to_all, inputs_bf16, codec, [N * m] * N, m, min_quant_bytes)
