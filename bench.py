@@ -377,6 +377,78 @@ def run_sweep(args, device):
             torch.cuda.empty_cache()
 
 
+COLL_OPS = ("reduce_scatter", "one_shot", "all_gather", "all_to_all")
+COLL_SIZES_BYTES = (16 << 20, 256 << 20)             # per-rank message
+
+
+def collective_bytes(op, codec, N, size):
+    """Algorithmic HBM bytes of one collective call.  size = elements of the size
+    argument (reduce-scatter / one-shot: n per rank; all-gather: m per rank;
+    all-to-all: m per segment, N * m per rank).  Quantising codecs: the N
+    messages are read and their wires written; reductions read the N wires back
+    and write one (reduce-scatter) or N (one-shot) BF16 results; all-gather and
+    all-to-all decode from the encoder's registers and write the outputs."""
+    c = CODEC_C[codec]
+    msg = N * size if op == "all_to_all" else size        # per-rank message, elements
+    out = {"reduce_scatter": 2 * size, "one_shot": N * 2 * size,
+           "all_gather": N * N * 2 * size, "all_to_all": N * N * 2 * size}[op]
+    if codec == "bf16":
+        return N * 2 * msg + out
+    stage1 = N * msg * (2 + c)
+    back = N * msg * c if op in ("reduce_scatter", "one_shot") else 0
+    return stage1 + back + out
+
+
+def run_collectives(args, device):
+    """One JSON line per (op, N, message size, codec) of the standalone
+    collectives and the one-shot all-reduce: GB/s (N x per-rank message bytes
+    / time) and the fraction of measured HBM peak (algorithmic bytes / time)."""
+    from quantized_precision_all_b200 import lpar as L
+    peak, _ = measured_peaks()
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for op in COLL_OPS:
+        for N in (2, 4, 8):
+            for mb in COLL_SIZES_BYTES:
+                msg = mb // 2
+                size = msg // N if op == "all_to_all" else msg
+                w = W.Workload("collective", N=N, n=msg, dist="student_t", nu=3, seed=9, codecs=("bf16",))
+                xs = W.make_inputs(w, device)
+                out_elems = N * size if op in ("all_gather", "all_to_all") else msg
+                outs = [torch.empty(out_elems, dtype=torch.bfloat16, device=device) for _ in range(N)]
+                ws = torch.empty(max(L.lpar_workspace_bytes(N, msg, c) for c in W.SWEEP_CODECS),
+                                 dtype=torch.uint8, device=device)
+
+                def call(codec):
+                    if op == "one_shot":
+                        L.lpar_allreduce(xs, msg, codec, outs, ws, ws.numel(), schedule="one_shot", stream=stream)
+                    else:
+                        src = [x[:size] for x in xs] if op == "all_gather" else xs
+                        getattr(L, "lpar_" + op)(src, size, codec, outs, ws, ws.numel(), stream=stream)
+
+                for codec in W.SWEEP_CODECS:
+                    for _ in range(3):
+                        call(codec)
+                    iters = 10
+                    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                           for _ in range(iters)]
+                    for e0, e1 in evs:
+                        flush.fill_(1)
+                        e0.record(stream)
+                        call(codec)
+                        e1.record(stream)
+                    torch.cuda.synchronize(device)
+                    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+                    alg = collective_bytes(op, codec, N, size)
+                    print(json.dumps({"collective": op, "N": N, "message_bytes": mb, "codec": codec, "ms": ms,
+                                      "GBps": N * mb / (ms * 1e-3) / 1e9,
+                                      "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
+                                      "algorithmic_bytes": alg, "peak": peak,
+                                      "l2": "256 MiB buffer rewritten before every timed call"}), flush=True)
+                del xs, outs, ws
+                torch.cuda.empty_cache()
+
+
 def workload_config(w, args):
     return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n,
             "message_bytes_per_rank": 2 * w.n, "codecs": list(w.codecs), "schedule": args.schedule,
@@ -397,6 +469,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
+    ap.add_argument("--collectives", action="store_true",
+                    help="one JSON line per standalone collective point instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.schedule == "auto":                # what the library picks for LPAR_SCHEDULE_AUTO
@@ -415,6 +489,9 @@ def main():
     torch.cuda.set_device(device)
     if args.sweep:
         run_sweep(args, device)
+        return
+    if args.collectives:
+        run_collectives(args, device)
         return
     if world > 1:
         import datetime

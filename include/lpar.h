@@ -103,10 +103,23 @@ typedef enum {
     LPAR_SCHEDULE_AUTO = 0,        /* the library's choice (currently LPAR_SCHEDULE_SINGLE_PASS) */
     LPAR_SCHEDULE_FUSED = 1,       /* quantise; reduce + requantise + decode in one kernel */
     LPAR_SCHEDULE_THREE_STAGE = 2, /* quantise; reduce + requantise; decode (three kernels) */
-    LPAR_SCHEDULE_SINGLE_PASS = 3  /* one kernel: each CTA quantises a chunk of every rank, then
+    LPAR_SCHEDULE_SINGLE_PASS = 3, /* one kernel: each CTA quantises a chunk of every rank, then
                                       reduces, requantises and decodes that chunk from the wires
                                       it has just written (same results, one launch) */
+    LPAR_SCHEDULE_ONE_SHOT = 4     /* a different algorithm, the one-shot ("flat") all-reduce of the
+                                      RCCLX page's Direct Data Access section: every rank reduces
+                                      all N stage-1 wires itself and rounds the FP32 sum once to
+                                      BF16, with no requantisation.  One quantisation stage instead
+                                      of two, so its results differ from the schedules above (they
+                                      equal lpar_reduce_scatter's, gathered). */
 } lpar_schedule_t;
+
+typedef enum {
+    LPAR_OP_ALLREDUCE = 0,
+    LPAR_OP_REDUCE_SCATTER = 1,
+    LPAR_OP_ALL_GATHER = 2,
+    LPAR_OP_ALL_TO_ALL = 3
+} lpar_collective_t;
 
 typedef struct {
     /* A quantising codec runs only when the per-rank message (2*n bytes) is at
@@ -160,10 +173,57 @@ lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec,
  * workspace: device memory of at least lpar_workspace_bytes(N, n, effective
  * codec) bytes, 16-byte aligned, contents ignored and overwritten.
  * opts may be NULL (always quantise, LPAR_SCHEDULE_AUTO).  Every schedule
- * gives the same bits. */
+ * gives the same bits, except LPAR_SCHEDULE_ONE_SHOT (a different algorithm,
+ * see lpar_schedule_t), which needs only N wires of the workspace. */
 lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                              void *const *out, void *workspace, size_t workspace_bytes,
                              const lpar_options_t *opts, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Standalone low-precision collectives (the RCCLX page's Low-Precision
+ * Collectives section: the quantised wire serves the other collectives too).
+ * Each rank's message is quantised once (stage 1) into a wire in the
+ * workspace; the receiver works from the wire.  No second quantisation: a
+ * reduction rounds its FP32 sum (ascending rank order from +0.0f) once to
+ * BF16.  Conventions as for lpar_allreduce (device buffers 16-byte aligned,
+ * host pointer arrays, asynchronous on `stream`, argument errors before any
+ * launch); outputs must not overlap the inputs, each other or the workspace.
+ * opts->min_quant_bytes applies to the per-rank message named below (smaller
+ * messages move the BF16 values themselves); opts->schedule is ignored;
+ * opts->stage_events[0] and [1] are recorded before and after the one kernel.
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes of a collective for the codec that runs (after the
+ * threshold): the all-reduce as lpar_workspace_bytes(N, size, codec); the
+ * others N wires of their per-rank message (reduce-scatter: n elements;
+ * all-gather: m; all-to-all: N * m), and 0 for BF16, when no workspace is
+ * needed and `workspace` may be NULL.  `size` is each call's size argument.
+ * 0 for N outside [1, LPAR_MAX_RANKS] or an unknown codec or op. */
+size_t lpar_collective_workspace_bytes(lpar_collective_t op, int N, size_t size, lpar_codec_t codec);
+
+/* Reduce-scatter of N BF16 messages of n elements (n a multiple of 2048): the
+ * T = n / 2048 tiles are split into N shards by the floor partition, shard j =
+ * tiles [j*T/N, (j+1)*T/N), and out[j] receives shard j of the BF16 sum from
+ * element 0 (so out[j] holds (floor((j+1)T/N) - floor(jT/N)) * 2048 values;
+ * an empty shard writes nothing).  Threshold on 2n bytes. */
+lpar_status_t lpar_reduce_scatter(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                                  void *const *out, void *workspace, size_t workspace_bytes,
+                                  const lpar_options_t *opts, cudaStream_t stream);
+
+/* All-gather: rank r contributes m elements (m a multiple of 2048); every
+ * out[j] (N * m values) receives rank r's contribution, decoded from rank r's
+ * wire, at elements [r*m, (r+1)*m).  Threshold on 2m bytes. */
+lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
+                              void *const *out, void *workspace, size_t workspace_bytes,
+                              const lpar_options_t *opts, cudaStream_t stream);
+
+/* All-to-all: inputs[r] holds N segments of m elements (m a multiple of 2048),
+ * segment j bound for rank j; out[j] (N * m values) receives rank r's segment
+ * j, decoded from rank r's wire, at elements [r*m, (r+1)*m).  Threshold on
+ * the whole per-rank message, 2*N*m bytes. */
+lpar_status_t lpar_all_to_all(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
+                              void *const *out, void *workspace, size_t workspace_bytes,
+                              const lpar_options_t *opts, cudaStream_t stream);
 
 /* Size of the workspace that lpar_allreduce_static keeps inside the library. */
 #define LPAR_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)

@@ -1,0 +1,431 @@
+// lpar_collectives.cu -- sm_100a kernels and C ABI of the standalone
+// low-precision collectives ("RCCLX: Innovating GPU communications on AMD
+// platforms", Low-Precision Collectives: the quantised wire carries the other
+// collectives too, compute stays in FP32) and of the one-shot all-reduce (its
+// Direct Data Access section: the flat algorithm, where every rank reduces all
+// inputs itself).
+//
+// Every collective quantises each rank's message once into that rank's wire
+// (the transmitted data, written to HBM), then:
+//   reduce-scatter   sums the dequantised wires of each tile in FP32 in rank
+//                    order from +0 and rounds once to BF16 into the tile's
+//                    shard owner (floor partition, as the all-reduce's shards)
+//   one-shot all-reduce   the same sum into every rank's output
+//   all-gather       decodes rank r's wire into every rank's output at r * m
+//   all-to-all       decodes segment j of rank r's wire into rank j's output at
+//                    r * m
+// The BF16 passthrough (below the threshold, or codec BF16) moves the BF16
+// values themselves.  Each quantising collective is one persistent kernel of
+// the single-pass shape (see lpar_kernels.cu): a CTA quantises a 4-tile chunk,
+// then reduces or decodes it while cp.async prefetches the next chunk.
+#include "lpar.h"
+#include "lpar_codec.cuh"
+#include "lpar_tiles.cuh"
+
+#include <algorithm>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lpar {
+
+// Floor partition of T tiles into N shards: shard j is [jT/N, (j+1)T/N), and
+// tile t belongs to shard ((t + 1) N - 1) / T (the largest j with jT/N <= t).
+__host__ __device__ __forceinline__ size_t shard_begin(int j, size_t T, int N) {
+    return (size_t)j * T / (size_t)N;
+}
+__host__ __device__ __forceinline__ int shard_of(size_t t, size_t T, int N) {
+    return (int)(((t + 1) * (size_t)N - 1) / T);
+}
+
+// Stage 1 of one rank's chunk from the staged BF16 (thread t's block) into the
+// wire; with WANT_V the decoded block also goes to `sink`.
+template <int C, bool WANT_V, class Sink>
+__device__ __forceinline__ void quantize_staged_block(const uint8_t *stage, uint8_t *wire_tile, int t,
+                                                      const Sink &sink) {
+    uint32_t x16[16];
+    stage_read(stage, t, x16);
+    float x[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
+    const float a = absmax_bf16x32(x16);
+    Packed<C> p;
+    encode<C, false, WANT_V>(x, a, p, sink);
+    store_block(wire_tile, t % kBlocksPerTile, p);
+}
+
+// ---------------------------------------------------------------------------
+// Reduce-scatter (ALL = false) and one-shot all-reduce (ALL = true), quantising
+// codecs.  Per chunk: stage 1 of every rank (prefetching the next rank's BF16
+// chunk), then each thread reads back the N wire blocks it wrote, sums them
+// and rounds to BF16; the staged chunk goes to the shard owners or to all.
+// ---------------------------------------------------------------------------
+template <int C, int N, bool ALL>
+__global__ void __launch_bounds__(kThreads, 4) k_reduce_bf16_single(const __grid_constant__ InPtrs in,
+                                                                    const __grid_constant__ OutPtrs wire,
+                                                                    const __grid_constant__ OutPtrs out,
+                                                                    size_t tiles, unsigned chunks) {
+    __shared__ __align__(128) uint8_t stage_in[2][kStageBytes];
+    __shared__ uint8_t *s_dst[kTilesPerCta];
+    const int t = threadIdx.x;
+    unsigned c = blockIdx.x;
+    if (c < chunks) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        stage_load_chunk(stage_in[0], in.p[0] + tile0 * (kTileElems * 2),
+                         (int)min((size_t)kTilesPerCta, tiles - tile0));
+    }
+    cp_async_commit();
+    int buf = 0;
+    for (; c < chunks; c += gridDim.x) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+        const bool active = t < ntiles * kBlocksPerTile;
+        const size_t tile = tile0 + t / kBlocksPerTile;
+        const int b = t % kBlocksPerTile;
+#pragma unroll 1
+        for (int r = 0; r < N; ++r) {
+            const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
+            if (cn < chunks) {
+                const size_t tn = (size_t)cn * kTilesPerCta;
+                stage_load_chunk(stage_in[buf ^ 1], in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
+                                 (int)min((size_t)kTilesPerCta, tiles - tn));
+            }
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncthreads();
+            if (active)
+                quantize_staged_block<C, false>(stage_in[buf], wire.p[r] + tile * Layout<C>::kTileBytes, t, NoSink{});
+            __syncthreads();                               // stage_in[buf] is refilled next
+            buf ^= 1;
+        }
+        // The buffer of the last rank's chunk is free until the next chunk's
+        // first prefetch (after the closing barrier): it stages the output.
+        uint8_t *stage_out = stage_in[buf ^ 1];
+        if (active) {
+            float acc[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = 0.0f;    // +0.0f, then ranks in ascending order
+#pragma unroll
+            for (int r = 0; r < N; ++r) {
+                Packed<C> p;
+                load_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
+                accumulate<C>(p, acc);
+            }
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = pack_bf16x2(acc[2 * k], acc[2 * k + 1]);
+            stage_write(stage_out, t, o);
+        }
+        if (!ALL && t < ntiles) {
+            const size_t tt = tile0 + t;
+            const int j = shard_of(tt, tiles, N);
+            s_dst[t] = out.p[j] + (tt - shard_begin(j, tiles, N)) * (kTileElems * 2);
+        }
+        __syncthreads();
+        if (ALL) stage_to_outputs(stage_out, out, N, tile0 * (kTileElems * 2), ntiles);
+        else stage_to_tile_dsts(stage_out, s_dst, ntiles);
+        __syncthreads();                                   // stage_out and s_dst are reused next chunk
+    }
+}
+
+// BF16 passthrough of the reductions: one tile (256 x 16 B) per CTA step, the
+// FP32 sum in rank order rounded once.  The shard owner advances with the
+// tile index (tiles are visited in increasing order), so no division per tile.
+template <int N, bool ALL>
+__global__ void __launch_bounds__(kThreads) k_bf16_reduce_to(const __grid_constant__ InPtrs in,
+                                                             const __grid_constant__ OutPtrs out, size_t tiles) {
+    const int t = threadIdx.x;
+    size_t tile = blockIdx.x;
+    if (tile >= tiles) return;
+    int j = ALL ? 0 : shard_of(tile, tiles, N);
+    size_t jb = ALL ? 0 : shard_begin(j, tiles, N), je = ALL ? 0 : shard_begin(j + 1, tiles, N);
+    for (; tile < tiles; tile += gridDim.x) {
+        if (!ALL) {
+            while (tile >= je) { ++j; jb = je; je = shard_begin(j + 1, tiles, N); }
+        }
+        const size_t off = tile * (kTileElems * 2) + 16 * (size_t)t;
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(in.p[r] + off);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc[2 * k] = __fadd_rn(acc[2 * k], bf16lo(w[k]));
+                acc[2 * k + 1] = __fadd_rn(acc[2 * k + 1], bf16hi(w[k]));
+            }
+        }
+        const uint4 o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                   pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        if (ALL) {
+#pragma unroll
+            for (int r = 0; r < N; ++r) *reinterpret_cast<uint4 *>(out.p[r] + off) = o;
+        } else {
+            *reinterpret_cast<uint4 *>(out.p[j] + (tile - jb) * (kTileElems * 2) + 16 * (size_t)t) = o;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// All-gather (A2A = false) and all-to-all (A2A = true), quantising codecs.
+// Work items (chunk c, rank r) of the ranks' messages (`tiles` tiles each);
+// the next item's BF16 chunk is prefetched while the current one is encoded.
+// The block's decoded values come from the encoder's registers (the value the
+// receiver decodes from the wire, which is written as the transmitted data).
+// seg_tiles is the segment length m / 2048 (all-gather: the whole message).
+// ---------------------------------------------------------------------------
+template <int C, bool A2A>
+__global__ void __launch_bounds__(kThreads, 4) k_gather_single(const __grid_constant__ InPtrs in,
+                                                               const __grid_constant__ OutPtrs wire,
+                                                               const __grid_constant__ OutPtrs out, size_t tiles,
+                                                               size_t seg_tiles, unsigned chunks, int N) {
+    __shared__ __align__(128) uint8_t stage_in[2][kStageBytes];
+    __shared__ uint8_t *s_dst[kTilesPerCta];
+    const int t = threadIdx.x;
+    unsigned c = blockIdx.x;
+    int r = 0;
+    if (c < chunks) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        stage_load_chunk(stage_in[0], in.p[0] + tile0 * (kTileElems * 2),
+                         (int)min((size_t)kTilesPerCta, tiles - tile0));
+    }
+    cp_async_commit();
+    int buf = 0;
+    while (c < chunks) {
+        unsigned cn = c;
+        int rn = r + 1;
+        if (rn == N) { rn = 0; cn += gridDim.x; }
+        if (cn < chunks) {
+            const size_t tn = (size_t)cn * kTilesPerCta;
+            stage_load_chunk(stage_in[buf ^ 1], in.p[rn] + tn * (kTileElems * 2),
+                             (int)min((size_t)kTilesPerCta, tiles - tn));
+        }
+        cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
+        // The decoded block replaces the thread's own input bytes in the same
+        // buffer: each thread reads its 64-B region in full before it writes it.
+        uint8_t *stage_out = stage_in[buf];
+        if (t < ntiles * kBlocksPerTile)
+            quantize_staged_block<C, true>(stage_in[buf],
+                                           wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t,
+                                           StageSink{stage_out, t});
+        if (A2A && t < ntiles) {
+            const size_t tt = tile0 + t;                   // tile of rank r's message
+            const size_t j = tt / seg_tiles;               // its segment = the receiving rank
+            s_dst[t] = out.p[j] + ((size_t)r * seg_tiles + (tt - j * seg_tiles)) * (kTileElems * 2);
+        }
+        __syncthreads();                                   // stage_out complete, stage_in[buf] consumed
+        if (A2A) stage_to_tile_dsts(stage_out, s_dst, ntiles);
+        else stage_to_outputs(stage_out, out, N, ((size_t)r * tiles + tile0) * (kTileElems * 2), ntiles);
+        __syncthreads();                                   // the buffer is refilled, s_dst rewritten, next item
+        buf ^= 1;
+        c = cn;
+        r = rn;
+    }
+}
+
+// BF16 passthrough of all-gather / all-to-all: copies, one tile of one rank per
+// CTA step (grid.y = rank).  The all-to-all segment advances with the tile.
+template <bool A2A>
+__global__ void __launch_bounds__(kThreads) k_bf16_gather(const __grid_constant__ InPtrs in,
+                                                          const __grid_constant__ OutPtrs out, size_t tiles,
+                                                          size_t seg_tiles, int N) {
+    const int t = threadIdx.x;
+    const int r = blockIdx.y;
+    size_t tile = blockIdx.x;
+    if (tile >= tiles) return;
+    size_t j = A2A ? tile / seg_tiles : 0, je = (j + 1) * seg_tiles;
+    for (; tile < tiles; tile += gridDim.x) {
+        const uint4 d = *reinterpret_cast<const uint4 *>(in.p[r] + tile * (kTileElems * 2) + 16 * (size_t)t);
+        if (A2A) {
+            while (tile >= je) { ++j; je += seg_tiles; }
+            const size_t dt = (size_t)r * seg_tiles + (tile - (je - seg_tiles));
+            *reinterpret_cast<uint4 *>(out.p[j] + dt * (kTileElems * 2) + 16 * (size_t)t) = d;
+        } else {
+            const size_t off = ((size_t)r * tiles + tile) * (kTileElems * 2) + 16 * (size_t)t;
+#pragma unroll
+            for (int k = 0; k < kMaxRanks; ++k)
+                if (k < N) *reinterpret_cast<uint4 *>(out.p[k] + off) = d;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (arguments validated by the callers).
+// ---------------------------------------------------------------------------
+static inline unsigned persistent_grid(unsigned chunks, unsigned resident) {
+    return std::min<unsigned>(chunks, std::max<unsigned>(1u, resident ? resident : 148u * 4u));
+}
+
+template <int C, int N, bool ALL>
+static void launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned grid = persistent_grid(chunks, resident_ctas(k_reduce_bf16_single<C, N, ALL>));
+    k_reduce_bf16_single<C, N, ALL><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, chunks);
+}
+
+template <int N, bool ALL>
+static void launch_rb_na(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles,
+                         cudaStream_t st) {
+    switch (codec) {
+    case kINT4: launch_rb_cna<kINT4, N, ALL>(in, wire, out, tiles, st); break;
+    case kINT3: launch_rb_cna<kINT3, N, ALL>(in, wire, out, tiles, st); break;
+    case kFP8: launch_rb_cna<kFP8, N, ALL>(in, wire, out, tiles, st); break;
+    case kMXFP4: launch_rb_cna<kMXFP4, N, ALL>(in, wire, out, tiles, st); break;
+    default: {
+        const unsigned grid = (unsigned)std::min<size_t>(tiles, (size_t)1 << 20);
+        k_bf16_reduce_to<N, ALL><<<grid, kThreads, 0, st>>>(in, out, tiles);
+    }
+    }
+}
+
+template <bool ALL>
+static void launch_rb_a(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
+                        cudaStream_t st) {
+    switch (N) {
+    case 1: launch_rb_na<1, ALL>(codec, in, wire, out, tiles, st); break;
+    case 2: launch_rb_na<2, ALL>(codec, in, wire, out, tiles, st); break;
+    case 3: launch_rb_na<3, ALL>(codec, in, wire, out, tiles, st); break;
+    case 4: launch_rb_na<4, ALL>(codec, in, wire, out, tiles, st); break;
+    case 5: launch_rb_na<5, ALL>(codec, in, wire, out, tiles, st); break;
+    case 6: launch_rb_na<6, ALL>(codec, in, wire, out, tiles, st); break;
+    case 7: launch_rb_na<7, ALL>(codec, in, wire, out, tiles, st); break;
+    case 8: launch_rb_na<8, ALL>(codec, in, wire, out, tiles, st); break;
+    default: break;
+    }
+}
+
+void launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
+                           size_t tiles, bool all, cudaStream_t st) {
+    if (all) launch_rb_a<true>(codec, in, wire, out, N, tiles, st);
+    else launch_rb_a<false>(codec, in, wire, out, N, tiles, st);
+}
+
+template <int C, bool A2A>
+static void launch_gather_c(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
+                            size_t seg_tiles, cudaStream_t st) {
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned grid = persistent_grid(chunks, resident_ctas(k_gather_single<C, A2A>));
+    k_gather_single<C, A2A><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, seg_tiles, chunks, N);
+}
+
+template <bool A2A>
+static void launch_gather(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
+                          size_t tiles, size_t seg_tiles, cudaStream_t st) {
+    switch (codec) {
+    case kINT4: launch_gather_c<kINT4, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
+    case kINT3: launch_gather_c<kINT3, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
+    case kFP8: launch_gather_c<kFP8, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
+    case kMXFP4: launch_gather_c<kMXFP4, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
+    default: {
+        const dim3 grid((unsigned)std::min<size_t>(tiles, (size_t)1 << 20), (unsigned)N);
+        k_bf16_gather<A2A><<<grid, kThreads, 0, st>>>(in, out, tiles, seg_tiles, N);
+    }
+    }
+}
+
+}  // namespace lpar
+
+using namespace lpar;
+
+// ---------------------------------------------------------------------------
+// The C ABI of the collectives.
+// ---------------------------------------------------------------------------
+LPAR_API size_t lpar_collective_workspace_bytes(lpar_collective_t op, int N, size_t n, lpar_codec_t codec) {
+    if (N < 1 || N > kMaxRanks || !codec_ok(codec)) return 0;
+    switch (op) {
+    case LPAR_OP_ALLREDUCE: return lpar_workspace_bytes(N, n, codec);
+    case LPAR_OP_REDUCE_SCATTER:
+    case LPAR_OP_ALL_GATHER: return codec == LPAR_CODEC_BF16 ? 0 : (size_t)N * lpar_wire_bytes(codec, n);
+    case LPAR_OP_ALL_TO_ALL: return codec == LPAR_CODEC_BF16 ? 0 : (size_t)N * lpar_wire_bytes(codec, (size_t)N * n);
+    default: return 0;
+    }
+}
+
+// Shared validation of the three collectives.  `n_msg` is the per-rank message
+// in elements (reduce-scatter: n; all-gather: m; all-to-all: N * m).
+static lpar_status_t collective_setup(lpar_collective_t op, const void *const *inputs, int N, size_t size,
+                                      lpar_codec_t codec, void *const *out, void *workspace,
+                                      size_t workspace_bytes, const lpar_options_t *opts, InPtrs &in, OutPtrs &o,
+                                      OutPtrs &wires, lpar_codec_t &eff, size_t &n_msg) {
+    if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
+    if (N < 1 || N > kMaxRanks || size % kTileElems != 0) return LPAR_ERR_INVALID_ARG;
+    if (size / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;   // also keeps N * size from wrapping
+    n_msg = op == LPAR_OP_ALL_TO_ALL ? (size_t)N * size : size;
+    if (n_msg / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
+    if (n_msg == 0) return LPAR_OK;
+    if (!inputs || !out) return LPAR_ERR_INVALID_ARG;
+    for (int r = 0; r < N; ++r) {
+        if (!inputs[r] || !out[r]) return LPAR_ERR_INVALID_ARG;
+        if (!aligned16(inputs[r]) || !aligned16(out[r])) return LPAR_ERR_MISALIGNED;
+        in.p[r] = static_cast<const uint8_t *>(inputs[r]);
+        o.p[r] = static_cast<uint8_t *>(out[r]);
+    }
+    eff = lpar_effective_codec(n_msg, codec, opts);
+    const size_t need = lpar_collective_workspace_bytes(op, N, size, eff);
+    if (need) {
+        if (!workspace) return LPAR_ERR_INVALID_ARG;
+        if (!aligned16(workspace)) return LPAR_ERR_MISALIGNED;
+        if (workspace_bytes < need) return LPAR_ERR_WORKSPACE_TOO_SMALL;
+        const size_t wb = lpar_wire_bytes(eff, n_msg);
+        for (int r = 0; r < N; ++r) wires.p[r] = static_cast<uint8_t *>(workspace) + (size_t)r * wb;
+    }
+    return LPAR_OK;
+}
+
+static inline void mark(const lpar_options_t *opts, int i, cudaStream_t stream) {
+    if (opts && opts->stage_events[i]) cudaEventRecord(opts->stage_events[i], stream);
+}
+
+LPAR_API lpar_status_t lpar_reduce_scatter(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                                           void *const *out, void *workspace, size_t workspace_bytes,
+                                           const lpar_options_t *opts, cudaStream_t stream) {
+    InPtrs in{};
+    OutPtrs o{}, wires{};
+    lpar_codec_t eff = codec;
+    size_t n_msg = 0;
+    const lpar_status_t st = collective_setup(LPAR_OP_REDUCE_SCATTER, inputs, N, n, codec, out, workspace,
+                                              workspace_bytes, opts, in, o, wires, eff, n_msg);
+    if (st != LPAR_OK || n_msg == 0) return st;
+    mark(opts, 0, stream);
+    launch_reduce_to_bf16(eff, in, wires, o, N, n / kTileElems, false, stream);
+    mark(opts, 1, stream);
+    return launch_status();
+}
+
+LPAR_API lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
+                                       void *const *out, void *workspace, size_t workspace_bytes,
+                                       const lpar_options_t *opts, cudaStream_t stream) {
+    InPtrs in{};
+    OutPtrs o{}, wires{};
+    lpar_codec_t eff = codec;
+    size_t n_msg = 0;
+    const lpar_status_t st = collective_setup(LPAR_OP_ALL_GATHER, inputs, N, m, codec, out, workspace,
+                                              workspace_bytes, opts, in, o, wires, eff, n_msg);
+    if (st != LPAR_OK || n_msg == 0) return st;
+    const size_t tiles = m / kTileElems;
+    mark(opts, 0, stream);
+    launch_gather<false>(eff, in, wires, o, N, tiles, tiles, stream);
+    mark(opts, 1, stream);
+    return launch_status();
+}
+
+LPAR_API lpar_status_t lpar_all_to_all(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
+                                       void *const *out, void *workspace, size_t workspace_bytes,
+                                       const lpar_options_t *opts, cudaStream_t stream) {
+    InPtrs in{};
+    OutPtrs o{}, wires{};
+    lpar_codec_t eff = codec;
+    size_t n_msg = 0;
+    const lpar_status_t st = collective_setup(LPAR_OP_ALL_TO_ALL, inputs, N, m, codec, out, workspace,
+                                              workspace_bytes, opts, in, o, wires, eff, n_msg);
+    if (st != LPAR_OK || n_msg == 0) return st;
+    mark(opts, 0, stream);
+    launch_gather<true>(eff, in, wires, o, N, n_msg / kTileElems, m / kTileElems, stream);
+    mark(opts, 1, stream);
+    return launch_status();
+}

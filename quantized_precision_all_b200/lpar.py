@@ -21,15 +21,18 @@ CODECS = {"bf16": LPAR_CODEC_BF16, "fp8": LPAR_CODEC_FP8_E4M3, "int4": LPAR_CODE
           "mxfp4": LPAR_CODEC_MXFP4}
 CODEC_NAMES = {v: k for k, v in CODECS.items()}
 LPAR_SCHEDULE_AUTO, LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE, LPAR_SCHEDULE_SINGLE_PASS = 0, 1, 2, 3
+LPAR_SCHEDULE_ONE_SHOT = 4
 SCHEDULES = {"auto": LPAR_SCHEDULE_AUTO, "fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE,
-             "single_pass": LPAR_SCHEDULE_SINGLE_PASS}
+             "single_pass": LPAR_SCHEDULE_SINGLE_PASS, "one_shot": LPAR_SCHEDULE_ONE_SHOT}
+OPS = {"allreduce": 0, "reduce_scatter": 1, "all_gather": 2, "all_to_all": 3}
 STATUS = {0: "LPAR_OK", 1: "LPAR_ERR_INVALID_ARG", 2: "LPAR_ERR_MISALIGNED",
           3: "LPAR_ERR_WORKSPACE_TOO_SMALL", 4: "LPAR_ERR_UNSUPPORTED", 5: "LPAR_ERR_CUDA"}
 TILE_ELEMS = 2048
 MAX_RANKS = 8
 
 EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
-           "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string")
+           "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string",
+           "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -59,6 +62,10 @@ def _load():
         "lpar_allreduce_static": (i32, [vpp, i32, sz, i32, vpp, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_effective_codec": (i32, [sz, i32, ctypes.POINTER(lpar_options_t)]),
         "lpar_status_string": (ctypes.c_char_p, [i32]),
+        "lpar_collective_workspace_bytes": (sz, [i32, i32, sz, i32]),
+        "lpar_reduce_scatter": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_all_gather": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_all_to_all": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -179,6 +186,38 @@ def lpar_status_string(status):
     return _lib.lpar_status_string(status).decode()
 
 
+def lpar_collective_workspace_bytes(op, N, size, codec):
+    return _lib.lpar_collective_workspace_bytes(OPS[op] if isinstance(op, str) else int(op), N, size, _codec(codec))
+
+
+def _collective(fn, name, inputs, size, codec, out, workspace, workspace_bytes, min_quant_bytes, stream, N,
+                stage_events):
+    ins = _ptr_array(inputs)
+    outs = _ptr_array(out)
+    N = len(inputs) if N is None else N
+    opts = _options(min_quant_bytes, "auto", stage_events)
+    _check(fn(ins[0] if ins else None, N, size, _codec(codec), outs[0] if outs else None, _ptr(workspace),
+              workspace_bytes, ctypes.byref(opts), _stream(stream)), name)
+
+
+def lpar_reduce_scatter(inputs, n, codec, out, workspace, workspace_bytes, min_quant_bytes=0, stream=None, N=None,
+                        stage_events=None):
+    _collective(_lib.lpar_reduce_scatter, "lpar_reduce_scatter", inputs, n, codec, out, workspace, workspace_bytes,
+                min_quant_bytes, stream, N, stage_events)
+
+
+def lpar_all_gather(inputs, m, codec, out, workspace, workspace_bytes, min_quant_bytes=0, stream=None, N=None,
+                    stage_events=None):
+    _collective(_lib.lpar_all_gather, "lpar_all_gather", inputs, m, codec, out, workspace, workspace_bytes,
+                min_quant_bytes, stream, N, stage_events)
+
+
+def lpar_all_to_all(inputs, m, codec, out, workspace, workspace_bytes, min_quant_bytes=0, stream=None, N=None,
+                    stage_events=None):
+    _collective(_lib.lpar_all_to_all, "lpar_all_to_all", inputs, m, codec, out, workspace, workspace_bytes,
+                min_quant_bytes, stream, N, stage_events)
+
+
 # ---- convenience: allocate with torch, then call the C ABI -----------------------
 def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedule="auto", stream=None):
     """All-reduce a list of N equal-size BF16 CUDA tensors; returns the N outputs."""
@@ -190,4 +229,48 @@ def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedu
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=inputs[0].device)
     lpar_allreduce(inputs, n, codec, out, workspace, workspace.numel(), min_quant_bytes, schedule, stream)
+    return out
+
+
+def shard_tiles(N, T):
+    """Tile range [t0, t1) of reduce-scatter shard j, j = 0..N-1 (floor partition)."""
+    return [(j * T // N, (j + 1) * T // N) for j in range(N)]
+
+
+def _workspace(op, N, size, codec, min_quant_bytes, device):
+    import torch
+    n_msg = N * size if op == "all_to_all" else size
+    need = lpar_collective_workspace_bytes(op, N, size, lpar_effective_codec(n_msg, codec, min_quant_bytes))
+    return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+
+
+def reduce_scatter(inputs, codec, min_quant_bytes=0, stream=None):
+    """Reduce-scatter of N equal-size BF16 CUDA tensors; returns the N shards."""
+    import torch
+    N, n = len(inputs), inputs[0].numel()
+    out = [torch.empty(max((t1 - t0) * TILE_ELEMS, 8), dtype=torch.bfloat16, device=inputs[0].device)
+           for t0, t1 in shard_tiles(N, n // TILE_ELEMS)]
+    ws = _workspace("reduce_scatter", N, n, codec, min_quant_bytes, inputs[0].device)
+    lpar_reduce_scatter(inputs, n, codec, out, ws, ws.numel(), min_quant_bytes, stream)
+    return [o[:(t1 - t0) * TILE_ELEMS] for o, (t0, t1) in zip(out, shard_tiles(N, n // TILE_ELEMS))]
+
+
+def all_gather(inputs, codec, min_quant_bytes=0, stream=None):
+    """All-gather of N BF16 CUDA tensors of m elements; returns N tensors of N * m."""
+    import torch
+    N, m = len(inputs), inputs[0].numel()
+    out = [torch.empty(N * m, dtype=torch.bfloat16, device=inputs[0].device) for _ in range(N)]
+    ws = _workspace("all_gather", N, m, codec, min_quant_bytes, inputs[0].device)
+    lpar_all_gather(inputs, m, codec, out, ws, ws.numel(), min_quant_bytes, stream)
+    return out
+
+
+def all_to_all(inputs, codec, min_quant_bytes=0, stream=None):
+    """All-to-all of N BF16 CUDA tensors of N * m elements (N segments of m)."""
+    import torch
+    N = len(inputs)
+    m = inputs[0].numel() // N
+    out = [torch.empty(N * m, dtype=torch.bfloat16, device=inputs[0].device) for _ in range(N)]
+    ws = _workspace("all_to_all", N, m, codec, min_quant_bytes, inputs[0].device)
+    lpar_all_to_all(inputs, m, codec, out, ws, ws.numel(), min_quant_bytes, stream)
     return out

@@ -136,6 +136,54 @@ def test_argument_errors_allreduce(L):
     assert lib.lpar_allreduce(None, 2, n, 2, None, A, ws, None, None) == 1
 
 
+def test_collective_workspace_bytes(L):
+    n = 2048 * 10
+    assert L.lpar_collective_workspace_bytes("allreduce", 2, n, "int4") == L.lpar_workspace_bytes(2, n, "int4")
+    assert L.lpar_collective_workspace_bytes("reduce_scatter", 3, n, "int3") == 3 * 10 * 896
+    assert L.lpar_collective_workspace_bytes("all_gather", 4, n, "mxfp4") == 4 * 10 * 1088
+    assert L.lpar_collective_workspace_bytes("all_to_all", 2, n, "fp8") == 2 * 20 * 2304
+    for op in ("reduce_scatter", "all_gather", "all_to_all"):
+        assert L.lpar_collective_workspace_bytes(op, 2, n, "bf16") == 0
+        assert L.lpar_collective_workspace_bytes(op, 9, n, "int4") == 0
+        assert L.lpar_collective_workspace_bytes(op, 2, n, 9) == 0
+    assert L.lpar_collective_workspace_bytes(7, 2, n, "int4") == 0
+
+
+@pytest.mark.parametrize("fn", ["lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all"])
+def test_argument_errors_collectives(L, fn):
+    call = getattr(L, fn)
+    op = fn[len("lpar_"):]
+    st = 0
+    n = 2048 * 4
+    ws = L.lpar_collective_workspace_bytes(op, 2, n, "int4")
+    assert status_of(call, [A, A], n, "int4", [A, A], A, ws - 16, stream=st) == 3
+    assert status_of(call, [A, A], n, "int4", [A, M], A, ws, stream=st) == 2
+    assert status_of(call, [M, A], n, "int4", [A, A], A, ws, stream=st) == 2
+    assert status_of(call, [A, A], n, "int4", [A, A], M, ws, stream=st) == 2
+    assert status_of(call, [A, 0], n, "int4", [A, A], A, ws, stream=st) == 1
+    assert status_of(call, [A, A], n, "int4", [A, A], 0, ws, stream=st) == 1      # workspace needed
+    assert status_of(call, [A, A], n + 1, "int4", [A, A], A, ws, stream=st) == 1
+    assert status_of(call, [A] * 9, n, "int4", [A] * 9, A, 10 ** 9, stream=st) == 1
+    assert status_of(call, [A, A], n, 11, [A, A], A, ws, stream=st) == 4
+    assert status_of(call, [A, A], 0, "int4", [A, A], 0, 0, stream=st) == 0       # empty: no-op
+    big = 2048 * (2 ** 33 + 1)
+    assert status_of(call, [A, A], big, "int4", [A, A], A, 10 ** 18, stream=st) == 1
+    assert status_of(call, [A] * 4, 2 ** 62, "int4", [A] * 4, A, 10 ** 18, stream=st) == 1   # 4 * 2^62 wraps
+    if op == "all_to_all":                                   # N * m above 2^44 although m is not
+        assert status_of(call, [A] * 4, 2 ** 43, "int4", [A] * 4, A, 2 ** 62, stream=st) == 1
+    lib = L.library()
+    opts = L.lpar_options_t(0, 0)
+    assert getattr(lib, fn)(None, 2, n, 2, None, A, ws, ctypes.byref(opts), None) == 1
+
+
+def test_one_shot_schedule_is_accepted_and_validated(L):
+    st = 0
+    n = 2048 * 4
+    ws = L.lpar_workspace_bytes(2, n, "int4")
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws - 16, schedule="one_shot", stream=st) == 3
+    assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws, schedule=5, stream=st) == 4
+
+
 def test_status_strings(L):
     for s in range(6):
         assert L.lpar_status_string(s)

@@ -43,7 +43,7 @@ class Guarded:
         return self.buf[GUARD:GUARD + self.nbytes]
 
     def ptr(self):
-        return self.t.data_ptr()
+        return self.buf.data_ptr() + GUARD          # also valid (and aligned) for an empty region
 
     def host(self):
         return self.t.cpu().numpy()
