@@ -343,22 +343,31 @@ __device__ __forceinline__ float add_sat(float a, float b) {
     return d;
 }
 
-// One element pair -> -q (q = RNE(x/s), see the header comment).
+// One element pair -> C3 = M + BIAS + q (q = RNE(x/s), see the header comment;
+// the offset BIAS is folded into the addend of the last step, which stays in
+// [2^23, 2^24), so the rounding is unchanged) and, when needed, -q.
 // STAGE2: clears bit 31 of `ok` when some q fails the exact verification.
-template <bool STAGE2>
-__device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, uint32_t &ok) {
-    const float2 r2 = splat(k.r), M2 = splat(kMagic), M4 = splat(kMagic2);
+template <bool STAGE2, bool WANT_NQ, int BIAS = 0>
+__device__ __forceinline__ float2 round_pair_c(float2 xv, const IntScale &k, uint32_t &ok, float2 &nq) {
+    const float2 r2 = splat(k.r), M4 = splat(kMagic2);
     const float2 C2 = fma2(xv, r2, M4);                // 2M + 2 k2 (exact product inside)
     const float2 nq2 = sub2(M4, C2);                   // -2 k2
-    const float2 B = sub2(C2, M2);                     // M + 2 k2
+    const float2 B = sub2(C2, splat(kMagic - (float)BIAS));   // M + BIAS + 2 k2
     const float2 f2 = fma2(xv, r2, nq2);               // x r - 2 k2
-    const float2 C3 = fma2(f2, splat(kEta), B);        // M + q
-    const float2 nq = sub2(M2, C3);                    // -q (exact)
+    const float2 C3 = fma2(f2, splat(kEta), B);        // M + BIAS + q
+    if (WANT_NQ || STAGE2) nq = sub2(splat(kMagic + (float)BIAS), C3);   // -q (exact)
     if (STAGE2) {
         const float2 e = fma2(nq, splat(k.s), xv);     // x - q s, exact
         const float2 d = fma2(e, e, splat(-k.t2));     // < 0 iff |e| <= s/2
         ok &= __float_as_uint(d.x) & __float_as_uint(d.y);
     }
+    return C3;
+}
+
+template <bool STAGE2>
+__device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, uint32_t &ok) {
+    float2 nq;
+    round_pair_c<STAGE2, true>(xv, k, ok, nq);
     return nq;
 }
 
@@ -392,41 +401,57 @@ __device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &
     return (ok >> 31) != 0u;
 }
 
-// INT3: lanes hold elements (16p + m, 16p + 8 + m).  hi = (q >= 0) =
-// clamp(1 + q, 0, 1) (one saturating add); low2 = q + 4 - 4 hi.  Chains (m = 7 .. 0) pack 8 elements per
-// lane: q2 bits Sum low2_m 4^m (16 bits), q1 bits Sum hi_m 2^m (8 bits).
+// INT3 from the integer bits of C3 = M + code (code = q + 4 in bits 0..2,
+// since M = 0x4B400000 as bits): lanes hold elements (4g + i, 16 + 4g + i).
+// PRMTs gather the code bytes of elements 4g..4g+3 into one word W_g, and two
+// multiplies move its bit fields into place without carries (every cross
+// term lands below the target byte, at distinct positions):
+//   (W & 0x03030303) * 0x01041040: byte 3 = the four low-2-bit fields (q2w);
+//   (W & 0x04040404) * 0x00408102: bits 24..27 = the four high bits (q1w),
+//   or * 0x04081020 for bits 28..31, so two groups combine with one OR.
+// Everything after the rounding runs on the integer ALU, not the FMA pipe.
+__device__ __forceinline__ uint32_t code_bytes4(float a, float b, float c, float d) {
+    return __byte_perm(__byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040),
+                       __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040), 0x5410);
+}
+
 template <bool STAGE2, bool WANT_V, class Sink>
 __device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &k, uint32_t (&q2w)[2],
                                           uint32_t &q1w, const Sink &sink) {
-    const float2 ns2 = splat(-k.s), M2 = splat(kMagic);
-    const float2 F4 = splat(4.f), F2 = splat(2.f);
+    const float2 ns2 = splat(-k.s);
     uint32_t ok = 0xFFFFFFFFu;
-    uint32_t q1b[2];
+    uint32_t lo[8], hi[8];
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        float2 Q = splat(0.f), R = splat(0.f);
+    for (int p = 0; p < 2; ++p) {                      // groups 2p, 2p+1: elements 8p..8p+7 and 16+8p..
         float2 v[8];
 #pragma unroll
-        for (int m = 7; m >= 0; --m) {
-            const float2 nq = round_pair<STAGE2>(make_float2(x[16 * p + m], x[16 * p + 8 + m]), k, ok);
-            const float2 hi = make_float2(add_sat(1.f, -nq.x), add_sat(1.f, -nq.y));   // (q >= 0)
-            const float2 u = fma2(hi, F4, nq);                      // 4 hi - q = 4 - low2
-            Q = fma2(Q, F4, u);
-            R = fma2(R, F2, hi);
-            if (WANT_V) v[m] = fma2(nq, ns2, splat(0.f));
+        for (int gg = 0; gg < 2; ++gg) {
+            const int g = 2 * p + gg;
+            float2 C[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float2 nq;
+                C[i] = round_pair_c<STAGE2, WANT_V, 4>(make_float2(x[4 * g + i], x[16 + 4 * g + i]), k, ok, nq);
+                if (WANT_V) v[4 * gg + i] = fma2(nq, ns2, splat(0.f));   // q s (+0 for q = 0)
+            }
+            const uint32_t W0 = code_bytes4(C[0].x, C[1].x, C[2].x, C[3].x);   // elements 4g .. 4g+3
+            const uint32_t W1 = code_bytes4(C[0].y, C[1].y, C[2].y, C[3].y);   // elements 16+4g ..
+            lo[g] = (W0 & 0x03030303u) * 0x01041040u;
+            lo[4 + g] = (W1 & 0x03030303u) * 0x01041040u;
+            hi[g] = (W0 & 0x04040404u) * ((g & 1) ? 0x04081020u : 0x00408102u);
+            hi[4 + g] = (W1 & 0x04040404u) * ((g & 1) ? 0x04081020u : 0x00408102u);
         }
-        const float2 P2 = sub2(splat(kMagic + 87380.0f), Q);       // 87380 = Sum_m 4 * 4^m
-        const float2 P1 = add2(R, M2);
-        q2w[p] = __byte_perm(__float_as_uint(P2.x), __float_as_uint(P2.y), 0x5410);
-        q1b[p] = __byte_perm(__float_as_uint(P1.x), __float_as_uint(P1.y), 0x0040);
-        if (WANT_V) {
-            sink.put(2 * p, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
-                                       pack_bf16x2(v[4].x, v[5].x), pack_bf16x2(v[6].x, v[7].x)));
-            sink.put(2 * p + 1, make_uint4(pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y),
-                                           pack_bf16x2(v[4].y, v[5].y), pack_bf16x2(v[6].y, v[7].y)));
+        if (WANT_V) {                                  // piece j = elements 8j .. 8j+7
+            sink.put(p, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
+                                   pack_bf16x2(v[4].x, v[5].x), pack_bf16x2(v[6].x, v[7].x)));
+            sink.put(2 + p, make_uint4(pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y),
+                                       pack_bf16x2(v[4].y, v[5].y), pack_bf16x2(v[6].y, v[7].y)));
         }
     }
-    q1w = __byte_perm(q1b[0], q1b[1], 0x5410);
+    q2w[0] = __byte_perm(__byte_perm(lo[0], lo[1], 0x0073), __byte_perm(lo[2], lo[3], 0x0073), 0x5410);
+    q2w[1] = __byte_perm(__byte_perm(lo[4], lo[5], 0x0073), __byte_perm(lo[6], lo[7], 0x0073), 0x5410);
+    q1w = __byte_perm(__byte_perm(hi[0] | hi[1], hi[2] | hi[3], 0x0073),
+                      __byte_perm(hi[4] | hi[5], hi[6] | hi[7], 0x0073), 0x5410);
     return (ok >> 31) != 0u;
 }
 

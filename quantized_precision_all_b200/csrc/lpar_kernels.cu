@@ -186,15 +186,17 @@ __global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_c
                                                                   uint8_t *gather,
                                                                   const __grid_constant__ OutPtrs out,
                                                                   size_t tiles, unsigned chunks) {
-    __shared__ __align__(128) uint8_t stage_in[2][kStageBytes];
-    __shared__ __align__(128) uint8_t stage_out[kStageBytes];
+    // A ring of three BF16 stages: the item in stage k is prefetched while the
+    // previous one is encoded, and stage k is refilled two items later, after
+    // a barrier that every thread passes only once done with it -- so one
+    // barrier per item.  The decoded chunk is staged in place of the last
+    // rank's input (each thread writes only the 64-B region it read).
+    __shared__ __align__(128) uint8_t stage[3][kStageBytes];
     const int t = threadIdx.x;
     unsigned c = blockIdx.x;
-    if (c < chunks) {
-        const size_t tile0 = (size_t)c * kTilesPerCta;
-        stage_load_chunk(stage_in[0], in.p[0] + tile0 * (kTileElems * 2),
-                         (int)min((size_t)kTilesPerCta, tiles - tile0));
-    }
+    if (c >= chunks) return;
+    stage_load_chunk(stage[0], in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
+                     (int)min((size_t)kTilesPerCta, tiles - (size_t)c * kTilesPerCta));
     cp_async_commit();
     int buf = 0;
     for (; c < chunks; c += gridDim.x) {
@@ -203,21 +205,23 @@ __global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_c
         const bool active = t < ntiles * kBlocksPerTile;
         const size_t tile = tile0 + t / kBlocksPerTile;
         const int b = t % kBlocksPerTile;
+        int last = buf;
 #pragma unroll 1
         for (int r = 0; r < N; ++r) {
             // prefetch the next item: rank r+1 of this chunk, or rank 0 of the next chunk
+            const int nb = buf == 2 ? 0 : buf + 1;
             const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
             if (cn < chunks) {
                 const size_t tn = (size_t)cn * kTilesPerCta;
-                stage_load_chunk(stage_in[buf ^ 1], in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
+                stage_load_chunk(stage[nb], in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
                                  (int)min((size_t)kTilesPerCta, tiles - tn));
             }
             cp_async_commit();
             cp_async_wait_prev();
-            __syncthreads();
+            __syncthreads();                           // item landed; stage nb's old item is done
             if (active) {
                 uint32_t x16[16];
-                stage_read(stage_in[buf], t, x16);
+                stage_read(stage[buf], t, x16);
                 float x[32];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
@@ -226,13 +230,12 @@ __global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_c
                 encode<C, false, false>(x, a, p, NoSink{});
                 store_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
             }
-            __syncthreads();                           // stage_in[buf] is refilled next
-            buf ^= 1;
+            last = buf;
+            buf = nb;
         }
-        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{stage_out, t});
+        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{stage[last], t});
         __syncthreads();
-        stage_to_outputs(stage_out, out, N, tile0 * (kTileElems * 2), ntiles);
-        __syncthreads();                               // stage_out is rewritten next chunk
+        stage_to_outputs(stage[last], out, N, tile0 * (kTileElems * 2), ntiles);
     }
 }
 
