@@ -628,3 +628,46 @@ int orc_all_to_all(const uint16_t *const *in_bf16, int N, size_t m, int codec,
     for (int r = 0; r < N; ++r) free(wires[r]);
     return codec;
 }
+
+/* ------------------------------------------------------------------------- */
+/* FP32 messages ([RX] Low-Precision Collectives: FP32 or BF16 inputs, FP8 on  */
+/* the wire, "up to 4:1" against FP32).  The same tiles and stages; the input  */
+/* blocks are binary32 values, and the result is the dequantised gathered     */
+/* value itself (binary32, no rounding).  The uncompressed passthrough sums   */
+/* the binary32 inputs in rank order from +0.0f.                               */
+/* ------------------------------------------------------------------------- */
+int orc_allreduce_f32(const float *const *in_f32, int N, size_t n, int codec,
+                      float *const *out_f32, size_t min_quant_bytes)
+{
+    if (N < 1 || N > ORC_MAX_RANKS || n % ORC_TILE_ELEMS != 0) return -1;
+    if (codec < ORC_BF16 || codec > ORC_MXFP4) return -1;
+    codec = effective(codec, 4 * n, min_quant_bytes);
+    size_t tiles = n / ORC_TILE_ELEMS;
+    if (codec == ORC_BF16) {                     /* passthrough: exact binary32 sum */
+        for (size_t i = 0; i < n; ++i) {
+            float acc = +0.0f;
+            for (int r = 0; r < N; ++r) acc = acc + in_f32[r][i];
+            for (int r = 0; r < N; ++r) out_f32[r][i] = acc;
+        }
+        return codec;
+    }
+    size_t tb = orc_tile_bytes(codec), wb = tiles * tb;
+    uint8_t *wires[ORC_MAX_RANKS];
+    uint8_t *gather = (uint8_t *)malloc(wb ? wb : 1);
+    if (!gather) return -1;
+    for (int r = 0; r < N; ++r) {
+        wires[r] = (uint8_t *)malloc(wb ? wb : 1);
+        if (!wires[r]) { for (int k = 0; k < r; ++k) free(wires[k]); free(gather); return -1; }
+        for (size_t t = 0; t < tiles; ++t)
+            orc_quant_tile(in_f32[r] + t * ORC_TILE_ELEMS, codec, wires[r] + t * tb);     /* stage 1 */
+    }
+    for (int j = 0; j < N; ++j) {                /* reduce-scatter shards, as in orc_allreduce */
+        size_t t0 = (size_t)j * tiles / (size_t)N, t1 = (size_t)(j + 1) * tiles / (size_t)N;
+        orc_reduce((const uint8_t *const *)wires, N, t0, t1 - t0, codec, gather);
+    }
+    for (size_t t = 0; t < tiles; ++t)            /* all-gather: the dequantised values */
+        for (int r = 0; r < N; ++r) orc_dequant_tile(gather + t * tb, codec, out_f32[r] + t * ORC_TILE_ELEMS);
+    for (int r = 0; r < N; ++r) free(wires[r]);
+    free(gather);
+    return codec;
+}

@@ -67,6 +67,10 @@ int orc_all_gather(const uint16_t *const *in_bf16, int N, size_t m, int codec,
 int orc_all_to_all(const uint16_t *const *in_bf16, int N, size_t m, int codec,
                    uint16_t *const *out_bf16, size_t min_quant_bytes);
 
+/* the all-reduce of binary32 messages (binary32 results; codec 0 = uncompressed) */
+int orc_allreduce_f32(const float *const *in_f32, int N, size_t n, int codec,
+                      float *const *out_f32, size_t min_quant_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,8 @@ def lib():
                                               ctypes.POINTER(u16p), sz]),
             "orc_all_to_all": (ctypes.c_int, [ctypes.POINTER(u16p), ctypes.c_int, sz, ctypes.c_int,
                                               ctypes.POINTER(u16p), sz]),
+            "orc_allreduce_f32": (ctypes.c_int, [ctypes.POINTER(f32p), ctypes.c_int, sz, ctypes.c_int,
+                                                 ctypes.POINTER(f32p), sz]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -279,3 +281,17 @@ def all_to_all(inputs_bf16, codec, min_quant_bytes=0):
     N = len(inputs_bf16)
     m = np.asarray(inputs_bf16[0]).size // N
     return _collective(lib().orc_all_to_all, inputs_bf16, codec, [N * m] * N, m, min_quant_bytes)
+
+
+def allreduce_f32(inputs_f32, codec, min_quant_bytes=0):
+    """All-reduce of N binary32 host arrays; returns (binary32 outputs, codec used)."""
+    ins = [np.ascontiguousarray(x, dtype=np.float32).reshape(-1) for x in inputs_f32]
+    n = ins[0].size
+    outs = [np.zeros(n, np.float32) for _ in ins]
+    fp = ctypes.POINTER(ctypes.c_float)
+    ia = (fp * len(ins))(*[_ptr(x, ctypes.c_float) for x in ins])
+    oa = (fp * len(outs))(*[_ptr(o, ctypes.c_float) for o in outs])
+    used = lib().orc_allreduce_f32(ia, len(ins), n, _codec(codec), oa, min_quant_bytes)
+    if used < 0:
+        raise ValueError("oracle rejected the arguments")
+    return outs, {v: k for k, v in CODECS.items()}[used]
