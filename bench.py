@@ -36,7 +36,8 @@ import workloads as W  # noqa: E402
 METRIC = "quantized all-reduce GB/s (N x input bytes/s) and % of HBM peak on 1 B200"
 TILE = 2048
 CODEC_C = {"bf16": 2.0, "fp8": 2304 / 2048, "int4": 1152 / 2048, "int3": 896 / 2048, "mxfp4": 1088 / 2048}
-KERNEL_SOURCES = ("quantized_precision_all_b200/csrc/lpar_kernels.cu", "quantized_precision_all_b200/csrc/lpar_codec.cuh")
+KERNEL_SOURCES = tuple("quantized_precision_all_b200/csrc/" + f for f in (
+    "lpar_kernels.cu", "lpar_codec.cuh", "lpar_tiles.cuh", "lpar_collectives.cu", "lpar_f32.cu"))
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 REF_TILES_PER_STEP = 256            # reference arm: 0.5 Mi elements per rank per step
 CPU_BASELINE_TILES = 16384          # cpu_baseline: 32 Mi elements (64 MiB) per rank
@@ -64,7 +65,9 @@ def measured_peaks():
 
 
 # ---- algorithmic bytes per launch (reads + writes the definition requires) ------
-def kernel_names(codec, schedule, N):
+def kernel_names(codec, schedule, N, f32=False):
+    if f32:
+        return ["k_f32_reduce<N=%d>" % N] if codec == "bf16" else ["k_allreduce_single_f32<%s,N=%d>" % (codec, N)]
     if codec == "bf16":
         return ["k_bf16_reduce<N=%d,fused>" % N] if schedule != "three_stage" else \
             ["k_bf16_reduce<N=%d>" % N, "k_broadcast"]
@@ -77,6 +80,11 @@ def kernel_names(codec, schedule, N):
 
 def algorithmic_bytes(kernel, codec, N, n):
     c = CODEC_C[codec]
+    if kernel.startswith("k_allreduce_single_f32"):
+        # N binary32 messages in, N wires out and back in, gathered wire out, N binary32 outputs out
+        return N * n * (4 + c) + n * (N * c + c + 4 * N)
+    if kernel.startswith("k_f32_reduce"):
+        return n * (4 * N + 4 + 4 * N)
     if kernel.startswith("k_allreduce_single"):
         # N BF16 messages in, N wires out and back in, gathered wire out, N outputs out
         return N * n * (2 + c) + n * (N * c + c + 2 * N)
@@ -188,16 +196,26 @@ def run_ours(args, rank, world, device):
 
     w = W.WORKLOADS[args.workload]
     N, n = w.N, w.n
+    f32 = w.dtype == "f32"
     xs = W.make_inputs(w, device)
     outs = [torch.empty_like(x) for x in xs]
-    ws_bytes = max(L.lpar_workspace_bytes(N, n, L.lpar_effective_codec(n, c, w.min_quant_bytes)) for c in w.codecs)
+
+    def eff_codec(c):                        # the threshold compares message bytes
+        return L.lpar_effective_codec(w.elem_bytes * n // 2, c, w.min_quant_bytes)
+
+    if f32:
+        ws_bytes = max(L.lpar_collective_workspace_bytes("allreduce_f32", N, n, eff_codec(c)) for c in w.codecs)
+        allreduce = L.lpar_allreduce_f32
+    else:
+        ws_bytes = max(L.lpar_workspace_bytes(N, n, eff_codec(c)) for c in w.codecs)
+        allreduce = L.lpar_allreduce
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(stage_events=None):
         for i, codec in enumerate(w.codecs):
-            L.lpar_allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream,
-                             stage_events=None if stage_events is None else stage_events[i])
+            allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream,
+                      stage_events=None if stage_events is None else stage_events[i])
 
     for _ in range(args.warmup):
         step()
@@ -231,9 +249,11 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     kern = {}
     for ci, codec in enumerate(w.codecs):
-        eff = L.lpar_effective_codec(n, codec, w.min_quant_bytes)
-        names = kernel_names(eff, args.schedule, N)
-        if eff == "bf16":
+        eff = eff_codec(codec)
+        names = kernel_names(eff, args.schedule, N, f32)
+        if f32:
+            bounds = [(0, 1)]
+        elif eff == "bf16":
             bounds = [(1, 2), (2, 3)]
         elif args.schedule == "single_pass":
             bounds = [(0, 1)]
@@ -248,23 +268,22 @@ def run_ours(args, rank, world, device):
         d["ms_per_launch"] = d["ms_total"] / d["launches"]
         d["algorithmic_bytes"] = algorithmic_bytes(name, d["codec"], N, n)
         d["achieved_gbs"] = d["algorithmic_bytes"] / (d["ms_per_launch"] * 1e-3) / 1e9
-    launches_per_step = sum(len(kernel_names(L.lpar_effective_codec(n, c, w.min_quant_bytes), args.schedule, N))
-                            for c in w.codecs)
+    launches_per_step = sum(len(kernel_names(eff_codec(c), args.schedule, N, f32)) for c in w.codecs)
 
     # (3) end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         e2e_steps = max(1, min(args.steps, 5))
-        h_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(N)]
+        h_in = [torch.empty(n, dtype=xs[0].dtype, pin_memory=True) for _ in range(N)]
         for h, x in zip(h_in, xs):
             h.copy_(x)
-        h_out = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(N)]
+        h_out = [torch.empty(n, dtype=xs[0].dtype, pin_memory=True) for _ in range(N)]
 
         def e2e_step():
             for x, h in zip(xs, h_in):
                 x.copy_(h, non_blocking=True)
             for codec in w.codecs:
-                L.lpar_allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
+                allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
                 for h, o in zip(h_out, outs):
                     h.copy_(o, non_blocking=True)
 
@@ -279,10 +298,12 @@ def run_ours(args, rank, world, device):
         s1.record(stream)
         torch.cuda.synchronize(device)
         e_ms = max_over_ranks(s0.elapsed_time(s1), world, device)
-        e2e = {"value": aggregate_gbs(world, N * 2 * n * len(w.codecs), e2e_steps, e_ms), "unit": "GB/s",
-               "h2d_bytes_per_step": N * 2 * n, "d2h_bytes_per_step": N * 2 * n * len(w.codecs),
+        eb = w.elem_bytes
+        e2e = {"value": aggregate_gbs(world, N * eb * n * len(w.codecs), e2e_steps, e_ms), "unit": "GB/s",
+               "h2d_bytes_per_step": N * eb * n, "d2h_bytes_per_step": N * eb * n * len(w.codecs),
                "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
-               "api": "lpar_allreduce with pinned host buffers copied in and out on the same stream"}
+               "api": "%s with pinned host buffers copied in and out on the same stream"
+                      % ("lpar_allreduce_f32" if f32 else "lpar_allreduce")}
         del h_in, h_out
 
     # (4) the oracle on the host cores, rank 0 at N=1 only
@@ -297,15 +318,20 @@ def run_ours(args, rank, world, device):
 def cpu_baseline(w, xs_dev, tiles=CPU_BASELINE_TILES):
     from oracle import oracle as O
     tiles = min(tiles, w.n // TILE)
-    xs = [x[:tiles * TILE].view(torch.int16).cpu().numpy().view("uint16") for x in xs_dev]
+    if w.dtype == "f32":
+        xs = [x[:tiles * TILE].cpu().numpy() for x in xs_dev]
+        fn = O.allreduce_f32
+    else:
+        xs = [x[:tiles * TILE].view(torch.int16).cpu().numpy().view("uint16") for x in xs_dev]
+        fn = O.allreduce
     t0 = time.perf_counter()
     for codec in w.codecs:
-        O.allreduce(xs, codec, w.min_quant_bytes)
+        fn(xs, codec, w.min_quant_bytes)
     dt = time.perf_counter() - t0
-    value = w.N * 2 * tiles * TILE * len(w.codecs) / dt / 1e9
+    value = w.N * w.elem_bytes * tiles * TILE * len(w.codecs) / dt / 1e9
     return {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "first %d tiles (%d MiB BF16) of each of the %d ranks, codecs %s, %.1f s single-threaded"
-                      % (tiles, tiles * TILE * 2 >> 20, w.N, "+".join(w.codecs), dt)}
+            "sample": "first %d tiles (%d MiB %s) of each of the %d ranks, codecs %s, %.1f s single-threaded"
+                      % (tiles, tiles * TILE * w.elem_bytes >> 20, w.dtype.upper(), w.N, "+".join(w.codecs), dt)}
 
 
 # ---- reference arm: the oracle as it stands, on the host --------------------------
@@ -313,11 +339,16 @@ def run_reference(args):
     from oracle import oracle as O
     w = W.WORKLOADS[args.workload]
     tiles = min(REF_TILES_PER_STEP, w.n // TILE)
-    xs = [x.view(torch.int16).numpy().view("uint16") for x in W.make_inputs(w, "cpu", n=tiles * TILE)]
+    if w.dtype == "f32":
+        xs = [x.numpy() for x in W.make_inputs(w, "cpu", n=tiles * TILE)]
+        fn = O.allreduce_f32
+    else:
+        xs = [x.view(torch.int16).numpy().view("uint16") for x in W.make_inputs(w, "cpu", n=tiles * TILE)]
+        fn = O.allreduce
 
     def step():
         for codec in w.codecs:
-            O.allreduce(xs, codec, w.min_quant_bytes)
+            fn(xs, codec, w.min_quant_bytes)
 
     for _ in range(args.warmup):
         step()
@@ -325,9 +356,9 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     dt = time.perf_counter() - t0
-    value = w.N * 2 * tiles * TILE * len(w.codecs) * args.steps / dt / 1e9
-    sample = "%d tiles (%d KiB BF16) per rank per step of workload %s, codecs %s" % (
-        tiles, tiles * TILE * 2 >> 10, w.name, "+".join(w.codecs))
+    value = w.N * w.elem_bytes * tiles * TILE * len(w.codecs) * args.steps / dt / 1e9
+    sample = "%d tiles (%d KiB %s) per rank per step of workload %s, codecs %s" % (
+        tiles, tiles * TILE * w.elem_bytes >> 10, w.dtype.upper(), w.name, "+".join(w.codecs))
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -450,11 +481,11 @@ def run_collectives(args, device):
 
 
 def workload_config(w, args):
-    return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n,
-            "message_bytes_per_rank": 2 * w.n, "codecs": list(w.codecs), "schedule": args.schedule,
+    return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n, "message_dtype": w.dtype,
+            "message_bytes_per_rank": w.message_bytes, "codecs": list(w.codecs), "schedule": args.schedule,
             "distribution": w.note, "min_quant_bytes": w.min_quant_bytes,
-            "l2": "inputs %d MiB > 126 MB L2: no flush between steps" % (w.N * 2 * w.n >> 20)
-            if w.N * 2 * w.n > 126e6 else "inputs fit in L2",
+            "l2": "inputs %d MiB > 126 MB L2: no flush between steps" % (w.N * w.message_bytes >> 20)
+            if w.N * w.message_bytes > 126e6 else "inputs fit in L2",
             "parallelism": "one independent instance per GPU"}
 
 
@@ -501,7 +532,7 @@ def main():
     w = res["w"]
     if rank == 0:
         peak, peak_src = measured_peaks()
-        step_bytes = w.N * 2 * w.n * len(w.codecs)
+        step_bytes = w.N * w.message_bytes * len(w.codecs)
         ms_per_step = res["ms"] / args.steps
         value = aggregate_gbs(world, step_bytes, args.steps, res["ms"])
         kern = res["kern"]

@@ -118,7 +118,8 @@ typedef enum {
     LPAR_OP_ALLREDUCE = 0,
     LPAR_OP_REDUCE_SCATTER = 1,
     LPAR_OP_ALL_GATHER = 2,
-    LPAR_OP_ALL_TO_ALL = 3
+    LPAR_OP_ALL_TO_ALL = 3,
+    LPAR_OP_ALLREDUCE_F32 = 4
 } lpar_collective_t;
 
 typedef struct {
@@ -195,10 +196,12 @@ lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_co
 
 /* Workspace bytes of a collective for the codec that runs (after the
  * threshold): the all-reduce as lpar_workspace_bytes(N, size, codec); the
- * others N wires of their per-rank message (reduce-scatter: n elements;
- * all-gather: m; all-to-all: N * m), and 0 for BF16, when no workspace is
- * needed and `workspace` may be NULL.  `size` is each call's size argument.
- * 0 for N outside [1, LPAR_MAX_RANKS] or an unknown codec or op. */
+ * all-reduce of binary32 messages (N + 1) wires, or 4 * size bytes for the
+ * uncompressed passthrough; the others N wires of their per-rank message
+ * (reduce-scatter: n elements; all-gather: m; all-to-all: N * m), and 0 for
+ * BF16, when no workspace is needed and `workspace` may be NULL.  `size` is
+ * each call's size argument.  0 for N outside [1, LPAR_MAX_RANKS] or an
+ * unknown codec or op. */
 size_t lpar_collective_workspace_bytes(lpar_collective_t op, int N, size_t size, lpar_codec_t codec);
 
 /* Reduce-scatter of N BF16 messages of n elements (n a multiple of 2048): the
@@ -224,6 +227,21 @@ lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t m, lpar_c
 lpar_status_t lpar_all_to_all(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
                               void *const *out, void *workspace, size_t workspace_bytes,
                               const lpar_options_t *opts, cudaStream_t stream);
+
+/* The all-reduce of N binary32 messages of n elements (the RCCLX page's
+ * Low-Precision Collectives: FP32 or BF16 inputs, FP8 for up to 4:1 against
+ * FP32).  Same codecs, tiles and stages as lpar_allreduce; each out[r] (n
+ * binary32 values) receives the dequantised gathered value itself, with no
+ * rounding to BF16.  LPAR_CODEC_BF16 selects the uncompressed passthrough:
+ * the binary32 sum in ascending rank order from +0.0f.  The threshold
+ * compares the binary32 message, 4n bytes.  Workspace:
+ * lpar_collective_workspace_bytes(LPAR_OP_ALLREDUCE_F32, N, n, effective
+ * codec).  Schedules: LPAR_SCHEDULE_AUTO and LPAR_SCHEDULE_SINGLE_PASS (one
+ * kernel); others return LPAR_ERR_UNSUPPORTED.  In place (out[r] ==
+ * inputs[r]) is allowed.  Stage events [0] and [1] bracket the kernel. */
+lpar_status_t lpar_allreduce_f32(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
+                                 void *const *out, void *workspace, size_t workspace_bytes,
+                                 const lpar_options_t *opts, cudaStream_t stream);
 
 /* Size of the workspace that lpar_allreduce_static keeps inside the library. */
 #define LPAR_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)

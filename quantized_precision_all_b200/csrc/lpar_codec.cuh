@@ -373,8 +373,8 @@ __device__ __forceinline__ float2 round_pair(float2 xv, const IntScale &k, uint3
 
 // INT4: lanes hold elements (8i + m, 8i + 4 + m); each lane packs 4 nibbles
 // (16 bits) with Q = Sum_m (-q_m) 16^m, P = (M + 0x8888) - Q.
-// Decoded BF16 output goes to `sink.put(piece, uint4)`: piece j holds the
-// packed words 4j..4j+3 (elements 8j..8j+7), written as soon as they exist.
+// Decoded values go to `sink.put(j, v0, ..., v7)`: piece j holds elements
+// 8j..8j+7 in order, handed over as soon as they exist.
 template <bool STAGE2, bool WANT_V, class Sink>
 __device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &k, uint32_t (&w)[4],
                                           const Sink &sink) {
@@ -394,8 +394,7 @@ __device__ __forceinline__ bool int4_fast(const float (&x)[32], const IntScale &
             float2 v[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) v[m] = fma2(nq[m], ns2, splat(0.f));   // q s (+0 for q = 0)
-            sink.put(i, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
-                                   pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y)));
+            sink.put(i, v[0].x, v[1].x, v[2].x, v[3].x, v[0].y, v[1].y, v[2].y, v[3].y);
         }
     }
     return (ok >> 31) != 0u;
@@ -442,10 +441,8 @@ __device__ __forceinline__ bool int3_fast(const float (&x)[32], const IntScale &
             hi[4 + g] = (W1 & 0x04040404u) * ((g & 1) ? 0x04081020u : 0x00408102u);
         }
         if (WANT_V) {                                  // piece j = elements 8j .. 8j+7
-            sink.put(p, make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
-                                   pack_bf16x2(v[4].x, v[5].x), pack_bf16x2(v[6].x, v[7].x)));
-            sink.put(2 + p, make_uint4(pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y),
-                                       pack_bf16x2(v[4].y, v[5].y), pack_bf16x2(v[6].y, v[7].y)));
+            sink.put(p, v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+            sink.put(2 + p, v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
         }
     }
     q2w[0] = __byte_perm(__byte_perm(lo[0], lo[1], 0x0073), __byte_perm(lo[2], lo[3], 0x0073), 0x5410);
@@ -475,12 +472,12 @@ __device__ __noinline__ void int_exact_codes(const float *x, IntScale k, uint8_t
 }
 
 template <bool WANT_V, class Sink>
-__device__ __forceinline__ void bf16_from_local(const float *v, const Sink &sink) {
+__device__ __forceinline__ void values_from_local(const float *v, const Sink &sink) {
     if (WANT_V) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            sink.put(j, make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                   pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7])));
+            sink.put(j, v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3], v[8 * j + 4], v[8 * j + 5],
+                     v[8 * j + 6], v[8 * j + 7]);
     }
 }
 
@@ -516,7 +513,7 @@ __device__ __forceinline__ void encode_int_exact_local(const float *xs, const In
     int_exact_codes<Layout<C>::kBits, WANT_V>(xs, k, cs, vs);
     if constexpr (C == kINT4) pack_int4_local(cs, p);
     else pack_int3_local(cs, p);
-    bf16_from_local<WANT_V>(vs, sink);
+    values_from_local<WANT_V>(vs, sink);
 }
 
 // Stage 1 (and any caller that keeps x): fast path, else copy x to local
@@ -548,12 +545,12 @@ __device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed
         p.scale = 0.f;
         if (WANT_V) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sink.put(j, make_uint4(0u, 0u, 0u, 0u));
+            for (int j = 0; j < 4; ++j) sink.put(j, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
     const float inv = __frcp_rn(s);                   // fl32(1 / s)
-    uint32_t o[4];
+    float o[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {                     // scalar IEEE products (subnormals kept)
         const uint32_t lo = pack_e4m3x2(__fmul_rn(x[4 * i], inv), __fmul_rn(x[4 * i + 1], inv));
@@ -561,9 +558,12 @@ __device__ __forceinline__ void encode_fp8(const float (&x)[32], float a, Packed
         p.w[i] = lo | (hi << 16);
         if (WANT_V) {                                 // scalar: e * s may be subnormal
             const uint32_t h0 = e4m3x2_to_h2(lo), h1 = e4m3x2_to_h2(hi);
-            o[2 * (i & 1)] = pack_bf16x2(__fmul_rn(h2f(h0, 0), s), __fmul_rn(h2f(h0, 1), s));
-            o[2 * (i & 1) + 1] = pack_bf16x2(__fmul_rn(h2f(h1, 0), s), __fmul_rn(h2f(h1, 1), s));
-            if (i & 1) sink.put(i >> 1, make_uint4(o[0], o[1], o[2], o[3]));
+            float *oi = o + 4 * (i & 1);
+            oi[0] = __fmul_rn(h2f(h0, 0), s);
+            oi[1] = __fmul_rn(h2f(h0, 1), s);
+            oi[2] = __fmul_rn(h2f(h1, 0), s);
+            oi[3] = __fmul_rn(h2f(h1, 1), s);
+            if (i & 1) sink.put(i >> 1, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
         }
     }
     p.scale = s;
@@ -596,11 +596,15 @@ __device__ __forceinline__ void encode_mxfp4(const float (&x)[32], float a, Pack
                              __fmul_rn(xi[4], m), __fmul_rn(xi[5], m), __fmul_rn(xi[6], m), __fmul_rn(xi[7], m));
         if (WANT_V) {                                             // E2M1 value * 2^E: exact, so is its BF16
             const float sv = mx_scale_value(ec);
-            uint32_t h[4], o[4];
+            uint32_t h[4];
+            float o[8];
             e2m1x8_to_h2(p.w[i], h);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = pack_bf16x2(__fmul_rn(h2f(h[k], 0), sv), __fmul_rn(h2f(h[k], 1), sv));
-            sink.put(i, make_uint4(o[0], o[1], o[2], o[3]));
+            for (int k = 0; k < 4; ++k) {
+                o[2 * k] = __fmul_rn(h2f(h[k], 0), sv);
+                o[2 * k + 1] = __fmul_rn(h2f(h[k], 1), sv);
+            }
+            sink.put(i, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
         }
     }
 }

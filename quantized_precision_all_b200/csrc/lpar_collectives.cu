@@ -264,7 +264,7 @@ static inline unsigned persistent_grid(unsigned chunks, unsigned resident) {
 template <int C, int N, bool ALL>
 static void launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned grid = persistent_grid(chunks, resident_ctas(k_reduce_bf16_single<C, N, ALL>));
+    const unsigned grid = persistent_grid(chunks, resident_ctas<k_reduce_bf16_single<C, N, ALL>>());
     k_reduce_bf16_single<C, N, ALL><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, chunks);
 }
 
@@ -309,7 +309,7 @@ template <int C, bool A2A>
 static void launch_gather_c(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
                             size_t seg_tiles, cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned grid = persistent_grid(chunks, resident_ctas(k_gather_single<C, A2A>));
+    const unsigned grid = persistent_grid(chunks, resident_ctas<k_gather_single<C, A2A>>());
     k_gather_single<C, A2A><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, seg_tiles, chunks, N);
 }
 
@@ -339,6 +339,8 @@ LPAR_API size_t lpar_collective_workspace_bytes(lpar_collective_t op, int N, siz
     if (N < 1 || N > kMaxRanks || !codec_ok(codec)) return 0;
     switch (op) {
     case LPAR_OP_ALLREDUCE: return lpar_workspace_bytes(N, n, codec);
+    case LPAR_OP_ALLREDUCE_F32:
+        return codec == LPAR_CODEC_BF16 ? 4 * n : (size_t)(N + 1) * lpar_wire_bytes(codec, n);
     case LPAR_OP_REDUCE_SCATTER:
     case LPAR_OP_ALL_GATHER: return codec == LPAR_CODEC_BF16 ? 0 : (size_t)N * lpar_wire_bytes(codec, n);
     case LPAR_OP_ALL_TO_ALL: return codec == LPAR_CODEC_BF16 ? 0 : (size_t)N * lpar_wire_bytes(codec, (size_t)N * n);

@@ -24,42 +24,6 @@
 
 namespace lpar {
 
-// Stage-2 rare path: recompute the block's FP32 sums from the N wires (same
-// arithmetic, so the same values) and requantise it exactly, one element at a
-// time.  Re-reading the wires lets the hot path drop the sums as it goes.
-template <int C, bool WANT_V, class Sink>
-__device__ __noinline__ void reduce_block_exact(const uint8_t *const *wp, int N, size_t tile, int b, Packed<C> *g,
-                                                Sink sink) {
-    constexpr int kBits = Layout<C>::kBits;
-    constexpr int kBias = 1 << (kBits - 1);
-    float acc[32];
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
-#pragma unroll 1
-    for (int r = 0; r < N; ++r) {
-        const uint8_t *tb = wp[r] + tile * Layout<C>::kTileBytes;
-        const float s = __half2float(__ushort_as_half(
-            *reinterpret_cast<const uint16_t *>(tb + Layout<C>::kScaleOff + 2 * b)));
-#pragma unroll 1
-        for (int j = 0; j < 32; ++j) {
-            int code;
-            if constexpr (C == kINT4) {
-                code = (tb[16 * b + j / 2] >> (4 * (j & 1))) & 0xF;
-            } else {
-                code = ((tb[8 * b + j / 4] >> (2 * (j & 3))) & 3) |
-                       (((tb[Layout<kINT3>::kQ1wOff + 4 * b + j / 8] >> (j & 7)) & 1) << 2);
-            }
-            acc[j] = __fadd_rn(acc[j], __fmul_rn((float)(code - kBias), s));   // exact product
-        }
-    }
-    float a = 0.f;
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) a = fmaxf(a, fabsf(acc[j]));
-    const IntScale k = int_scale<kBits>(a);
-    g->scale = k.bits;
-    encode_int_exact_local<C, WANT_V>(acc, k, *g, sink);
-}
-
 // ---------------------------------------------------------------------------
 // K1: stage 1 for every rank.  Persistent: CTA b handles the work items
 // (chunk c, rank r) for c = b, b + gridDim.x, ... and r = 0..N-1 (a chunk is 4
@@ -117,39 +81,6 @@ __global__ void __launch_bounds__(kThreads, 5) k_quantize(const __grid_constant_
 // K2 / K23: tiles [tile_begin, tile_end) of N wires -> gathered wire (and,
 // when FUSED, the decoded BF16 result into every out[r]).
 // ---------------------------------------------------------------------------
-// Stage 2 for one block: thread-owned block b of `tile`, N wires -> gathered
-// wire (and the decoded BF16 words into `sink`).
-template <int C, int N, bool WANT_V, class Sink>
-__device__ __forceinline__ void reduce_block(const uint8_t *const *wp, size_t tile, int b, uint8_t *gather,
-                                             const Sink &sink) {
-    Packed<C> p[N];
-#pragma unroll
-    for (int r = 0; r < N; ++r) load_block(wp[r] + tile * Layout<C>::kTileBytes, b, p[r]);
-    float acc[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;          // +0.0f, then ranks in ascending order
-#pragma unroll
-    for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
-    const float a = absmax_f32x32(acc);
-    Packed<C> g;
-    if constexpr (C == kFP8) {
-        encode_fp8<WANT_V>(acc, a, g, sink);
-    } else if constexpr (C == kMXFP4) {
-        encode_mxfp4<WANT_V>(acc, a, g, sink);
-    } else {
-        const IntScale k = int_scale<Layout<C>::kBits>(a);
-        g.scale = k.bits;
-        bool ok = k.fast;
-        if constexpr (C == kINT4) {
-            if (ok) ok = int4_fast<true, WANT_V>(acc, k, g.w, sink);
-        } else {
-            if (ok) ok = int3_fast<true, WANT_V>(acc, k, g.q2w, g.q1w, sink);
-        }
-        if (!ok) reduce_block_exact<C, WANT_V>(wp, N, tile, b, &g, sink);
-    }
-    store_block(gather + tile * Layout<C>::kTileBytes, b, g);
-}
-
 template <int C, int N, bool FUSED>
 __global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InPtrs wires, uint8_t *gather,
                                                      const __grid_constant__ OutPtrs out, size_t tile_begin,
@@ -308,7 +239,7 @@ static inline unsigned grid_for_tiles(size_t tiles) { return (unsigned)((tiles +
 template <int C>
 static void launch_quantize_c(const InPtrs &in, const OutPtrs &wire, int N, size_t tiles, cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned res = resident_ctas(k_quantize<C>);
+    const unsigned res = resident_ctas<k_quantize<C>>();
     // every CTA walks all N ranks of its chunks: size the grid in chunks
     const unsigned per_rank = (res ? res : 148u * 4u);
     const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, per_rank));
@@ -374,7 +305,7 @@ template <int C, int N>
 static void launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
                              cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned res = resident_ctas(k_allreduce_single<C, N>);
+    const unsigned res = resident_ctas<k_allreduce_single<C, N>>();
     const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 4u));
     k_allreduce_single<C, N><<<grid, kThreads, 0, st>>>(in, wire, g, o, tiles, chunks);
 }

@@ -90,14 +90,71 @@ __device__ __forceinline__ void store_block(uint8_t *tile, int b, const Packed<k
 }
 
 // Destinations for the decoded BF16 words of a block (piece j = 16 B).
+// ---------------------------------------------------------------------------
+// binary32 messages: 128 B per thread (its 32-element block), eight 16-B
+// pieces, swizzled as piece j of thread t at 128 t + 16 (j ^ (t & 7)): a
+// warp's coalesced 16-B accesses (four threads' blocks) and its per-thread
+// accesses (one piece of 32 threads) both spread over all eight 16-B bank
+// groups, four accesses each.  A 4-tile chunk is 32 KiB.
+// ---------------------------------------------------------------------------
+constexpr int kStageBytesF32 = kThreads * 128;
+
+__device__ __forceinline__ int swz32(int t, int j) { return 128 * t + 16 * (j ^ (t & 7)); }
+
+__device__ __forceinline__ void stage_load_chunk_f32(uint8_t *stage, const uint8_t *src, int ntiles) {
+    const int t = threadIdx.x;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int g = t + kThreads * k;                 // 16-B piece of the chunk (512 per tile)
+        if (g < ntiles * 512) cp_async16(stage + swz32(g >> 3, g & 7), src + 16 * (size_t)g);
+    }
+}
+
+__device__ __forceinline__ void stage_read_f32(const uint8_t *stage, int t, float (&x)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 q = *reinterpret_cast<const float4 *>(stage + swz32(t, j));
+        x[4 * j] = q.x; x[4 * j + 1] = q.y; x[4 * j + 2] = q.z; x[4 * j + 3] = q.w;
+    }
+}
+
+__device__ __forceinline__ void stage_to_outputs_f32(const uint8_t *stage, const OutPtrs &out, int N, size_t byte0,
+                                                     int ntiles) {
+    const int t = threadIdx.x;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int g = t + kThreads * k;
+        if (g < ntiles * 512) {
+            const uint4 d = *reinterpret_cast<const uint4 *>(stage + swz32(g >> 3, g & 7));
+#pragma unroll
+            for (int r = 0; r < kMaxRanks; ++r)
+                if (r < N) *reinterpret_cast<uint4 *>(out.p[r] + byte0 + 16 * (size_t)g) = d;
+        }
+    }
+}
+
+// Destinations of the decoded values of a block: put(j, v0..v7) receives
+// elements 8j..8j+7 (binary32, exact dequantised values).
 struct NoSink {
-    __device__ __forceinline__ void put(int, uint4) const {}
+    __device__ __forceinline__ void put(int, float, float, float, float, float, float, float, float) const {}
 };
-struct StageSink {                                   // thread t's 64-B region of the stage
+struct StageSink {                                   // BF16 (RNE) into thread t's 64-B region of the stage
     uint8_t *stage;
     int t;
-    __device__ __forceinline__ void put(int j, uint4 v) const {
-        *reinterpret_cast<uint4 *>(stage + swz(t, j)) = v;
+    __device__ __forceinline__ void put(int j, float a0, float a1, float a2, float a3, float a4, float a5, float a6,
+                                        float a7) const {
+        *reinterpret_cast<uint4 *>(stage + swz(t, j)) =
+            make_uint4(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3), pack_bf16x2(a4, a5), pack_bf16x2(a6, a7));
+    }
+};
+
+struct StageSinkF32 {                                // binary32 into thread t's 128-B region
+    uint8_t *stage;
+    int t;
+    __device__ __forceinline__ void put(int j, float a0, float a1, float a2, float a3, float a4, float a5, float a6,
+                                        float a7) const {
+        *reinterpret_cast<float4 *>(stage + swz32(t, 2 * j)) = make_float4(a0, a1, a2, a3);
+        *reinterpret_cast<float4 *>(stage + swz32(t, 2 * j + 1)) = make_float4(a4, a5, a6, a7);
     }
 };
 
@@ -122,6 +179,75 @@ __device__ __forceinline__ void decode(const Packed<C> &p, uint32_t (&o)[16]) {
     else if constexpr (C == kINT3) decode_int3(p, o);
     else if constexpr (C == kMXFP4) decode_mxfp4(p, o);
     else decode_fp8(p, o);
+}
+
+// Stage-2 rare path: recompute the block's FP32 sums from the N wires (same
+// arithmetic, so the same values) and requantise it exactly, one element at a
+// time.  Re-reading the wires lets the hot path drop the sums as it goes.
+template <int C, bool WANT_V, class Sink>
+__device__ __noinline__ void reduce_block_exact(const uint8_t *const *wp, int N, size_t tile, int b, Packed<C> *g,
+                                                Sink sink) {
+    constexpr int kBits = Layout<C>::kBits;
+    constexpr int kBias = 1 << (kBits - 1);
+    float acc[32];
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+#pragma unroll 1
+    for (int r = 0; r < N; ++r) {
+        const uint8_t *tb = wp[r] + tile * Layout<C>::kTileBytes;
+        const float s = __half2float(__ushort_as_half(
+            *reinterpret_cast<const uint16_t *>(tb + Layout<C>::kScaleOff + 2 * b)));
+#pragma unroll 1
+        for (int j = 0; j < 32; ++j) {
+            int code;
+            if constexpr (C == kINT4) {
+                code = (tb[16 * b + j / 2] >> (4 * (j & 1))) & 0xF;
+            } else {
+                code = ((tb[8 * b + j / 4] >> (2 * (j & 3))) & 3) |
+                       (((tb[Layout<kINT3>::kQ1wOff + 4 * b + j / 8] >> (j & 7)) & 1) << 2);
+            }
+            acc[j] = __fadd_rn(acc[j], __fmul_rn((float)(code - kBias), s));   // exact product
+        }
+    }
+    float a = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) a = fmaxf(a, fabsf(acc[j]));
+    const IntScale k = int_scale<kBits>(a);
+    g->scale = k.bits;
+    encode_int_exact_local<C, WANT_V>(acc, k, *g, sink);
+}
+
+// Stage 2 for one block: thread-owned block b of `tile`, N wires -> gathered
+// wire (and the decoded BF16 words into `sink`).
+template <int C, int N, bool WANT_V, class Sink>
+__device__ __forceinline__ void reduce_block(const uint8_t *const *wp, size_t tile, int b, uint8_t *gather,
+                                             const Sink &sink) {
+    Packed<C> p[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) load_block(wp[r] + tile * Layout<C>::kTileBytes, b, p[r]);
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;          // +0.0f, then ranks in ascending order
+#pragma unroll
+    for (int r = 0; r < N; ++r) accumulate<C>(p[r], acc);
+    const float a = absmax_f32x32(acc);
+    Packed<C> g;
+    if constexpr (C == kFP8) {
+        encode_fp8<WANT_V>(acc, a, g, sink);
+    } else if constexpr (C == kMXFP4) {
+        encode_mxfp4<WANT_V>(acc, a, g, sink);
+    } else {
+        const IntScale k = int_scale<Layout<C>::kBits>(a);
+        g.scale = k.bits;
+        bool ok = k.fast;
+        if constexpr (C == kINT4) {
+            if (ok) ok = int4_fast<true, WANT_V>(acc, k, g.w, sink);
+        } else {
+            if (ok) ok = int3_fast<true, WANT_V>(acc, k, g.q2w, g.q1w, sink);
+        }
+        if (!ok) reduce_block_exact<C, WANT_V>(wp, N, tile, b, &g, sink);
+    }
+    store_block(gather + tile * Layout<C>::kTileBytes, b, g);
 }
 
 // Thread t's 64-B BF16 block <-> the swizzled stage.
@@ -182,10 +308,12 @@ __device__ __forceinline__ void stage_load_chunk(uint8_t *stage, const uint8_t *
 // ---------------------------------------------------------------------------
 // Host-side helpers.
 // ---------------------------------------------------------------------------
-// Resident CTAs of a kernel on the current device (SM count x occupancy), cached
-// per device and kernel; 0 when the query fails.
-template <class K>
-static unsigned resident_ctas(K kernel) {
+// Resident CTAs of a kernel on the current device (SM count x occupancy at
+// `smem` bytes of dynamic shared memory), cached per device and per kernel
+// (the template argument is the kernel itself, so every kernel has its own
+// cache); 0 when the query fails.
+template <auto Kernel>
+static unsigned resident_ctas(int smem = 0) {
     static std::atomic<unsigned> cache[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
@@ -193,10 +321,23 @@ static unsigned resident_ctas(K kernel) {
     if (v) return v;
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, Kernel, kThreads, smem) != cudaSuccess) return 0;
     v = (unsigned)(sms * (per_sm > 0 ? per_sm : 1));
     cache[dev].store(v, std::memory_order_relaxed);
     return v;
+}
+
+// The opt-in to more than 48 KiB of dynamic shared memory, made once per
+// device and per kernel; false when it fails.
+template <auto Kernel>
+static bool allow_dynamic_smem(int bytes) {
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    if (done[dev].load(std::memory_order_relaxed)) return true;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done[dev].store(1, std::memory_order_relaxed);
+    return true;
 }
 
 static inline bool codec_ok(int c) { return c >= LPAR_CODEC_BF16 && c <= LPAR_CODEC_MXFP4; }

@@ -24,7 +24,7 @@ LPAR_SCHEDULE_AUTO, LPAR_SCHEDULE_FUSED, LPAR_SCHEDULE_THREE_STAGE, LPAR_SCHEDUL
 LPAR_SCHEDULE_ONE_SHOT = 4
 SCHEDULES = {"auto": LPAR_SCHEDULE_AUTO, "fused": LPAR_SCHEDULE_FUSED, "three_stage": LPAR_SCHEDULE_THREE_STAGE,
              "single_pass": LPAR_SCHEDULE_SINGLE_PASS, "one_shot": LPAR_SCHEDULE_ONE_SHOT}
-OPS = {"allreduce": 0, "reduce_scatter": 1, "all_gather": 2, "all_to_all": 3}
+OPS = {"allreduce": 0, "reduce_scatter": 1, "all_gather": 2, "all_to_all": 3, "allreduce_f32": 4}
 STATUS = {0: "LPAR_OK", 1: "LPAR_ERR_INVALID_ARG", 2: "LPAR_ERR_MISALIGNED",
           3: "LPAR_ERR_WORKSPACE_TOO_SMALL", 4: "LPAR_ERR_UNSUPPORTED", 5: "LPAR_ERR_CUDA"}
 TILE_ELEMS = 2048
@@ -32,7 +32,8 @@ MAX_RANKS = 8
 
 EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
            "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string",
-           "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all")
+           "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all",
+           "lpar_allreduce_f32")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -66,6 +67,7 @@ def _load():
         "lpar_reduce_scatter": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_all_gather": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_all_to_all": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_allreduce_f32": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -182,6 +184,18 @@ def lpar_allreduce_static(inputs, n, codec, out, min_quant_bytes=0, schedule="au
                                       ctypes.byref(opts), _stream(stream)), "lpar_allreduce_static")
 
 
+def lpar_allreduce_f32(inputs, n, codec, out, workspace, workspace_bytes, min_quant_bytes=0, schedule="auto",
+                       stream=None, N=None, stage_events=None):
+    """All-reduce of N binary32 messages (binary32 results)."""
+    ins = _ptr_array(inputs)
+    outs = _ptr_array(out)
+    N = len(inputs) if N is None else N
+    opts = _options(min_quant_bytes, schedule, stage_events)
+    _check(_lib.lpar_allreduce_f32(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+                                   _ptr(workspace), workspace_bytes, ctypes.byref(opts), _stream(stream)),
+           "lpar_allreduce_f32")
+
+
 def lpar_status_string(status):
     return _lib.lpar_status_string(status).decode()
 
@@ -273,4 +287,17 @@ def all_to_all(inputs, codec, min_quant_bytes=0, stream=None):
     out = [torch.empty(N * m, dtype=torch.bfloat16, device=inputs[0].device) for _ in range(N)]
     ws = _workspace("all_to_all", N, m, codec, min_quant_bytes, inputs[0].device)
     lpar_all_to_all(inputs, m, codec, out, ws, ws.numel(), min_quant_bytes, stream)
+    return out
+
+
+def allreduce_f32(inputs, codec, out=None, min_quant_bytes=0, stream=None):
+    """All-reduce a list of N equal-size binary32 CUDA tensors; returns the N outputs."""
+    import torch
+    N, n = len(inputs), inputs[0].numel()
+    if out is None:
+        out = [torch.empty_like(x) for x in inputs]
+    eff = lpar_effective_codec(2 * n, codec, min_quant_bytes)      # threshold on 4n bytes
+    need = lpar_collective_workspace_bytes("allreduce_f32", N, n, eff)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=inputs[0].device)
+    lpar_allreduce_f32(inputs, n, codec, out, ws, ws.numel(), min_quant_bytes, "auto", stream)
     return out

@@ -176,6 +176,24 @@ def test_argument_errors_collectives(L, fn):
     assert getattr(lib, fn)(None, 2, n, 2, None, A, ws, ctypes.byref(opts), None) == 1
 
 
+def test_argument_errors_allreduce_f32(L):
+    st = 0
+    n = 2048 * 4
+    need = L.lpar_collective_workspace_bytes("allreduce_f32", 2, n, "fp8")
+    assert need == 3 * 4 * 2304
+    assert L.lpar_collective_workspace_bytes("allreduce_f32", 2, n, "bf16") == 4 * n
+    ok = dict(stream=st)
+    assert status_of(L.lpar_allreduce_f32, [A, A], n, "fp8", [A, A], A, need - 16, **ok) == 3
+    assert status_of(L.lpar_allreduce_f32, [A, M], n, "fp8", [A, A], A, need, **ok) == 2
+    assert status_of(L.lpar_allreduce_f32, [A, A], n, "fp8", [A, A], M, need, **ok) == 2
+    assert status_of(L.lpar_allreduce_f32, [A, A], n, "fp8", [A, A], 0, need, **ok) == 1
+    assert status_of(L.lpar_allreduce_f32, [A, A], n + 4, "fp8", [A, A], A, need, **ok) == 1
+    assert status_of(L.lpar_allreduce_f32, [A] * 9, n, "fp8", [A] * 9, A, 10 ** 9, **ok) == 1
+    assert status_of(L.lpar_allreduce_f32, [A, A], n, 12, [A, A], A, need, **ok) == 4
+    assert status_of(L.lpar_allreduce_f32, [A, A], n, "fp8", [A, A], A, need, schedule="fused", **ok) == 4
+    assert status_of(L.lpar_allreduce_f32, [A, A], 0, "fp8", [A, A], A, 0, **ok) == 0
+
+
 def test_one_shot_schedule_is_accepted_and_validated(L):
     st = 0
     n = 2048 * 4

@@ -6,7 +6,8 @@ names those workloads.  Both the CUDA path and the CPU oracle consume its output
 
 Recipe (rank r of a workload with seed S): a ``torch.Generator`` on the chosen
 device seeded with ``S * 1009 + r`` draws binary32 values, which are rounded to
-BF16 (round to nearest even) by ``Tensor.to(torch.bfloat16)``.
+BF16 (round to nearest even) by ``Tensor.to(torch.bfloat16)`` (binary32
+workloads keep the draws).
 Distributions:
   * ``normal``            N(0, sigma^2)
   * ``normal_outliers``   N(0, 1), then round(0.1% * n) positions per rank,
@@ -34,10 +35,15 @@ class Workload:
     min_quant_bytes: int = 0
     shape: Optional[Tuple[int, ...]] = None
     note: str = ""
+    dtype: str = "bf16"         # message element type: bf16, or f32 (binary32 messages)
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
 
     @property
     def message_bytes(self) -> int:
-        return 2 * self.n
+        return self.elem_bytes * self.n
 
 
 # The workloads of the pages' problem statement (TP activations of LLM serving).
@@ -62,6 +68,11 @@ WORKLOADS = {
              "INT3 then INT4 back to back"),
 }
 
+WORKLOADS["prefill_fp8_f32"] = Workload(
+    "prefill_fp8_f32", N=8, n=2048 * 8192, dist="student_t", nu=4, seed=3, codecs=("fp8", "bf16"),
+    shape=(2048, 8192), dtype="f32",
+    note="prefill-shaped, binary32 messages: N=8 x (2048 tokens x 8192 hidden) FP32 = 64 MiB per rank, "
+         "Student-t nu=4, FP8 e4m3 (4:1 against FP32) and the uncompressed FP32 sum")
 WORKLOADS["large_mxfp4"] = Workload(
     "large_mxfp4", N=2, n=512 * 1024 * 1024, dist="normal", sigma=0.02, seed=4, codecs=("mxfp4",),
     note="large message, FP4 mode: N=2 x 512 Mi BF16 (1 GiB per rank), N(0, 0.02^2), MXFP4")
@@ -109,8 +120,11 @@ def _draw_f32(w: Workload, r: int, n: int, device) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, device="cpu", n: Optional[int] = None) -> List[torch.Tensor]:
-    """N BF16 tensors of n elements each (default: the workload's n)."""
+    """N tensors of n elements each (default: the workload's n): BF16, or the
+    binary32 draws themselves for an f32 workload."""
     n = w.n if n is None else n
+    if w.dtype == "f32":
+        return [_draw_f32(w, r, n, device) for r in range(w.N)]
     return [_draw_f32(w, r, n, device).to(torch.bfloat16) for r in range(w.N)]
 
 
