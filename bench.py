@@ -367,6 +367,21 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def oracle_gbs(op, N, codec, tiles=64):
+    """The oracle's rate on a small seeded sample (its cost per tile does not
+    depend on the message size): GB/s of N x per-rank message bytes, one core."""
+    from oracle import oracle as O
+    w = W.Workload("oracle_sample", N=N, n=tiles * TILE, dist="student_t", nu=3, seed=9, codecs=(codec,))
+    xs = [x.view(torch.int16).numpy().view("uint16") for x in W.make_inputs(w, "cpu")]
+    fn = {"allreduce": O.allreduce, "reduce_scatter": O.reduce_scatter, "one_shot": O.allreduce_oneshot,
+          "all_gather": O.all_gather, "all_to_all": O.all_to_all}[op]
+    t0 = time.perf_counter()
+    fn(xs, codec)
+    dt = time.perf_counter() - t0
+    return {"value": N * 2 * tiles * TILE / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d tiles per rank, N=%d, %s, %s" % (tiles, N, codec, op)}
+
+
 def run_sweep(args, device):
     """One JSON line per sweep point (N, message size, codec): GB/s and the
     fraction of measured HBM peak the whole call reaches (its algorithmic
@@ -374,6 +389,7 @@ def run_sweep(args, device):
     from quantized_precision_all_b200 import lpar as L
     peak, peak_src = measured_peaks()
     stream = torch.cuda.current_stream(device)
+    cpu = {(N, c): oracle_gbs("allreduce", N, c) for N in W.SWEEP_RANKS for c in W.SWEEP_CODECS}
     for N in W.SWEEP_RANKS:
         for mb in W.SWEEP_SIZES_BYTES:
             w = W.sweep_workload(N, mb, "bf16")
@@ -403,7 +419,7 @@ def run_sweep(args, device):
                                   "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
                                   "l2": "256 MiB buffer rewritten before every timed call",
                                   "note": "L2-resident / launch-bound" if N * mb < (16 << 20) else "",
-                                  "peak": peak}), flush=True)
+                                  "peak": peak, "cpu_baseline": cpu[(N, codec)]}), flush=True)
             del xs, outs, ws, flush
             torch.cuda.empty_cache()
 
@@ -438,6 +454,7 @@ def run_collectives(args, device):
     peak, _ = measured_peaks()
     stream = torch.cuda.current_stream(device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    cpu = {(op, N, c): oracle_gbs(op, N, c) for op in COLL_OPS for N in (2, 4, 8) for c in W.SWEEP_CODECS}
     for op in COLL_OPS:
         for N in (2, 4, 8):
             for mb in COLL_SIZES_BYTES:
@@ -474,7 +491,7 @@ def run_collectives(args, device):
                     print(json.dumps({"collective": op, "N": N, "message_bytes": mb, "codec": codec, "ms": ms,
                                       "GBps": N * mb / (ms * 1e-3) / 1e9,
                                       "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
-                                      "algorithmic_bytes": alg, "peak": peak,
+                                      "algorithmic_bytes": alg, "peak": peak, "cpu_baseline": cpu[(op, N, codec)],
                                       "l2": "256 MiB buffer rewritten before every timed call"}), flush=True)
                 del xs, outs, ws
                 torch.cuda.empty_cache()
