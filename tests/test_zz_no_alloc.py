@@ -22,7 +22,7 @@ def L():
     return lpar
 
 
-@pytest.mark.parametrize("codec,N", [("int3", 2), ("int4", 2), ("fp8", 8), ("bf16", 3)])
+@pytest.mark.parametrize("codec,N", [("int3", 2), ("int4", 2), ("fp8", 8), ("mxfp4", 4), ("bf16", 3)])
 def test_static_workspace_equals_caller_workspace_on_two_calls(L, codec, N):
     n = 2048 * 37
     g = torch.Generator(device="cuda").manual_seed(900 + N)
