@@ -562,3 +562,53 @@ def test_sweep_sampled_tiles(L, N):
                     assert np.array_equal(g, ref[0]), (N, mb, codec, schedule)
         del xs, outs, ws
         torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# Streams and graphs: the library never synchronises and keeps no per-call
+# state, so calls on two streams at once, and calls captured in a CUDA graph
+# and replayed on new inputs, give the oracle's results.
+# ---------------------------------------------------------------------------
+def test_two_streams_at_once(L):
+    n = 2048 * 64
+    jobs = []
+    for k, codec in enumerate(("int3", "mxfp4")):
+        xs = [adversarial_bf16(n, 1200 + 10 * k + r) for r in range(3)]
+        dx = [torch.from_numpy(x.view(np.int16)).cuda() for x in xs]
+        outs = [torch.empty_like(d) for d in dx]
+        ws = torch.empty(L.lpar_workspace_bytes(3, n, codec), dtype=torch.uint8, device="cuda")
+        jobs.append((codec, xs, dx, outs, ws, torch.cuda.Stream()))
+    torch.cuda.synchronize()
+    for codec, xs, dx, outs, ws, s in jobs:
+        for _ in range(3):                               # several calls in flight on each stream
+            L.lpar_allreduce(dx, n, codec, outs, ws, ws.numel(), stream=s)
+    torch.cuda.synchronize()
+    for codec, xs, dx, outs, ws, s in jobs:
+        ref, _ = O.allreduce(xs, codec)
+        for o in outs:
+            assert np.array_equal(o.cpu().numpy().view(np.uint16), ref[0])
+
+
+@pytest.mark.parametrize("codec,schedule", [("int4", "auto"), ("fp8", "fused"), ("int3", "three_stage"),
+                                            ("mxfp4", "one_shot")])
+def test_captured_in_a_cuda_graph(L, codec, schedule):
+    n, N = 2048 * 16, 2
+    dx = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(N)]
+    outs = [torch.empty_like(d) for d in dx]
+    ws = torch.empty(L.lpar_workspace_bytes(N, n, codec), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):                           # a first call outside capture fills the host caches
+        L.lpar_allreduce(dx, n, codec, outs, ws, ws.numel(), schedule=schedule, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        L.lpar_allreduce(dx, n, codec, outs, ws, ws.numel(), schedule=schedule, stream=s)
+    for k in range(2):                                   # replay on new inputs
+        xs = [adversarial_bf16(n, 1300 + 10 * k + r) for r in range(N)]
+        for d, x in zip(dx, xs):
+            d.copy_(torch.from_numpy(x.view(np.int16)))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = (O.allreduce_oneshot if schedule == "one_shot" else O.allreduce)(xs, codec)[0]
+        for o in outs:
+            assert np.array_equal(o.cpu().numpy().view(np.uint16), ref[0])
