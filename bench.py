@@ -270,7 +270,18 @@ def run_ours(args, rank, world, device):
         d["achieved_gbs"] = d["algorithmic_bytes"] / (d["ms_per_launch"] * 1e-3) / 1e9
     launches_per_step = sum(len(kernel_names(eff_codec(c), args.schedule, N, f32)) for c in w.codecs)
 
-    # (3) end to end through the public API with host buffers
+    # (3) parity and accuracy of this step's outputs on sampled tiles (outside the timed region)
+    accuracy = {}
+    if not f32:
+        T = n // TILE
+        rng = torch.Generator().manual_seed(11)
+        sample = torch.unique(torch.cat([torch.tensor([0, T - 1]), torch.randint(0, T, (62,), generator=rng)]))
+        for codec in w.codecs:
+            allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
+            torch.cuda.synchronize(device)
+            accuracy[codec] = sample_check(xs, outs, codec, sample.numpy(), w.min_quant_bytes)
+
+    # (4) end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         e2e_steps = max(1, min(args.steps, 5))
@@ -306,13 +317,13 @@ def run_ours(args, rank, world, device):
                       % ("lpar_allreduce_f32" if f32 else "lpar_allreduce")}
         del h_in, h_out
 
-    # (4) the oracle on the host cores, rank 0 at N=1 only
+    # (5) the oracle on the host cores, rank 0 at N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, xs)
 
     return {"ms": ms_max, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
-            "e2e": e2e, "cpu": cpu, "w": w}
+            "e2e": e2e, "cpu": cpu, "w": w, "accuracy": accuracy}
 
 
 def cpu_baseline(w, xs_dev, tiles=CPU_BASELINE_TILES):
@@ -367,6 +378,26 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def sample_check(xs, outs, codec, tiles, min_quant_bytes=0):
+    """Bit-exact comparison of sampled output tiles with the oracle, the error
+    of those tiles against the exact (binary64) sum of the inputs, and a hash of
+    the sampled input bytes.  Tiles are independent, so a sample is exact."""
+    from oracle import oracle as O
+    idx = torch.from_numpy((tiles[:, None] * TILE + torch.arange(TILE).numpy()[None, :]).reshape(-1)).to(xs[0].device)
+    ins = [x[idx].view(torch.int16).cpu().numpy().view("uint16") for x in xs]
+    got = [o[idx].view(torch.int16).cpu().numpy().view("uint16") for o in outs]
+    ref, _ = O.allreduce(ins, codec, min_quant_bytes)
+    parity = all((g == ref[0]).all() for g in got)
+    exact = sum(O.bf16_bits_to_f32(x).astype("float64") for x in ins)
+    err = O.bf16_bits_to_f32(got[0]).astype("float64") - exact
+    h = hashlib.blake2b(digest_size=8)
+    for x in ins:
+        h.update(x.tobytes())
+    return {"parity_bit_exact": bool(parity), "sampled_tiles": int(len(tiles)),
+            "max_abs_err_vs_exact": float(abs(err).max()), "rms_err_vs_exact": float((err ** 2).mean() ** 0.5),
+            "input_sample_blake2b": h.hexdigest()}
+
+
 def oracle_gbs(op, N, codec, tiles=64):
     """The oracle's rate on a small seeded sample (its cost per tile does not
     depend on the message size): GB/s of N x per-rank message bytes, one core."""
@@ -390,15 +421,30 @@ def run_sweep(args, device):
     peak, peak_src = measured_peaks()
     stream = torch.cuda.current_stream(device)
     cpu = {(N, c): oracle_gbs("allreduce", N, c) for N in W.SWEEP_RANKS for c in W.SWEEP_CODECS}
+    done = set()
+    if args.resume and os.path.exists(args.resume):   # restart: skip the points already written
+        with open(args.resume) as f:
+            for line in f:
+                if line.startswith("{"):
+                    d = json.loads(line)
+                    done.add((d["N"], d["message_bytes"], d["codec"]))
+    sink = open(args.resume, "a") if args.resume else None
     for N in W.SWEEP_RANKS:
         for mb in W.SWEEP_SIZES_BYTES:
+            if all((N, mb, c) in done for c in W.SWEEP_CODECS):
+                continue
             w = W.sweep_workload(N, mb, "bf16")
             xs = W.make_inputs(w, device)
             outs = [torch.empty_like(x) for x in xs]
             wsb = max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS)
             ws = torch.empty(wsb, dtype=torch.uint8, device=device)
             flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # > L2, rewritten between calls
+            T = w.n // TILE
+            rng = torch.Generator().manual_seed(5000 + N)
+            sample = torch.unique(torch.cat([torch.tensor([0, T - 1]), torch.randint(0, T, (2,), generator=rng)]))
             for codec in W.SWEEP_CODECS:
+                if (N, mb, codec) in done:
+                    continue
                 iters = max(3, min(50, int(2e9 / (N * mb))))
                 for _ in range(3):
                     L.lpar_allreduce(xs, w.n, codec, outs, ws, wsb, schedule=args.schedule, stream=stream)
@@ -413,13 +459,18 @@ def run_sweep(args, device):
                 ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
                 names = kernel_names(codec, args.schedule, N)
                 alg = sum(algorithmic_bytes(k, codec, N, w.n) for k in names)
-                print(json.dumps({"sweep": True, "N": N, "message_bytes": mb, "codec": codec,
+                row = json.dumps({"sweep": True, "N": N, "message_bytes": mb, "codec": codec,
                                   "schedule": args.schedule, "ms": ms,
-                                  "GBps": N * mb / (ms * 1e-3) / 1e9,
+                                  "GBps": N * mb / (ms * 1e-3) / 1e9, "algorithmic_bytes": alg,
                                   "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
                                   "l2": "256 MiB buffer rewritten before every timed call",
                                   "note": "L2-resident / launch-bound" if N * mb < (16 << 20) else "",
-                                  "peak": peak, "cpu_baseline": cpu[(N, codec)]}), flush=True)
+                                  "peak": peak, "cpu_baseline": cpu[(N, codec)], "seed": w.seed,
+                                  **sample_check(xs, outs, codec, sample.numpy())})
+                print(row, flush=True)
+                if sink:
+                    sink.write(row + "\n")
+                    sink.flush()
             del xs, outs, ws, flush
             torch.cuda.empty_cache()
 
@@ -517,6 +568,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
+    ap.add_argument("--resume", default=None,
+                    help="with --sweep: append rows to this JSONL file and skip the points it already holds")
     ap.add_argument("--collectives", action="store_true",
                     help="one JSON line per standalone collective point instead of the bench line")
     args = ap.parse_args()
@@ -576,6 +629,7 @@ def main():
             "clocks": res["clocks"],
             "e2e": res["e2e"],
             "cpu_baseline": res["cpu"],
+            "accuracy": res["accuracy"],
             "source_sha": source_sha(),
         }
         print(json.dumps(line), flush=True)

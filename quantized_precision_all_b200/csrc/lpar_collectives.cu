@@ -386,6 +386,7 @@ static inline void mark(const lpar_options_t *opts, int i, cudaStream_t stream) 
 LPAR_API lpar_status_t lpar_reduce_scatter(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                                            void *const *out, void *workspace, size_t workspace_bytes,
                                            const lpar_options_t *opts, cudaStream_t stream) {
+    NvtxRange trace("lpar_reduce_scatter");
     InPtrs in{};
     OutPtrs o{}, wires{};
     lpar_codec_t eff = codec;
@@ -402,6 +403,7 @@ LPAR_API lpar_status_t lpar_reduce_scatter(const void *const *inputs, int N, siz
 LPAR_API lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
                                        void *const *out, void *workspace, size_t workspace_bytes,
                                        const lpar_options_t *opts, cudaStream_t stream) {
+    NvtxRange trace("lpar_all_gather");
     InPtrs in{};
     OutPtrs o{}, wires{};
     lpar_codec_t eff = codec;
@@ -419,6 +421,7 @@ LPAR_API lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t 
 LPAR_API lpar_status_t lpar_all_to_all(const void *const *inputs, int N, size_t m, lpar_codec_t codec,
                                        void *const *out, void *workspace, size_t workspace_bytes,
                                        const lpar_options_t *opts, cudaStream_t stream) {
+    NvtxRange trace("lpar_all_to_all");
     InPtrs in{};
     OutPtrs o{}, wires{};
     lpar_codec_t eff = codec;

@@ -154,6 +154,7 @@ using namespace lpar;
 LPAR_API lpar_status_t lpar_allreduce_f32(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                                           void *const *out, void *workspace, size_t workspace_bytes,
                                           const lpar_options_t *opts, cudaStream_t stream) {
+    NvtxRange trace("lpar_allreduce_f32");
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     const int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_AUTO;
     if (schedule != LPAR_SCHEDULE_AUTO && schedule != LPAR_SCHEDULE_SINGLE_PASS) return LPAR_ERR_UNSUPPORTED;

@@ -400,6 +400,7 @@ LPAR_API const char *lpar_status_string(lpar_status_t s) {
 
 LPAR_API lpar_status_t lpar_quantize(const void *in_bf16, size_t n, lpar_codec_t codec, void *wire,
                                      cudaStream_t stream) {
+    NvtxRange trace("lpar_quantize");
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     if (n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
@@ -420,6 +421,7 @@ LPAR_API lpar_status_t lpar_quantize(const void *in_bf16, size_t n, lpar_codec_t
 
 LPAR_API lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_begin, size_t tile_count,
                                    lpar_codec_t codec, void *wire_out, cudaStream_t stream) {
+    NvtxRange trace("lpar_reduce");
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     if (N < 1 || N > kMaxRanks || !wires) return LPAR_ERR_INVALID_ARG;
     if (tile_begin + tile_count < tile_begin || tile_count > kMaxTiles) return LPAR_ERR_INVALID_ARG;
@@ -446,6 +448,7 @@ LPAR_API lpar_status_t lpar_reduce(const void *const *wires, int N, size_t tile_
 
 LPAR_API lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t codec, void *out_bf16,
                                    cudaStream_t stream) {
+    NvtxRange trace("lpar_decode");
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     if (n % kTileElems != 0 || n / kTileElems > kMaxTiles) return LPAR_ERR_INVALID_ARG;
     if (n == 0) return LPAR_OK;
@@ -461,6 +464,7 @@ LPAR_API lpar_status_t lpar_decode(const void *wire, size_t n, lpar_codec_t code
 LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                                       void *const *out, void *workspace, size_t workspace_bytes,
                                       const lpar_options_t *opts, cudaStream_t stream) {
+    NvtxRange trace("lpar_allreduce");
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_AUTO;
     if (schedule != LPAR_SCHEDULE_AUTO && schedule != LPAR_SCHEDULE_FUSED &&

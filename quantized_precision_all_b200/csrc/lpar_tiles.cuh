@@ -16,6 +16,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #ifndef LPAR_API
 #define LPAR_API extern "C" __attribute__((visibility("default")))
@@ -342,6 +343,15 @@ static bool allow_dynamic_smem(int bytes) {
 
 static inline bool codec_ok(int c) { return c >= LPAR_CODEC_BF16 && c <= LPAR_CODEC_MXFP4; }
 static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around one C ABI call (host-side enqueue), for profilers that
+// record NVTX; without an attached tool it costs a predicted branch.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 static inline lpar_status_t launch_status() {
     return cudaGetLastError() == cudaSuccess ? LPAR_OK : LPAR_ERR_CUDA;
