@@ -200,3 +200,30 @@ def test_large_sampled_tiles(L, op):
                         assert np.array_equal(got, trip[k * 2048:(k + 1) * 2048]), (op, codec, r, t)
         del outs, ws
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# The cross-process all-reduce on the GPU: the library's stages with NCCL
+# collectives.  Only one GPU is available, so this runs one process (the
+# exchanges are NCCL calls on one rank); the orchestration at 2-4 ranks is
+# covered on CPU with gloo (tests/test_distributed_host.py).
+# ---------------------------------------------------------------------------
+def test_cross_process_allreduce_one_rank_nccl(L):
+    import socket
+    import torch.distributed as dist
+    from quantized_precision_all_b200.distributed import DistributedAllreduce
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        ar = DistributedAllreduce()
+        for codec in ("int3", "int4", "fp8", "mxfp4", "bf16"):
+            x = adversarial_bf16(2048 * 6, 4200)
+            out = ar.allreduce(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16), codec)
+            torch.cuda.synchronize()
+            ref, _ = O.allreduce([x], codec)
+            assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), ref[0]), codec
+    finally:
+        dist.destroy_process_group()
