@@ -10,9 +10,13 @@
 //   K23 k_reduce<.., true>   K2 plus the decode of the gathered block straight
 //                        from registers into every rank's BF16 output
 //   K3  k_decode        gathered wire -> BF16 into every rank's output
+//   K123 k_allreduce_single  all three stages in one persistent kernel (the
+//                        default schedule)
 // The BF16 passthrough uses k_bf16_reduce (FP32 sum, one BF16 rounding) and
-// k_broadcast (plain copies).  The work decomposition and the staging are
-// described in lpar_tiles.cuh.
+// k_broadcast (plain copies).  The one-shot schedule's kernel lives with the
+// standalone collectives (lpar_collectives.cu), the binary32 all-reduce in
+// lpar_f32.cu.  The work decomposition and the staging are described in
+// lpar_tiles.cuh.
 #include "lpar.h"
 #include "lpar_codec.cuh"
 #include "lpar_tiles.cuh"
