@@ -510,10 +510,16 @@ def run_collectives(args, device):
     peak, _ = measured_peaks()
     stream = torch.cuda.current_stream(device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    cpu = {(op, N, c): oracle_gbs(op, N, c) for op in COLL_OPS for N in (2, 4, 8) for c in W.SWEEP_CODECS}
-    for op in COLL_OPS:
-        for N in (2, 4, 8):
-            for mb in COLL_SIZES_BYTES:
+    cpu = {(op, N, c): oracle_gbs(op, N, c) for op in (args.coll_op and [args.coll_op] or COLL_OPS)
+           for N in (args.coll_n and [args.coll_n] or (2, 4, 8))
+           for c in (args.coll_codec and [args.coll_codec] or W.SWEEP_CODECS)}
+    ops = [args.coll_op] if args.coll_op else COLL_OPS
+    ranks = [args.coll_n] if args.coll_n else (2, 4, 8)
+    sizes = [args.coll_mib << 20] if args.coll_mib else COLL_SIZES_BYTES
+    codecs = [args.coll_codec] if args.coll_codec else W.SWEEP_CODECS
+    for op in ops:
+        for N in ranks:
+            for mb in sizes:
                 msg = mb // 2
                 size = msg // N if op == "all_to_all" else msg
                 w = W.Workload("collective", N=N, n=msg, dist="student_t", nu=3, seed=9, codecs=("bf16",))
@@ -530,7 +536,7 @@ def run_collectives(args, device):
                         src = [x[:size] for x in xs] if op == "all_gather" else xs
                         getattr(L, "lpar_" + op)(src, size, codec, outs, ws, ws.numel(), stream=stream)
 
-                for codec in W.SWEEP_CODECS:
+                for codec in codecs:
                     for _ in range(3):
                         call(codec)
                     iters = 10
@@ -577,6 +583,11 @@ def main():
                     help="with --sweep: append rows to this JSONL file and skip the points it already holds")
     ap.add_argument("--collectives", action="store_true",
                     help="one JSON line per standalone collective point instead of the bench line")
+    ap.add_argument("--coll-op", choices=["reduce_scatter", "one_shot", "all_gather", "all_to_all"], default=None,
+                    help="with --collectives: only this collective")
+    ap.add_argument("--coll-n", type=int, default=None, help="with --collectives: only this N")
+    ap.add_argument("--coll-mib", type=int, default=None, help="with --collectives: only this per-rank MiB size")
+    ap.add_argument("--coll-codec", default=None, help="with --collectives: only this codec")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.schedule == "auto":                # what the library picks for LPAR_SCHEDULE_AUTO
