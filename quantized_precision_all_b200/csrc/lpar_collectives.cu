@@ -180,52 +180,59 @@ __global__ void __launch_bounds__(kThreads, 4) k_gather_single(const __grid_cons
                                                                const __grid_constant__ OutPtrs wire,
                                                                const __grid_constant__ OutPtrs out, size_t tiles,
                                                                size_t seg_tiles, unsigned chunks, int N) {
-    __shared__ __align__(128) uint8_t stage_in[2][kStageBytes];
-    __shared__ uint8_t *s_dst[kTilesPerCta];
+    // A ring of three BF16 stages.  Item i is staged in stage i % 3 while item
+    // i + 1 is prefetched into the next stage; its decoded chunk replaces its
+    // input in place (in element order; each thread writes only the 64-B
+    // region it read) and leaves through bulk copies issued by lanes of warp 0,
+    // which read the stage while item i + 1 is encoded.  Those lanes wait for
+    // the copies to finish reading before the barrier that precedes the
+    // stage's refill (item i + 2's prefetch).
+    __shared__ __align__(1024) uint8_t stage[3][kStageBytes];
     const int t = threadIdx.x;
     unsigned c = blockIdx.x;
+    if (c >= chunks) return;
     int r = 0;
-    if (c < chunks) {
-        const size_t tile0 = (size_t)c * kTilesPerCta;
-        stage_load_chunk(stage_in[0], in.p[0] + tile0 * (kTileElems * 2),
-                         (int)min((size_t)kTilesPerCta, tiles - tile0));
-    }
+    stage_load_chunk(stage[0], in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
+                     (int)min((size_t)kTilesPerCta, tiles - (size_t)c * kTilesPerCta));
     cp_async_commit();
     int buf = 0;
     while (c < chunks) {
         unsigned cn = c;
         int rn = r + 1;
         if (rn == N) { rn = 0; cn += gridDim.x; }
+        const int nb = buf == 2 ? 0 : buf + 1;
         if (cn < chunks) {
             const size_t tn = (size_t)cn * kTilesPerCta;
-            stage_load_chunk(stage_in[buf ^ 1], in.p[rn] + tn * (kTileElems * 2),
-                             (int)min((size_t)kTilesPerCta, tiles - tn));
+            stage_load_chunk(stage[nb], in.p[rn] + tn * (kTileElems * 2), (int)min((size_t)kTilesPerCta, tiles - tn));
         }
         cp_async_commit();
         cp_async_wait_prev();
-        __syncthreads();
+        __syncthreads();                                   // item landed
         const size_t tile0 = (size_t)c * kTilesPerCta;
         const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
-        // The decoded block replaces the thread's own input bytes in the same
-        // buffer: each thread reads its 64-B region in full before it writes it.
-        uint8_t *stage_out = stage_in[buf];
         if (t < ntiles * kBlocksPerTile)
-            quantize_staged_block<C, true>(stage_in[buf],
-                                           wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t,
-                                           StageSink{stage_out, t});
-        if (A2A && t < ntiles) {
-            const size_t tt = tile0 + t;                   // tile of rank r's message
-            const size_t j = tt / seg_tiles;               // its segment = the receiving rank
-            s_dst[t] = out.p[j] + ((size_t)r * seg_tiles + (tt - j * seg_tiles)) * (kTileElems * 2);
+            quantize_staged_block<C, true>(stage[buf], wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes,
+                                           t, StageSinkLinear{stage[buf], t});
+        fence_async_smem();
+        if (t < 32) bulk_wait_read<0>();                  // the previous item's copies have read their stage
+        __syncthreads();                                   // decoded chunk complete
+        if (A2A) {
+            if (t < ntiles) {                              // tile t of rank r's message -> its segment's rank
+                const size_t tt = tile0 + t;
+                const size_t j = tt / seg_tiles;
+                bulk_store(out.p[j] + ((size_t)r * seg_tiles + (tt - j * seg_tiles)) * (kTileElems * 2),
+                           stage[buf] + t * (kTileElems * 2), kTileElems * 2);
+            }
+        } else if (t < N) {                                // the chunk to output t at rank r's place
+            bulk_store(out.p[t] + ((size_t)r * tiles + tile0) * (kTileElems * 2), stage[buf],
+                       (unsigned)ntiles * (kTileElems * 2));
         }
-        __syncthreads();                                   // stage_out complete, stage_in[buf] consumed
-        if (A2A) stage_to_tile_dsts(stage_out, s_dst, ntiles);
-        else stage_to_outputs(stage_out, out, N, ((size_t)r * tiles + tile0) * (kTileElems * 2), ntiles);
-        __syncthreads();                                   // the buffer is refilled, s_dst rewritten, next item
-        buf ^= 1;
+        if (t < 32) bulk_commit();
+        buf = nb;
         c = cn;
         r = rn;
     }
+    if (t < 32) bulk_wait_all();
 }
 
 // BF16 passthrough of all-gather / all-to-all: copies, one tile of one rank per

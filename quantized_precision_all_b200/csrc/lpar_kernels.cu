@@ -115,22 +115,36 @@ __global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InP
 // itself (same thread, program order).  The next rank's BF16 chunk is
 // prefetched with cp.async while the current one is processed.
 // ---------------------------------------------------------------------------
+// Stages in the single-pass ring (measured on B200, one process timing the
+// variants alternately): four -- three CTAs per SM, 80 registers a thread --
+// for FP8 and, from four ranks on, for INT4 and MXFP4; three -- four CTAs per
+// SM, 64 registers -- for INT3 (its ALU-bound encode wants the warps) and for
+// INT4 and MXFP4 with fewer ranks.
 template <int C, int N>
-__global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_constant__ InPtrs in,
-                                                                  const __grid_constant__ OutPtrs wire,
-                                                                  uint8_t *gather,
-                                                                  const __grid_constant__ OutPtrs out,
-                                                                  size_t tiles, unsigned chunks) {
-    // A ring of three BF16 stages: the item in stage k is prefetched while the
-    // previous one is encoded, and stage k is refilled two items later, after
-    // a barrier that every thread passes only once done with it -- so one
-    // barrier per item.  The decoded chunk is staged in place of the last
-    // rank's input (each thread writes only the 64-B region it read).
-    __shared__ __align__(128) uint8_t stage[3][kStageBytes];
+__host__ __device__ constexpr int ring_stages() { return (C == kFP8 || (C != kINT3 && N >= 4)) ? 4 : 3; }
+template <int C, int N>
+__host__ __device__ constexpr int ring_smem() { return ring_stages<C, N>() * kStageBytes; }
+
+template <int C, int N>
+__global__ void __launch_bounds__(kThreads, ring_stages<C, N>() == 3 ? 4 : 3)
+    k_allreduce_single(const __grid_constant__ InPtrs in, const __grid_constant__ OutPtrs wire, uint8_t *gather,
+                       const __grid_constant__ OutPtrs out, size_t tiles, unsigned chunks) {
+    // A ring of S BF16 stages: item i is staged in stage i % S while item i + 1
+    // is prefetched, and stage i % S is refilled S - 1 items later, after a
+    // barrier that every thread passes only once done with it -- one barrier
+    // per item.  The decoded chunk is staged in place of the last rank's input
+    // (in element order; each thread writes only the 64-B region it read) and
+    // leaves through bulk copies issued by lanes of warp 0, which wait for
+    // them to finish reading before the barrier that precedes the stage's
+    // refill: the next item's (S = 3) or the one after (S = 4), so that with
+    // four stages the copies overlap the encode of the next item.
+    constexpr int S = ring_stages<C, N>();
+    static_assert(S == 3 || S == 4, "ring of three or four stages");
+    extern __shared__ __align__(1024) uint8_t ring[];
     const int t = threadIdx.x;
     unsigned c = blockIdx.x;
     if (c >= chunks) return;
-    stage_load_chunk(stage[0], in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
+    stage_load_chunk(ring, in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
                      (int)min((size_t)kTilesPerCta, tiles - (size_t)c * kTilesPerCta));
     cp_async_commit();
     int buf = 0;
@@ -144,19 +158,26 @@ __global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_c
 #pragma unroll 1
         for (int r = 0; r < N; ++r) {
             // prefetch the next item: rank r+1 of this chunk, or rank 0 of the next chunk
-            const int nb = buf == 2 ? 0 : buf + 1;
+            const int nb = buf + 1 == S ? 0 : buf + 1;
             const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
             if (cn < chunks) {
                 const size_t tn = (size_t)cn * kTilesPerCta;
-                stage_load_chunk(stage[nb], in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
+                stage_load_chunk(ring + nb * kStageBytes, in.p[(r + 1 < N) ? r + 1 : 0] + tn * (kTileElems * 2),
                                  (int)min((size_t)kTilesPerCta, tiles - tn));
             }
             cp_async_commit();
             cp_async_wait_prev();
+            if constexpr (S == 3) {                    // the last chunk's copies
+                if (r == 0 && t < 32) bulk_wait_read<0>();
+            } else if constexpr (N == 1) {             // the copies of the chunk before last
+                if (t < 32) bulk_wait_read<1>();
+            } else {                                   // the last chunk's copies, from its second item on
+                if (r == 1 && t < 32) bulk_wait_read<0>();
+            }
             __syncthreads();                           // item landed; stage nb's old item is done
             if (active) {
                 uint32_t x16[16];
-                stage_read(stage[buf], t, x16);
+                stage_read(ring + buf * kStageBytes, t, x16);
                 float x[32];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
@@ -168,10 +189,14 @@ __global__ void __launch_bounds__(kThreads, 4) k_allreduce_single(const __grid_c
             last = buf;
             buf = nb;
         }
-        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{stage[last], t});
+        uint8_t *const so = ring + last * kStageBytes;
+        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSinkLinear{so, t});
+        fence_async_smem();
         __syncthreads();
-        stage_to_outputs(stage[last], out, N, tile0 * (kTileElems * 2), ntiles);
+        if (t < N) bulk_store(out.p[t] + tile0 * (kTileElems * 2), so, (unsigned)ntiles * (kTileElems * 2));
+        if (t < 32) bulk_commit();
     }
+    if (t < 32) bulk_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -306,38 +331,40 @@ static void launch_bf16_reduce(const InPtrs &in, int N, uint8_t *g, const OutPtr
 }
 
 template <int C, int N>
-static void launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
+static bool launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
                              cudaStream_t st) {
+    if (!allow_dynamic_smem<k_allreduce_single<C, N>>(ring_smem<C, N>())) return false;
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned res = resident_ctas<k_allreduce_single<C, N>>();
-    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 4u));
-    k_allreduce_single<C, N><<<grid, kThreads, 0, st>>>(in, wire, g, o, tiles, chunks);
+    const unsigned res = resident_ctas<k_allreduce_single<C, N>>(ring_smem<C, N>());
+    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 3u));
+    k_allreduce_single<C, N><<<grid, kThreads, ring_smem<C, N>(), st>>>(in, wire, g, o, tiles, chunks);
+    return true;
 }
 
 template <int C>
-static void launch_single_c(const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
+static bool launch_single_c(const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
                             size_t tiles, cudaStream_t st) {
     switch (N) {
-    case 1: launch_single_cn<C, 1>(in, wire, g, o, tiles, st); break;
-    case 2: launch_single_cn<C, 2>(in, wire, g, o, tiles, st); break;
-    case 3: launch_single_cn<C, 3>(in, wire, g, o, tiles, st); break;
-    case 4: launch_single_cn<C, 4>(in, wire, g, o, tiles, st); break;
-    case 5: launch_single_cn<C, 5>(in, wire, g, o, tiles, st); break;
-    case 6: launch_single_cn<C, 6>(in, wire, g, o, tiles, st); break;
-    case 7: launch_single_cn<C, 7>(in, wire, g, o, tiles, st); break;
-    case 8: launch_single_cn<C, 8>(in, wire, g, o, tiles, st); break;
-    default: break;
+    case 1: return launch_single_cn<C, 1>(in, wire, g, o, tiles, st);
+    case 2: return launch_single_cn<C, 2>(in, wire, g, o, tiles, st);
+    case 3: return launch_single_cn<C, 3>(in, wire, g, o, tiles, st);
+    case 4: return launch_single_cn<C, 4>(in, wire, g, o, tiles, st);
+    case 5: return launch_single_cn<C, 5>(in, wire, g, o, tiles, st);
+    case 6: return launch_single_cn<C, 6>(in, wire, g, o, tiles, st);
+    case 7: return launch_single_cn<C, 7>(in, wire, g, o, tiles, st);
+    case 8: return launch_single_cn<C, 8>(in, wire, g, o, tiles, st);
+    default: return false;
     }
 }
 
-static void launch_single(int codec, const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
+static bool launch_single(int codec, const InPtrs &in, const OutPtrs &wire, int N, uint8_t *g, const OutPtrs &o,
                           size_t tiles, cudaStream_t st) {
     switch (codec) {
-    case kINT4: launch_single_c<kINT4>(in, wire, N, g, o, tiles, st); break;
-    case kINT3: launch_single_c<kINT3>(in, wire, N, g, o, tiles, st); break;
-    case kFP8: launch_single_c<kFP8>(in, wire, N, g, o, tiles, st); break;
-    case kMXFP4: launch_single_c<kMXFP4>(in, wire, N, g, o, tiles, st); break;
-    default: break;
+    case kINT4: return launch_single_c<kINT4>(in, wire, N, g, o, tiles, st);
+    case kINT3: return launch_single_c<kINT3>(in, wire, N, g, o, tiles, st);
+    case kFP8: return launch_single_c<kFP8>(in, wire, N, g, o, tiles, st);
+    case kMXFP4: return launch_single_c<kMXFP4>(in, wire, N, g, o, tiles, st);
+    default: return false;
     }
 }
 
@@ -535,7 +562,7 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
     uint8_t *gather = ws + (size_t)N * wb;
     mark(0);
     if (schedule == LPAR_SCHEDULE_SINGLE_PASS) {
-        launch_single(eff, in, wires, N, gather, o, tiles, stream);
+        if (!launch_single(eff, in, wires, N, gather, o, tiles, stream)) return LPAR_ERR_CUDA;
         mark(1);
         return launch_status();
     }

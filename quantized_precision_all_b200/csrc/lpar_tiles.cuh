@@ -43,6 +43,25 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// Bulk asynchronous copies from shared to global memory, done by the TMA engine
+// (no tensor map: both addresses 16-B aligned, a multiple of 16 bytes).  Each
+// issuing thread tracks its own groups: commit after its copies, wait_read<K>
+// before the shared source is rewritten (at most K newest groups still read
+// it), wait_all before the CTA exits.  Shared-memory writes of the generic
+// proxy reach the copies through fence_async_smem() and a barrier.
+__device__ __forceinline__ void bulk_store(void *gmem, const void *smem, unsigned bytes) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem), "r"(s), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int K>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(K) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // Packed block <-> tile bytes.
 // ---------------------------------------------------------------------------
@@ -145,6 +164,16 @@ struct StageSink {                                   // BF16 (RNE) into thread t
     __device__ __forceinline__ void put(int j, float a0, float a1, float a2, float a3, float a4, float a5, float a6,
                                         float a7) const {
         *reinterpret_cast<uint4 *>(stage + swz(t, j)) =
+            make_uint4(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3), pack_bf16x2(a4, a5), pack_bf16x2(a6, a7));
+    }
+};
+
+struct StageSinkLinear {                             // BF16 (RNE), thread t's 64-B region in element order
+    uint8_t *stage;                                  // (the layout a bulk copy sends as it is)
+    int t;
+    __device__ __forceinline__ void put(int j, float a0, float a1, float a2, float a3, float a4, float a5, float a6,
+                                        float a7) const {
+        *reinterpret_cast<uint4 *>(stage + 64 * t + 16 * j) =
             make_uint4(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3), pack_bf16x2(a4, a5), pack_bf16x2(a6, a7));
     }
 };
