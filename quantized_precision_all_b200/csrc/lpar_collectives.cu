@@ -175,24 +175,40 @@ __global__ void __launch_bounds__(kThreads) k_bf16_reduce_to(const __grid_consta
 // receiver decodes from the wire, which is written as the transmitted data).
 // seg_tiles is the segment length m / 2048 (all-gather: the whole message).
 // ---------------------------------------------------------------------------
+// Stages in the gather ring (measured on B200, one process timing the
+// variants alternately): the all-gather's time does not move from three to six
+// stages, so it keeps three (four CTAs per SM); the all-to-all, whose copies
+// are one tile each, gains from deeper rings -- five stages for FP8 (9% at
+// N = 8), four for the others (2-4%).
 template <int C, bool A2A>
-__global__ void __launch_bounds__(kThreads, 4) k_gather_single(const __grid_constant__ InPtrs in,
-                                                               const __grid_constant__ OutPtrs wire,
-                                                               const __grid_constant__ OutPtrs out, size_t tiles,
-                                                               size_t seg_tiles, unsigned chunks, int N) {
-    // A ring of three BF16 stages.  Item i is staged in stage i % 3 while item
+__host__ __device__ constexpr int gather_stages() { return A2A ? (C == kFP8 ? 5 : 4) : 3; }
+template <int C, bool A2A>
+__host__ __device__ constexpr int gather_smem() { return gather_stages<C, A2A>() * kStageBytes; }
+template <int C, bool A2A>
+__host__ __device__ constexpr int gather_min_ctas() {       // CTAs per SM the ring's shared memory allows
+    return gather_stages<C, A2A>() == 3 ? 4 : (gather_stages<C, A2A>() == 4 ? 3 : 2);
+}
+
+template <int C, bool A2A>
+__global__ void __launch_bounds__(kThreads, gather_min_ctas<C, A2A>())
+    k_gather_single(const __grid_constant__ InPtrs in, const __grid_constant__ OutPtrs wire,
+                    const __grid_constant__ OutPtrs out, size_t tiles, size_t seg_tiles, unsigned chunks, int N) {
+    // A ring of S BF16 stages.  Item i is staged in stage i % S while item
     // i + 1 is prefetched into the next stage; its decoded chunk replaces its
     // input in place (in element order; each thread writes only the 64-B
     // region it read) and leaves through bulk copies issued by lanes of warp 0,
-    // which read the stage while item i + 1 is encoded.  Those lanes wait for
-    // the copies to finish reading before the barrier that precedes the
-    // stage's refill (item i + 2's prefetch).
-    __shared__ __align__(1024) uint8_t stage[3][kStageBytes];
+    // which read the stage while the following items are encoded.  Stage i % S
+    // is refilled by item i + S - 1's prefetch, so before the barrier that
+    // closes item i + S - 2 those lanes wait until at most the S - 3 newest
+    // groups of copies are still reading.
+    constexpr int S = gather_stages<C, A2A>();
+    static_assert(S >= 3 && S <= 5, "ring of three to five stages");
+    extern __shared__ __align__(1024) uint8_t ring[];
     const int t = threadIdx.x;
     unsigned c = blockIdx.x;
     if (c >= chunks) return;
     int r = 0;
-    stage_load_chunk(stage[0], in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
+    stage_load_chunk(ring, in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2),
                      (int)min((size_t)kTilesPerCta, tiles - (size_t)c * kTilesPerCta));
     cp_async_commit();
     int buf = 0;
@@ -200,31 +216,33 @@ __global__ void __launch_bounds__(kThreads, 4) k_gather_single(const __grid_cons
         unsigned cn = c;
         int rn = r + 1;
         if (rn == N) { rn = 0; cn += gridDim.x; }
-        const int nb = buf == 2 ? 0 : buf + 1;
+        const int nb = buf + 1 == S ? 0 : buf + 1;
         if (cn < chunks) {
             const size_t tn = (size_t)cn * kTilesPerCta;
-            stage_load_chunk(stage[nb], in.p[rn] + tn * (kTileElems * 2), (int)min((size_t)kTilesPerCta, tiles - tn));
+            stage_load_chunk(ring + nb * kStageBytes, in.p[rn] + tn * (kTileElems * 2),
+                             (int)min((size_t)kTilesPerCta, tiles - tn));
         }
         cp_async_commit();
         cp_async_wait_prev();
         __syncthreads();                                   // item landed
+        uint8_t *const st = ring + buf * kStageBytes;
         const size_t tile0 = (size_t)c * kTilesPerCta;
         const int ntiles = (int)min((size_t)kTilesPerCta, tiles - tile0);
         if (t < ntiles * kBlocksPerTile)
-            quantize_staged_block<C, true>(stage[buf], wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes,
-                                           t, StageSinkLinear{stage[buf], t});
+            quantize_staged_block<C, true>(st, wire.p[r] + (tile0 + t / kBlocksPerTile) * Layout<C>::kTileBytes, t,
+                                           StageSinkLinear{st, t});
         fence_async_smem();
-        if (t < 32) bulk_wait_read<0>();                  // the previous item's copies have read their stage
+        if (t < 32) bulk_wait_read<S - 3>();
         __syncthreads();                                   // decoded chunk complete
         if (A2A) {
             if (t < ntiles) {                              // tile t of rank r's message -> its segment's rank
                 const size_t tt = tile0 + t;
                 const size_t j = tt / seg_tiles;
                 bulk_store(out.p[j] + ((size_t)r * seg_tiles + (tt - j * seg_tiles)) * (kTileElems * 2),
-                           stage[buf] + t * (kTileElems * 2), kTileElems * 2);
+                           st + t * (kTileElems * 2), kTileElems * 2);
             }
         } else if (t < N) {                                // the chunk to output t at rank r's place
-            bulk_store(out.p[t] + ((size_t)r * tiles + tile0) * (kTileElems * 2), stage[buf],
+            bulk_store(out.p[t] + ((size_t)r * tiles + tile0) * (kTileElems * 2), st,
                        (unsigned)ntiles * (kTileElems * 2));
         }
         if (t < 32) bulk_commit();
@@ -313,24 +331,28 @@ void launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, con
 }
 
 template <int C, bool A2A>
-static void launch_gather_c(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
+static bool launch_gather_c(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
                             size_t seg_tiles, cudaStream_t st) {
+    constexpr int smem = gather_smem<C, A2A>();
+    if (!allow_dynamic_smem<k_gather_single<C, A2A>>(smem)) return false;
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned grid = persistent_grid(chunks, resident_ctas<k_gather_single<C, A2A>>());
-    k_gather_single<C, A2A><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, seg_tiles, chunks, N);
+    const unsigned grid = persistent_grid(chunks, resident_ctas<k_gather_single<C, A2A>>(smem));
+    k_gather_single<C, A2A><<<grid, kThreads, smem, st>>>(in, wire, out, tiles, seg_tiles, chunks, N);
+    return true;
 }
 
 template <bool A2A>
-static void launch_gather(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
+static bool launch_gather(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
                           size_t tiles, size_t seg_tiles, cudaStream_t st) {
     switch (codec) {
-    case kINT4: launch_gather_c<kINT4, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
-    case kINT3: launch_gather_c<kINT3, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
-    case kFP8: launch_gather_c<kFP8, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
-    case kMXFP4: launch_gather_c<kMXFP4, A2A>(in, wire, out, N, tiles, seg_tiles, st); break;
+    case kINT4: return launch_gather_c<kINT4, A2A>(in, wire, out, N, tiles, seg_tiles, st);
+    case kINT3: return launch_gather_c<kINT3, A2A>(in, wire, out, N, tiles, seg_tiles, st);
+    case kFP8: return launch_gather_c<kFP8, A2A>(in, wire, out, N, tiles, seg_tiles, st);
+    case kMXFP4: return launch_gather_c<kMXFP4, A2A>(in, wire, out, N, tiles, seg_tiles, st);
     default: {
         const dim3 grid((unsigned)std::min<size_t>(tiles, (size_t)1 << 20), (unsigned)N);
         k_bf16_gather<A2A><<<grid, kThreads, 0, st>>>(in, out, tiles, seg_tiles, N);
+        return true;
     }
     }
 }
@@ -420,7 +442,7 @@ LPAR_API lpar_status_t lpar_all_gather(const void *const *inputs, int N, size_t 
     if (st != LPAR_OK || n_msg == 0) return st;
     const size_t tiles = m / kTileElems;
     mark(opts, 0, stream);
-    launch_gather<false>(eff, in, wires, o, N, tiles, tiles, stream);
+    if (!launch_gather<false>(eff, in, wires, o, N, tiles, tiles, stream)) return LPAR_ERR_CUDA;
     mark(opts, 1, stream);
     return launch_status();
 }
@@ -437,7 +459,7 @@ LPAR_API lpar_status_t lpar_all_to_all(const void *const *inputs, int N, size_t 
                                               workspace_bytes, opts, in, o, wires, eff, n_msg);
     if (st != LPAR_OK || n_msg == 0) return st;
     mark(opts, 0, stream);
-    launch_gather<true>(eff, in, wires, o, N, n_msg / kTileElems, m / kTileElems, stream);
+    if (!launch_gather<true>(eff, in, wires, o, N, n_msg / kTileElems, m / kTileElems, stream)) return LPAR_ERR_CUDA;
     mark(opts, 1, stream);
     return launch_status();
 }
