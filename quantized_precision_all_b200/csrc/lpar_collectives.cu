@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, gather_min_ctas<C, A2A>())
         c = cn;
         r = rn;
     }
-    if (t < 32) bulk_wait_all();
+    if (t < 32) bulk_wait_read<0>();                  // the stage outlives no copy that reads it
 }
 
 // BF16 passthrough of all-gather / all-to-all: copies, one tile of one rank per

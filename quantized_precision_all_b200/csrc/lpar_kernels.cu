@@ -115,30 +115,44 @@ __global__ void __launch_bounds__(kThreads) k_reduce(const __grid_constant__ InP
 // itself (same thread, program order).  The next rank's BF16 chunk is
 // prefetched with cp.async while the current one is processed.
 // ---------------------------------------------------------------------------
-// Stages in the single-pass ring (measured on B200, one process timing the
-// variants alternately): four -- three CTAs per SM, 80 registers a thread --
-// for FP8 and, from four ranks on, for INT4 and MXFP4; three -- four CTAs per
-// SM, 64 registers -- for INT3 (its ALU-bound encode wants the warps) and for
-// INT4 and MXFP4 with fewer ranks.
-template <int C, int N>
-__host__ __device__ constexpr int ring_stages() { return (C == kFP8 || (C != kINT3 && N >= 4)) ? 4 : 3; }
-template <int C, int N>
-__host__ __device__ constexpr int ring_smem() { return ring_stages<C, N>() * kStageBytes; }
+// Output of the single-pass kernel.  BULK: the decoded chunk is staged in
+// element order and sent by the TMA engine (bulk shared->global copies), so a
+// CTA moves on while the copies drain; otherwise every thread stores its
+// share of the staged chunk to each output.  The copies add about 2 us of
+// latency to a call and win on throughput, so the launcher takes them from
+// kBulkMinBytes of input (N x message bytes) on (measured on B200 with the
+// variants timed alternately in one process: below about 128 MiB the
+// synchronous stores are faster, above it the copies by 2-12%).
+constexpr size_t kBulkMinBytes = (size_t)128 << 20;
 
-template <int C, int N>
-__global__ void __launch_bounds__(kThreads, ring_stages<C, N>() == 3 ? 4 : 3)
+// Stages in the single-pass ring (measured the same way): with the bulk
+// copies, four -- three CTAs per SM, 80 registers a thread -- for FP8 and,
+// from four ranks on, for INT4 and MXFP4; three -- four CTAs per SM, 64
+// registers -- for INT3 (its ALU-bound encode wants the warps) and for INT4
+// and MXFP4 with fewer ranks.  The synchronous stores need three.
+template <int C, int N, bool BULK>
+__host__ __device__ constexpr int ring_stages() {
+    return (BULK && (C == kFP8 || (C != kINT3 && N >= 4))) ? 4 : 3;
+}
+template <int C, int N, bool BULK>
+__host__ __device__ constexpr int ring_smem() { return ring_stages<C, N, BULK>() * kStageBytes; }
+
+template <int C, int N, bool BULK>
+__global__ void __launch_bounds__(kThreads, ring_stages<C, N, BULK>() == 3 ? 4 : 3)
     k_allreduce_single(const __grid_constant__ InPtrs in, const __grid_constant__ OutPtrs wire, uint8_t *gather,
                        const __grid_constant__ OutPtrs out, size_t tiles, unsigned chunks) {
     // A ring of S BF16 stages: item i is staged in stage i % S while item i + 1
     // is prefetched, and stage i % S is refilled S - 1 items later, after a
     // barrier that every thread passes only once done with it -- one barrier
     // per item.  The decoded chunk is staged in place of the last rank's input
-    // (in element order; each thread writes only the 64-B region it read) and
-    // leaves through bulk copies issued by lanes of warp 0, which wait for
-    // them to finish reading before the barrier that precedes the stage's
-    // refill: the next item's (S = 3) or the one after (S = 4), so that with
-    // four stages the copies overlap the encode of the next item.
-    constexpr int S = ring_stages<C, N>();
+    // (each thread writes only the 64-B region it read).  Synchronous output:
+    // every thread copies its share to the N outputs before the next item's
+    // barrier.  Bulk output: the chunk leaves through copies issued by lanes
+    // of warp 0, which wait for them to finish reading before the barrier
+    // that precedes the stage's refill -- the next item's (S = 3) or the one
+    // after (S = 4), so that with four stages the copies overlap the encode
+    // of the next item.
+    constexpr int S = ring_stages<C, N, BULK>();
     static_assert(S == 3 || S == 4, "ring of three or four stages");
     extern __shared__ __align__(1024) uint8_t ring[];
     const int t = threadIdx.x;
@@ -167,12 +181,14 @@ __global__ void __launch_bounds__(kThreads, ring_stages<C, N>() == 3 ? 4 : 3)
             }
             cp_async_commit();
             cp_async_wait_prev();
-            if constexpr (S == 3) {                    // the last chunk's copies
-                if (r == 0 && t < 32) bulk_wait_read<0>();
-            } else if constexpr (N == 1) {             // the copies of the chunk before last
-                if (t < 32) bulk_wait_read<1>();
-            } else {                                   // the last chunk's copies, from its second item on
-                if (r == 1 && t < 32) bulk_wait_read<0>();
+            if constexpr (BULK) {
+                if constexpr (S == 3) {                // the last chunk's copies
+                    if (r == 0 && t < 32) bulk_wait_read<0>();
+                } else if constexpr (N == 1) {         // the copies of the chunk before last
+                    if (t < 32) bulk_wait_read<1>();
+                } else {                               // the last chunk's copies, from its second item on
+                    if (r == 1 && t < 32) bulk_wait_read<0>();
+                }
             }
             __syncthreads();                           // item landed; stage nb's old item is done
             if (active) {
@@ -190,13 +206,21 @@ __global__ void __launch_bounds__(kThreads, ring_stages<C, N>() == 3 ? 4 : 3)
             buf = nb;
         }
         uint8_t *const so = ring + last * kStageBytes;
-        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSinkLinear{so, t});
-        fence_async_smem();
-        __syncthreads();
-        if (t < N) bulk_store(out.p[t] + tile0 * (kTileElems * 2), so, (unsigned)ntiles * (kTileElems * 2));
-        if (t < 32) bulk_commit();
+        if constexpr (BULK) {
+            if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSinkLinear{so, t});
+            fence_async_smem();
+            __syncthreads();
+            if (t < N) bulk_store(out.p[t] + tile0 * (kTileElems * 2), so, (unsigned)ntiles * (kTileElems * 2));
+            if (t < 32) bulk_commit();
+        } else {
+            if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{so, t});
+            __syncthreads();
+            stage_to_outputs(so, out, N, tile0 * (kTileElems * 2), ntiles);
+        }
     }
-    if (t < 32) bulk_wait_all();
+    if constexpr (BULK) {
+        if (t < 32) bulk_wait_read<0>();              // the stage outlives no copy that reads it
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -330,15 +354,24 @@ static void launch_bf16_reduce(const InPtrs &in, int N, uint8_t *g, const OutPtr
     }
 }
 
+template <int C, int N, bool BULK>
+static bool launch_single_cnb(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
+                              cudaStream_t st) {
+    constexpr int smem = ring_smem<C, N, BULK>();
+    if (!allow_dynamic_smem<k_allreduce_single<C, N, BULK>>(smem)) return false;
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned res = resident_ctas<k_allreduce_single<C, N, BULK>>(smem);
+    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 3u));
+    k_allreduce_single<C, N, BULK><<<grid, kThreads, smem, st>>>(in, wire, g, o, tiles, chunks);
+    return true;
+}
+
 template <int C, int N>
 static bool launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
                              cudaStream_t st) {
-    if (!allow_dynamic_smem<k_allreduce_single<C, N>>(ring_smem<C, N>())) return false;
-    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned res = resident_ctas<k_allreduce_single<C, N>>(ring_smem<C, N>());
-    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 3u));
-    k_allreduce_single<C, N><<<grid, kThreads, ring_smem<C, N>(), st>>>(in, wire, g, o, tiles, chunks);
-    return true;
+    if ((size_t)N * tiles * (kTileElems * 2) >= kBulkMinBytes)
+        return launch_single_cnb<C, N, true>(in, wire, g, o, tiles, st);
+    return launch_single_cnb<C, N, false>(in, wire, g, o, tiles, st);
 }
 
 template <int C>

@@ -47,8 +47,10 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // (no tensor map: both addresses 16-B aligned, a multiple of 16 bytes).  Each
 // issuing thread tracks its own groups: commit after its copies, wait_read<K>
 // before the shared source is rewritten (at most K newest groups still read
-// it), wait_all before the CTA exits.  Shared-memory writes of the generic
-// proxy reach the copies through fence_async_smem() and a barrier.
+// it), and wait_read<0> before the CTA exits, since its shared memory is then
+// released; the global writes themselves are complete when the grid is.
+// Shared-memory writes of the generic proxy reach the copies through
+// fence_async_smem() and a barrier.
 __device__ __forceinline__ void bulk_store(void *gmem, const void *smem, unsigned bytes) {
     const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem), "r"(s), "r"(bytes)
@@ -59,7 +61,6 @@ template <int K>
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(K) : "memory");
 }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------

@@ -531,6 +531,44 @@ def test_workload_large_sampled_tiles(L, name):
 
 
 # ---------------------------------------------------------------------------
+# The single-pass kernel's bulk output path (messages of N x 2n >= 128 MiB) with
+# odd rank counts and a ragged last chunk (T % 4 == 3).  Student-t inputs drawn
+# on the GPU, with adversarial tiles planted at the sampled positions; sampled
+# tiles are compared bit for bit.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4"])
+@pytest.mark.parametrize("N", [1, 3, 5])
+def test_bulk_output_path_ragged_tail(L, codec, N):
+    T = -(-(128 << 20) // (N * 4096))
+    T += (3 - T % 4) % 4                             # T % 4 == 3: the last chunk holds three tiles
+    assert N * T * 4096 >= (128 << 20) and T % 4 == 3
+    n = T * 2048
+    g = torch.Generator(device="cuda")
+    xs = []
+    for r in range(N):
+        g.manual_seed(77 * 1009 + r)
+        z = torch.randn(n, generator=g, device="cuda")
+        c = sum(torch.randn(n, generator=g, device="cuda") ** 2 for _ in range(3))
+        xs.append((z / torch.sqrt(c / 3)).to(torch.bfloat16))
+    rng = np.random.default_rng(600 + N)
+    tiles = np.unique(np.concatenate([np.arange(4), np.arange(T - 7, T), rng.choice(T, 48, replace=False)]))
+    idx = torch.from_numpy((tiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
+    for r in range(N):                               # adversarial blocks at the sampled tiles
+        adv = adversarial_bf16(len(tiles) * 2048, 6100 + 10 * N + r)
+        xs[r][idx] = torch.from_numpy(adv.view(np.int16)).cuda().view(torch.bfloat16)
+    sample_in = [x[idx].view(torch.int16).cpu().numpy().view(np.uint16) for x in xs]
+    ref, _ = O.allreduce(sample_in, codec)
+    outs = [torch.empty_like(x) for x in xs]
+    ws = torch.empty(L.lpar_workspace_bytes(N, n, codec), dtype=torch.uint8, device="cuda")
+    L.lpar_allreduce(xs, n, codec, outs, ws, ws.numel(), schedule="single_pass")
+    torch.cuda.synchronize()
+    for o in outs:
+        assert np.array_equal(o[idx].view(torch.int16).cpu().numpy().view(np.uint16), ref[0]), (codec, N)
+    del xs, outs, ws
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # The sweep: 128 KiB ... 1 GiB per rank, N in {2, 4, 8}, every codec, Student-t
 # (nu = 3).  Each point runs at full size on the GPU; the oracle checks the
 # first and last tile plus 62 seeded random tiles (a tile's result depends only
