@@ -262,6 +262,43 @@ lpar_status_t lpar_allreduce_f32(const void *const *inputs, int N, size_t n, lpa
 lpar_status_t lpar_allreduce_static(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                                     void *const *out, const lpar_options_t *opts, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The all-reduce of messages held in host memory.  The pages have no
+ * counterpart; it serves callers whose tensors live on the host.  A tile's
+ * result depends only on the same tile of every rank, so the message is
+ * reduced chunk by chunk (chunks of whole tiles) on three streams of the
+ * library's own -- upload of chunk k + 1, lpar_allreduce of chunk k (in place,
+ * in device staging) and download of chunk k - 1 at the same time -- and the
+ * result equals that of one lpar_allreduce of the whole message with the same
+ * options.  The threshold opts->min_quant_bytes is decided once on the whole
+ * message (2n bytes); opts->schedule applies to every chunk; stage events [0]
+ * and [1] are recorded on `stream` before the first copy and after the last.
+ * ------------------------------------------------------------------------- */
+
+/* Device bytes lpar_allreduce_host needs for chunks of `chunk` elements (a
+ * multiple of 2048) with `codec` (the one that runs after the threshold):
+ * three staging slots of N chunks plus the workspace of one chunk.  0 for N
+ * outside [1, LPAR_MAX_RANKS], chunk 0 or not a multiple of 2048, or an
+ * unknown codec. */
+size_t lpar_host_staging_bytes(int N, size_t chunk, lpar_codec_t codec);
+
+/* host_inputs[r], host_out[r]: N host arrays of n BF16 values (n a multiple of
+ * 2048); host_out[r] may equal host_inputs[r].  Page-locked host memory
+ * (cudaHostAlloc or cudaHostRegister) lets the copies overlap each other and
+ * the kernels; pageable memory gives the same result with the copies
+ * serialised.  chunk: elements per chunk, a multiple of 2048 (a chunk larger
+ * than n is n).  device: at least lpar_host_staging_bytes(N, min(chunk, n),
+ * effective codec) bytes of device memory, 16-byte aligned, owned by the
+ * caller.  The work is ordered after earlier work on `stream`, and later work
+ * on `stream` runs after the last result has reached host memory; the call
+ * returns once everything is enqueued.  Not for stream capture (the library
+ * creates and releases its streams inside the call).  Argument errors are
+ * returned before anything is enqueued; after LPAR_ERR_CUDA, work already
+ * enqueued may still run. */
+lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
+                                  void *const *host_out, size_t chunk, void *device, size_t device_bytes,
+                                  const lpar_options_t *opts, cudaStream_t stream);
+
 /* The codec lpar_allreduce runs for these arguments after the threshold. */
 lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts);
 

@@ -1,0 +1,145 @@
+// lpar_host.cu -- lpar_allreduce_host: the all-reduce of messages held in host
+// memory, with the copies in both directions and the kernels overlapped.
+//
+// A tile's result depends only on the same tile of every rank, so the message
+// can be reduced chunk by chunk (chunks of whole tiles) and the result is the
+// one a single lpar_allreduce of the whole message gives.  Three streams carry
+// the work of chunk k, in a ring of three device staging slots (slot k % 3,
+// each holding the N ranks' chunk, reduced in place):
+//   up    waits until slot k % 3 has been copied out (chunk k - 3), copies the
+//         N input chunks in;
+//   comp  waits for them, runs lpar_allreduce in place;
+//   down  waits for it, copies the N result chunks out.
+// So the upload of chunk k + 1, the kernel of chunk k and the download of
+// chunk k - 1 run at the same time: with page-locked host buffers the time is
+// bound by the slower PCIe direction instead of the sum of both.  The
+// threshold is decided once, on the whole message, and every chunk runs with
+// the codec it selects.  The streams and events are created per call and
+// released when their work is done; the library keeps nothing.
+#include "lpar.h"
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#define LPAR_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr size_t kTile = 2048;   // elements per tile
+constexpr int kSlots = 3;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round16(size_t b) { return (b + 15) & ~(size_t)15; }
+
+// Byte layout of the device buffer: kSlots x N chunk buffers (2 * chunk bytes
+// each, 16-byte aligned), then the workspace of one chunk.
+size_t chunk_buffer_bytes(size_t chunk) { return round16(2 * chunk); }
+
+struct Pipeline {
+    cudaStream_t st[3] = {nullptr, nullptr, nullptr};   // up, comp, down
+    cudaEvent_t start = nullptr, up[kSlots] = {}, comp[kSlots] = {}, down[kSlots] = {};
+    bool ok = true;
+
+    Pipeline() {
+        for (auto &s : st) ok = ok && cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&start, cudaEventDisableTiming) == cudaSuccess;
+        for (int k = 0; k < kSlots; ++k) {
+            ok = ok && cudaEventCreateWithFlags(&up[k], cudaEventDisableTiming) == cudaSuccess;
+            ok = ok && cudaEventCreateWithFlags(&comp[k], cudaEventDisableTiming) == cudaSuccess;
+            ok = ok && cudaEventCreateWithFlags(&down[k], cudaEventDisableTiming) == cudaSuccess;
+        }
+    }
+    // Destroying a stream or an event with work pending returns at once; the
+    // resources are released when the work completes.
+    ~Pipeline() {
+        for (auto &s : st)
+            if (s) cudaStreamDestroy(s);
+        if (start) cudaEventDestroy(start);
+        for (int k = 0; k < kSlots; ++k) {
+            if (up[k]) cudaEventDestroy(up[k]);
+            if (comp[k]) cudaEventDestroy(comp[k]);
+            if (down[k]) cudaEventDestroy(down[k]);
+        }
+    }
+};
+
+}  // namespace
+
+LPAR_API size_t lpar_host_staging_bytes(int N, size_t chunk, lpar_codec_t codec) {
+    if (N < 1 || N > LPAR_MAX_RANKS || chunk == 0 || chunk % kTile) return 0;
+    const size_t ws = lpar_workspace_bytes(N, chunk, codec);
+    if (ws == 0 && codec != LPAR_CODEC_BF16) return 0;
+    return (size_t)kSlots * N * chunk_buffer_bytes(chunk) + round16(ws);
+}
+
+LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
+                                           void *const *host_out, size_t chunk, void *device, size_t device_bytes,
+                                           const lpar_options_t *opts, cudaStream_t stream) {
+    if (N < 1 || N > LPAR_MAX_RANKS || n % kTile || chunk == 0 || chunk % kTile) return LPAR_ERR_INVALID_ARG;
+    if (codec < LPAR_CODEC_BF16 || codec > LPAR_CODEC_MXFP4) return LPAR_ERR_UNSUPPORTED;
+    if (opts && opts->schedule > LPAR_SCHEDULE_ONE_SHOT) return LPAR_ERR_UNSUPPORTED;
+    if (n == 0) return LPAR_OK;
+    if (!host_inputs || !host_out || !device) return LPAR_ERR_INVALID_ARG;
+    for (int r = 0; r < N; ++r)
+        if (!host_inputs[r] || !host_out[r]) return LPAR_ERR_INVALID_ARG;
+    if (!aligned16(device)) return LPAR_ERR_MISALIGNED;
+    if (chunk > n) chunk = n;
+    const lpar_codec_t eff = lpar_effective_codec(n, codec, opts);    // decided on the whole message
+    if (device_bytes < lpar_host_staging_bytes(N, chunk, eff)) return LPAR_ERR_WORKSPACE_TOO_SMALL;
+
+    lpar_options_t per_chunk{};
+    per_chunk.min_quant_bytes = 0;
+    per_chunk.schedule = opts ? opts->schedule : LPAR_SCHEDULE_AUTO;
+    uint8_t *const base = static_cast<uint8_t *>(device);
+    const size_t cb = chunk_buffer_bytes(chunk);
+    uint8_t *const ws = base + (size_t)kSlots * N * cb;
+    const size_t ws_bytes = device_bytes - (size_t)kSlots * N * cb;
+
+    Pipeline p;
+    if (!p.ok) return LPAR_ERR_CUDA;
+    cudaStream_t up = p.st[0], comp = p.st[1], down = p.st[2];
+    if (opts && opts->stage_events[0]) cudaEventRecord(opts->stage_events[0], stream);
+    if (cudaEventRecord(p.start, stream) != cudaSuccess) return LPAR_ERR_CUDA;
+    for (cudaStream_t s : p.st)
+        if (cudaStreamWaitEvent(s, p.start, 0) != cudaSuccess) return LPAR_ERR_CUDA;
+
+    const size_t chunks = (n + chunk - 1) / chunk;
+    int last = 0;
+    for (size_t k = 0; k < chunks; ++k) {
+        const int s = (int)(k % kSlots);
+        const size_t e0 = k * chunk, elems = (n - e0 < chunk) ? n - e0 : chunk;
+        const void *in[LPAR_MAX_RANKS];
+        void *out[LPAR_MAX_RANKS];
+        for (int r = 0; r < N; ++r) {
+            uint8_t *slot = base + ((size_t)s * N + r) * cb;
+            in[r] = slot;
+            out[r] = slot;
+        }
+        bool ok = true;
+        // up: the slot is free once chunk k - 3 has been copied out
+        if (k >= kSlots) ok = ok && cudaStreamWaitEvent(up, p.down[s], 0) == cudaSuccess;
+        for (int r = 0; r < N && ok; ++r)
+            ok = cudaMemcpyAsync(out[r], static_cast<const uint8_t *>(host_inputs[r]) + 2 * e0, 2 * elems,
+                                 cudaMemcpyHostToDevice, up) == cudaSuccess;
+        ok = ok && cudaEventRecord(p.up[s], up) == cudaSuccess;
+        // comp: the all-reduce of the chunk, in place
+        ok = ok && cudaStreamWaitEvent(comp, p.up[s], 0) == cudaSuccess;
+        if (!ok) return LPAR_ERR_CUDA;
+        const lpar_status_t st = lpar_allreduce(in, N, elems, eff, out, ws, ws_bytes, &per_chunk, comp);
+        if (st != LPAR_OK) return st;
+        ok = cudaEventRecord(p.comp[s], comp) == cudaSuccess;
+        // down: the N result chunks back to the host
+        ok = ok && cudaStreamWaitEvent(down, p.comp[s], 0) == cudaSuccess;
+        for (int r = 0; r < N && ok; ++r)
+            ok = cudaMemcpyAsync(static_cast<uint8_t *>(host_out[r]) + 2 * e0, out[r], 2 * elems,
+                                 cudaMemcpyDeviceToHost, down) == cudaSuccess;
+        ok = ok && cudaEventRecord(p.down[s], down) == cudaSuccess;
+        if (!ok) return LPAR_ERR_CUDA;
+        last = s;
+    }
+    // later work on `stream` runs after the last download (the down stream is in order)
+    if (cudaStreamWaitEvent(stream, p.down[last], 0) != cudaSuccess) return LPAR_ERR_CUDA;
+    if (opts && opts->stage_events[1]) cudaEventRecord(opts->stage_events[1], stream);
+    return cudaGetLastError() == cudaSuccess ? LPAR_OK : LPAR_ERR_CUDA;
+}

@@ -33,7 +33,7 @@ MAX_RANKS = 8
 EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
            "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string",
            "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all",
-           "lpar_allreduce_f32")
+           "lpar_allreduce_f32", "lpar_host_staging_bytes", "lpar_allreduce_host")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -68,6 +68,8 @@ def _load():
         "lpar_all_gather": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_all_to_all": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_allreduce_f32": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_host_staging_bytes": (sz, [i32, sz, i32]),
+        "lpar_allreduce_host": (i32, [vpp, i32, sz, i32, vpp, sz, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -101,11 +103,21 @@ def _ptr(x):
     return x.data_ptr()
 
 
-def _ptr_array(xs):
+def _ptr_array(xs, conv=None):
     if xs is None:
         return None
-    arr = (ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs])
+    arr = (ctypes.c_void_p * len(xs))(*[(conv or _ptr)(x) for x in xs])
     return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+
+
+def _host_ptr(x):
+    if x is None or isinstance(x, int):
+        return x
+    if x.is_cuda:
+        raise ValueError("lpar: host buffers must live in host memory")
+    if not x.is_contiguous():
+        raise ValueError("lpar: tensors must be contiguous")
+    return x.data_ptr()
 
 
 def _stream(stream):
@@ -200,6 +212,23 @@ def lpar_status_string(status):
     return _lib.lpar_status_string(status).decode()
 
 
+def lpar_host_staging_bytes(N, chunk, codec):
+    return _lib.lpar_host_staging_bytes(N, chunk, _codec(codec))
+
+
+def lpar_allreduce_host(host_inputs, n, codec, host_out, chunk, device, device_bytes, min_quant_bytes=0,
+                        schedule="auto", stream=None, N=None, stage_events=None):
+    """All-reduce of N messages in host memory (pinned for overlap), chunk by
+    chunk through `device` staging of lpar_host_staging_bytes bytes."""
+    ins = _ptr_array(host_inputs, _host_ptr)
+    outs = _ptr_array(host_out, _host_ptr)
+    N = len(host_inputs) if N is None else N
+    opts = _options(min_quant_bytes, schedule, stage_events)
+    _check(_lib.lpar_allreduce_host(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None, chunk,
+                                    _ptr(device), device_bytes, ctypes.byref(opts), _stream(stream)),
+           "lpar_allreduce_host")
+
+
 def lpar_collective_workspace_bytes(op, N, size, codec):
     return _lib.lpar_collective_workspace_bytes(OPS[op] if isinstance(op, str) else int(op), N, size, _codec(codec))
 
@@ -243,6 +272,28 @@ def allreduce(inputs, codec, out=None, workspace=None, min_quant_bytes=0, schedu
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=inputs[0].device)
     lpar_allreduce(inputs, n, codec, out, workspace, workspace.numel(), min_quant_bytes, schedule, stream)
+    return out
+
+
+HOST_CHUNK_ELEMS = 8 << 20          # 16 MiB of BF16 per rank per chunk
+
+
+def allreduce_host(host_inputs, codec, out=None, chunk=HOST_CHUNK_ELEMS, device_buffer=None, min_quant_bytes=0,
+                   schedule="auto", stream=None, device=None):
+    """All-reduce a list of N equal-size BF16 host tensors (pin them for overlap)
+    through the device in chunks; returns the N host outputs (pinned when
+    allocated here).  The result equals `allreduce` of the same values."""
+    import torch
+    n = host_inputs[0].numel()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in host_inputs]
+    c = max(2048, min(chunk, n))
+    need = lpar_host_staging_bytes(len(host_inputs), c, lpar_effective_codec(n, codec, min_quant_bytes))
+    if device_buffer is None:
+        device_buffer = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    lpar_allreduce_host(host_inputs, n, codec, out, c, device_buffer, device_buffer.numel(), min_quant_bytes,
+                        schedule, stream)
     return out
 
 

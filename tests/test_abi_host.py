@@ -202,6 +202,39 @@ def test_one_shot_schedule_is_accepted_and_validated(L):
     assert status_of(L.lpar_allreduce, [A, A], n, "int4", [A, A], A, ws, schedule=5, stream=st) == 4
 
 
+def test_host_staging_bytes(L):
+    c = 2048 * 8
+    assert L.lpar_host_staging_bytes(2, c, "int3") == 3 * 2 * 2 * c + L.lpar_workspace_bytes(2, c, "int3")
+    assert L.lpar_host_staging_bytes(8, c, "bf16") == 3 * 8 * 2 * c + L.lpar_workspace_bytes(8, c, "bf16")
+    assert L.lpar_host_staging_bytes(0, c, "int4") == 0
+    assert L.lpar_host_staging_bytes(9, c, "int4") == 0
+    assert L.lpar_host_staging_bytes(2, 0, "int4") == 0
+    assert L.lpar_host_staging_bytes(2, c + 4, "int4") == 0
+    assert L.lpar_host_staging_bytes(2, c, 11) == 0
+
+
+def test_argument_errors_allreduce_host(L):
+    # host "addresses" are never touched: every call fails in validation first
+    H = 0x10000
+    n, c = 2048 * 6, 2048 * 4
+    need = L.lpar_host_staging_bytes(2, c, "int4")
+    f = L.lpar_allreduce_host
+    assert status_of(f, [H, H], n, "int4", [H, H], c, A, need - 16, stream=0) == 3
+    assert status_of(f, [H, H], n, "int4", [H, H], c, M, need, stream=0) == 2
+    assert status_of(f, [H, H], n, "int4", [H, H], c, 0, need, stream=0) == 1
+    assert status_of(f, [H, 0], n, "int4", [H, H], c, A, need, stream=0) == 1
+    assert status_of(f, [H, H], n + 2, "int4", [H, H], c, A, need, stream=0) == 1
+    assert status_of(f, [H, H], n, "int4", [H, H], c + 2, A, need, stream=0) == 1
+    assert status_of(f, [H, H], n, "int4", [H, H], 0, A, need, stream=0) == 1
+    assert status_of(f, [H] * 9, n, "int4", [H] * 9, c, A, 10 ** 9, stream=0) == 1
+    assert status_of(f, [H, H], n, 12, [H, H], c, A, need, stream=0) == 4
+    assert status_of(f, [H, H], n, "int4", [H, H], c, A, need, schedule=5, stream=0) == 4
+    assert status_of(f, [H, H], 0, "int4", [H, H], c, A, 0, stream=0) == 0
+    # a chunk larger than the message is the message: staging for n suffices
+    small = L.lpar_host_staging_bytes(2, n, "int4")
+    assert status_of(f, [H, H], n, "int4", [H, H], 2048 * 64, A, small - 16, stream=0) == 3
+
+
 def test_status_strings(L):
     for s in range(6):
         assert L.lpar_status_string(s)
