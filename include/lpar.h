@@ -293,8 +293,9 @@ size_t lpar_host_staging_bytes(int N, size_t chunk, lpar_codec_t codec);
  * on `stream` runs after the last result has reached host memory; the call
  * returns once everything is enqueued.  Not for stream capture (the library
  * creates and releases its streams inside the call).  Argument errors are
- * returned before anything is enqueued; after LPAR_ERR_CUDA, work already
- * enqueued may still run. */
+ * returned before anything is enqueued; after an error returned once copies
+ * or kernels were enqueued, later work on `stream` still runs after them, so
+ * the buffers may be released once `stream` has passed the call. */
 lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
                                   void *const *host_out, size_t chunk, void *device, size_t device_bytes,
                                   const lpar_options_t *opts, cudaStream_t stream);

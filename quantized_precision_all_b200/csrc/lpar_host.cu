@@ -105,8 +105,8 @@ LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N
         if (cudaStreamWaitEvent(s, p.start, 0) != cudaSuccess) return LPAR_ERR_CUDA;
 
     const size_t chunks = (n + chunk - 1) / chunk;
-    int last = 0;
-    for (size_t k = 0; k < chunks; ++k) {
+    lpar_status_t status = LPAR_OK;
+    for (size_t k = 0; k < chunks && status == LPAR_OK; ++k) {
         const int s = (int)(k % kSlots);
         const size_t e0 = k * chunk, elems = (n - e0 < chunk) ? n - e0 : chunk;
         const void *in[LPAR_MAX_RANKS];
@@ -125,9 +125,9 @@ LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N
         ok = ok && cudaEventRecord(p.up[s], up) == cudaSuccess;
         // comp: the all-reduce of the chunk, in place
         ok = ok && cudaStreamWaitEvent(comp, p.up[s], 0) == cudaSuccess;
-        if (!ok) return LPAR_ERR_CUDA;
-        const lpar_status_t st = lpar_allreduce(in, N, elems, eff, out, ws, ws_bytes, &per_chunk, comp);
-        if (st != LPAR_OK) return st;
+        if (!ok) { status = LPAR_ERR_CUDA; break; }
+        status = lpar_allreduce(in, N, elems, eff, out, ws, ws_bytes, &per_chunk, comp);
+        if (status != LPAR_OK) break;
         ok = cudaEventRecord(p.comp[s], comp) == cudaSuccess;
         // down: the N result chunks back to the host
         ok = ok && cudaStreamWaitEvent(down, p.comp[s], 0) == cudaSuccess;
@@ -135,11 +135,17 @@ LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N
             ok = cudaMemcpyAsync(static_cast<uint8_t *>(host_out[r]) + 2 * e0, out[r], 2 * elems,
                                  cudaMemcpyDeviceToHost, down) == cudaSuccess;
         ok = ok && cudaEventRecord(p.down[s], down) == cudaSuccess;
-        if (!ok) return LPAR_ERR_CUDA;
-        last = s;
+        if (!ok) status = LPAR_ERR_CUDA;
     }
-    // later work on `stream` runs after the last download (the down stream is in order)
-    if (cudaStreamWaitEvent(stream, p.down[last], 0) != cudaSuccess) return LPAR_ERR_CUDA;
+    // Later work on `stream` runs after everything enqueued here, also after an
+    // error, so that the caller may release the staging and host buffers once
+    // `stream` has passed this point.
+    for (int i = 0; i < 3; ++i) {
+        cudaEvent_t done = i == 0 ? p.up[0] : (i == 1 ? p.comp[0] : p.down[0]);
+        if (cudaEventRecord(done, p.st[i]) != cudaSuccess || cudaStreamWaitEvent(stream, done, 0) != cudaSuccess)
+            status = LPAR_ERR_CUDA;
+    }
+    if (status != LPAR_OK) return status;
     if (opts && opts->stage_events[1]) cudaEventRecord(opts->stage_events[1], stream);
     return cudaGetLastError() == cudaSuccess ? LPAR_OK : LPAR_ERR_CUDA;
 }
