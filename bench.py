@@ -72,14 +72,32 @@ def measured_peaks():
 
 
 # ---- algorithmic bytes per launch (reads + writes the definition requires) ------
-def kernel_names(codec, schedule, N, f32=False):
+# The library's choice of the single-pass kernel form (lpar_kernels.cu,
+# launch_single_cn): warp-local for INT3 with N <= 2 or below 512 MiB of input
+# and for INT4 / MXFP4 below 128 MiB of input, CTA-wide otherwise and for FP8.
+BULK_MIN_BYTES = 128 << 20
+INT3_WARP_MAX_BYTES = 512 << 20
+
+
+def single_pass_kernel(codec, N, n):
+    in_bytes = N * 2 * n
+    if codec == "fp8":
+        warp = False
+    elif codec == "int3":
+        warp = N <= 2 or in_bytes < INT3_WARP_MAX_BYTES
+    else:
+        warp = in_bytes < BULK_MIN_BYTES
+    return ("k_allreduce_single_warp<%s,N=%d>" if warp else "k_allreduce_single<%s,N=%d>") % (codec, N)
+
+
+def kernel_names(codec, schedule, N, f32=False, n=None):
     if f32:
         return ["k_f32_reduce<N=%d>" % N] if codec == "bf16" else ["k_allreduce_single_f32<%s,N=%d>" % (codec, N)]
     if codec == "bf16":
         return ["k_bf16_reduce<N=%d,fused>" % N] if schedule != "three_stage" else \
             ["k_bf16_reduce<N=%d>" % N, "k_broadcast"]
     if schedule == "single_pass":
-        return ["k_allreduce_single<%s,N=%d>" % (codec, N)]
+        return [single_pass_kernel(codec, N, n) if n is not None else "k_allreduce_single<%s,N=%d>" % (codec, N)]
     if schedule == "fused":
         return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d,fused>" % (codec, N)]
     return ["k_quantize<%s>" % codec, "k_reduce<%s,N=%d>" % (codec, N), "k_decode<%s>" % codec]
@@ -257,7 +275,7 @@ def run_ours(args, rank, world, device):
     kern = {}
     for ci, codec in enumerate(w.codecs):
         eff = eff_codec(codec)
-        names = kernel_names(eff, args.schedule, N, f32)
+        names = kernel_names(eff, args.schedule, N, f32, n)
         if f32:
             bounds = [(0, 1)]
         elif eff == "bf16":

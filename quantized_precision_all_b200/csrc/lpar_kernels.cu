@@ -223,6 +223,68 @@ __global__ void __launch_bounds__(kThreads, ring_stages<C, N, BULK>() == 3 ? 4 :
     }
 }
 
+// K123, warp-local form (issue-bound cases: INT3 with few ranks, and the
+// smaller messages of INT4 and MXFP4).  Every warp works on its own half tile
+// of the chunk (blocks 32w .. 32w+31) and touches only its own 2 KiB of each
+// stage: its lanes copy them in, read them, stage the decoded blocks there and
+// store them to every output, so warps never wait for each other (__syncwarp
+// only).  A ring of three stages per warp: item i is staged in stage i % 3
+// while item i + 1 is prefetched, and refilled two items later, after the
+// warp's next __syncwarp.  The decoded chunk is staged in place of the last
+// rank's input.  Without CTA barriers the warps drift apart, which costs DRAM
+// efficiency when HBM is the bound: there the CTA-wide form is faster.
+template <int C, int N>
+__global__ void __launch_bounds__(kThreads, 4)
+    k_allreduce_single_warp(const __grid_constant__ InPtrs in, const __grid_constant__ OutPtrs wire, uint8_t *gather,
+                            const __grid_constant__ OutPtrs out, size_t tiles, unsigned chunks) {
+    constexpr int S = 3;
+    extern __shared__ __align__(1024) uint8_t ring[];
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    const int wt = w >> 1;                                 // the warp's tile within a chunk
+    unsigned c = blockIdx.x;
+    if (c >= chunks) return;
+    auto has = [&](unsigned cc) { return (size_t)cc * kTilesPerCta + wt < tiles; };
+    if (has(c)) warp_load(ring, in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2), w, lane);
+    cp_async_commit();
+    int buf = 0;
+    for (; c < chunks; c += gridDim.x) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const bool active = has(c);
+        const size_t tile = tile0 + wt;
+        const int b = t % kBlocksPerTile;
+        int last = buf;
+#pragma unroll 1
+        for (int r = 0; r < N; ++r) {
+            // prefetch the next item: rank r+1 of this chunk, or rank 0 of the next chunk
+            const int nb = buf + 1 == S ? 0 : buf + 1;
+            const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
+            if (cn < chunks && has(cn))
+                warp_load(ring + nb * kStageBytes,
+                          in.p[(r + 1 < N) ? r + 1 : 0] + (size_t)cn * kTilesPerCta * (kTileElems * 2), w, lane);
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncwarp();                                  // the warp's item landed
+            if (active) {
+                uint32_t x16[16];
+                stage_read(ring + buf * kStageBytes, t, x16);
+                float x[32];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) { x[2 * k] = bf16lo(x16[k]); x[2 * k + 1] = bf16hi(x16[k]); }
+                const float a = absmax_bf16x32(x16);
+                Packed<C> p;
+                encode<C, false, false>(x, a, p, NoSink{});
+                store_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
+            }
+            last = buf;
+            buf = nb;
+        }
+        uint8_t *const so = ring + last * kStageBytes;
+        if (active) reduce_block<C, N, true>(wire.p, tile, b, gather, StageSink{so, t});
+        __syncwarp();
+        if (active) warp_to_outputs(so, out, N, tile0 * (kTileElems * 2), w, lane);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // K3: gathered wire -> BF16 in every out[r].  grid = ceil(tiles / 4).
 // ---------------------------------------------------------------------------
@@ -367,11 +429,38 @@ static bool launch_single_cnb(const InPtrs &in, const OutPtrs &wire, uint8_t *g,
 }
 
 template <int C, int N>
+static bool launch_single_warp(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
+                               cudaStream_t st) {
+    constexpr int smem = 3 * kStageBytes;
+    if (!allow_dynamic_smem<k_allreduce_single_warp<C, N>>(smem)) return false;
+    const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    const unsigned res = resident_ctas<k_allreduce_single_warp<C, N>>(smem);
+    const unsigned grid = std::min<unsigned>(chunks, std::max<unsigned>(1u, res ? res : 148u * 4u));
+    k_allreduce_single_warp<C, N><<<grid, kThreads, smem, st>>>(in, wire, g, o, tiles, chunks);
+    return true;
+}
+
+// Which form of K123 runs (measured on B200, the forms timed alternately in one
+// process): the warp-local kernel for INT3 with one or two ranks at any size
+// (7-11% faster: its encode is issue-bound and the CTA barriers cost issue
+// slots) and for INT3 below kInt3WarpMaxBytes of input, and for INT4 and MXFP4
+// below kBulkMinBytes (up to 11% faster there); the CTA-wide kernel otherwise
+// (HBM-bound: 5-15% faster, with the bulk copies from kBulkMinBytes), and
+// always for FP8.
+constexpr size_t kInt3WarpMaxBytes = (size_t)512 << 20;
+
+template <int C, int N>
 static bool launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
                              cudaStream_t st) {
-    if ((size_t)N * tiles * (kTileElems * 2) >= kBulkMinBytes)
+    const size_t in_bytes = (size_t)N * tiles * (kTileElems * 2);
+    if constexpr (C == kFP8) {
+        if (in_bytes >= kBulkMinBytes) return launch_single_cnb<C, N, true>(in, wire, g, o, tiles, st);
+        return launch_single_cnb<C, N, false>(in, wire, g, o, tiles, st);
+    } else {
+        const bool warp = C == kINT3 ? (N <= 2 || in_bytes < kInt3WarpMaxBytes) : in_bytes < kBulkMinBytes;
+        if (warp) return launch_single_warp<C, N>(in, wire, g, o, tiles, st);
         return launch_single_cnb<C, N, true>(in, wire, g, o, tiles, st);
-    return launch_single_cnb<C, N, false>(in, wire, g, o, tiles, st);
+    }
 }
 
 template <int C>

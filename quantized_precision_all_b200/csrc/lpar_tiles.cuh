@@ -336,6 +336,35 @@ __device__ __forceinline__ void stage_load_chunk(uint8_t *stage, const uint8_t *
     }
 }
 
+// Warp-local staging.  Warp w of a CTA owns blocks 32w .. 32w + 31 of the
+// chunk (half of tile w / 2): bytes [2048w, 2048w + 2048) of a 16-KiB stage.
+// Its lanes copy exactly those bytes (lane l: 16-B pieces 128w + l + 32k,
+// k = 0..3, so every copy instruction of the warp covers 512 contiguous
+// bytes), read only them and send only them, so the warp needs no barrier
+// with the other warps: __syncwarp orders its lanes' accesses.
+constexpr int kWarpBytes = 2048;
+
+__device__ __forceinline__ void warp_load(uint8_t *stage, const uint8_t *chunk_src, int w, int lane) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int g = 128 * w + lane + 32 * k;
+        cp_async16(stage + swz(g >> 2, g & 3), chunk_src + 16 * (size_t)g);
+    }
+}
+
+// The warp's 2 KiB of a swizzled BF16 stage to every output at byte0.
+__device__ __forceinline__ void warp_to_outputs(const uint8_t *stage, const OutPtrs &out, int N, size_t byte0, int w,
+                                                int lane) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int g = 128 * w + lane + 32 * k;
+        const uint4 d = *reinterpret_cast<const uint4 *>(stage + swz(g >> 2, g & 3));
+#pragma unroll
+        for (int r = 0; r < kMaxRanks; ++r)
+            if (r < N) *reinterpret_cast<uint4 *>(out.p[r] + byte0 + 16 * (size_t)g) = d;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Host-side helpers.
 // ---------------------------------------------------------------------------

@@ -531,15 +531,16 @@ def test_workload_large_sampled_tiles(L, name):
 
 
 # ---------------------------------------------------------------------------
-# The single-pass kernel's bulk output path (messages of N x 2n >= 128 MiB) with
-# odd rank counts and a ragged last chunk (T % 4 == 3).  Student-t inputs drawn
-# on the GPU, with adversarial tiles planted at the sampled positions; sampled
-# tiles are compared bit for bit.
+# The single-pass kernel's CTA-wide form with bulk output copies (from 128 MiB
+# of input, N x 2n; INT3 from 512 MiB and N >= 3) with odd rank counts and a
+# ragged last chunk (T % 4 == 3); INT3 with N = 1 runs the warp-local form at
+# every size.  Student-t inputs drawn on the GPU, with adversarial tiles
+# planted at the sampled positions; sampled tiles are compared bit for bit.
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4"])
 @pytest.mark.parametrize("N", [1, 3, 5])
 def test_bulk_output_path_ragged_tail(L, codec, N):
-    T = -(-(128 << 20) // (N * 4096))
+    T = -(-((512 if codec == "int3" else 128) << 20) // (N * 4096))
     T += (3 - T % 4) % 4                             # T % 4 == 3: the last chunk holds three tiles
     assert N * T * 4096 >= (128 << 20) and T % 4 == 3
     n = T * 2048
