@@ -127,6 +127,76 @@ __global__ void __launch_bounds__(kThreads, 4) k_reduce_bf16_single(const __grid
     }
 }
 
+// The warp-local form of the reductions (see k_allreduce_single_warp): every
+// warp copies, encodes, reduces and stores only its own half tile of the
+// chunk, so no CTA barrier is needed; a ring of three stages per warp, the
+// BF16 sums staged in place of the last rank's input.
+template <int C, int N, bool ALL>
+__global__ void __launch_bounds__(kThreads, 4) k_reduce_bf16_warp(const __grid_constant__ InPtrs in,
+                                                                  const __grid_constant__ OutPtrs wire,
+                                                                  const __grid_constant__ OutPtrs out,
+                                                                  size_t tiles, unsigned chunks) {
+    constexpr int S = 3;
+    extern __shared__ __align__(1024) uint8_t ring[];
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    const int wt = w >> 1;                                 // the warp's tile within a chunk
+    unsigned c = blockIdx.x;
+    if (c >= chunks) return;
+    auto has = [&](unsigned cc) { return (size_t)cc * kTilesPerCta + wt < tiles; };
+    if (has(c)) warp_load(ring, in.p[0] + (size_t)c * kTilesPerCta * (kTileElems * 2), w, lane);
+    cp_async_commit();
+    int buf = 0;
+    for (; c < chunks; c += gridDim.x) {
+        const size_t tile0 = (size_t)c * kTilesPerCta;
+        const bool active = has(c);
+        const size_t tile = tile0 + wt;
+        const int b = t % kBlocksPerTile;
+        int last = buf;
+#pragma unroll 1
+        for (int r = 0; r < N; ++r) {
+            const int nb = buf + 1 == S ? 0 : buf + 1;
+            const unsigned cn = (r + 1 < N) ? c : c + gridDim.x;
+            if (cn < chunks && has(cn))
+                warp_load(ring + nb * kStageBytes,
+                          in.p[(r + 1 < N) ? r + 1 : 0] + (size_t)cn * kTilesPerCta * (kTileElems * 2), w, lane);
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncwarp();                                  // the warp's item landed
+            if (active)
+                quantize_staged_block<C, false>(ring + buf * kStageBytes, wire.p[r] + tile * Layout<C>::kTileBytes,
+                                                t, NoSink{});
+            last = buf;
+            buf = nb;
+        }
+        uint8_t *const so = ring + last * kStageBytes;
+        if (active) {
+            float acc[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = 0.0f;    // +0.0f, then ranks in ascending order
+#pragma unroll
+            for (int r = 0; r < N; ++r) {
+                Packed<C> p;
+                load_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
+                accumulate<C>(p, acc);
+            }
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = pack_bf16x2(acc[2 * k], acc[2 * k + 1]);
+            stage_write(so, t, o);
+        }
+        __syncwarp();
+        if (active) {
+            if (ALL) {
+                warp_to_outputs(so, out, N, tile0 * (kTileElems * 2), w, lane);
+            } else {
+                const int j = shard_of(tile, tiles, N);
+                warp_to_dst(so, out.p[j] + (tile - shard_begin(j, tiles, N)) * (kTileElems * 2) + (w & 1) * kWarpBytes,
+                            w, lane);
+            }
+        }
+    }
+}
+
 // BF16 passthrough of the reductions: one tile (256 x 16 B) per CTA step, the
 // FP32 sum in rank order rounded once.  The shard owner advances with the
 // tile index (tiles are visited in increasing order), so no division per tile.
@@ -286,9 +356,29 @@ static inline unsigned persistent_grid(unsigned chunks, unsigned resident) {
     return std::min<unsigned>(chunks, std::max<unsigned>(1u, resident ? resident : 148u * 4u));
 }
 
+// Which form of the reductions runs (measured on B200, the forms timed
+// alternately in one process): the warp-local form below 128 MiB of input for
+// every codec but FP8 (5-10% faster) and, for the reduce-scatter, for INT3 at
+// every size (6-9%) and for INT4 and MXFP4 from four ranks on (8% at N = 8);
+// the CTA-wide form for FP8, for the one-shot from 128 MiB (4-9%) and for the
+// reduce-scatter of INT4 and MXFP4 with fewer ranks (3-9%).
+static inline bool rs_warp_form(int C, int N, bool ALL, size_t in_bytes) {
+    if (C == kFP8) return false;
+    if (in_bytes < ((size_t)128 << 20)) return true;
+    if (ALL) return false;
+    return C == kINT3 || N >= 4;
+}
+
 template <int C, int N, bool ALL>
 static void launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+    if (rs_warp_form(C, N, ALL, (size_t)N * tiles * (kTileElems * 2))) {
+        constexpr int smem = 3 * kStageBytes;
+        if (!allow_dynamic_smem<k_reduce_bf16_warp<C, N, ALL>>(smem)) return;   // reported by launch_status
+        const unsigned grid = persistent_grid(chunks, resident_ctas<k_reduce_bf16_warp<C, N, ALL>>(smem));
+        k_reduce_bf16_warp<C, N, ALL><<<grid, kThreads, smem, st>>>(in, wire, out, tiles, chunks);
+        return;
+    }
     const unsigned grid = persistent_grid(chunks, resident_ctas<k_reduce_bf16_single<C, N, ALL>>());
     k_reduce_bf16_single<C, N, ALL><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, chunks);
 }

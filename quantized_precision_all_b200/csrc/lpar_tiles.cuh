@@ -365,6 +365,16 @@ __device__ __forceinline__ void warp_to_outputs(const uint8_t *stage, const OutP
     }
 }
 
+// The warp's 2 KiB of a swizzled BF16 stage to one destination (the warp's
+// half tile there).
+__device__ __forceinline__ void warp_to_dst(const uint8_t *stage, uint8_t *dst, int w, int lane) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int q = lane + 32 * k, g = 128 * w + q;
+        *reinterpret_cast<uint4 *>(dst + 16 * (size_t)q) = *reinterpret_cast<const uint4 *>(stage + swz(g >> 2, g & 3));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Host-side helpers.
 // ---------------------------------------------------------------------------
