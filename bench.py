@@ -295,7 +295,7 @@ def run_ours(args, rank, world, device):
         d["achieved_gbs"] = d["algorithmic_bytes"] / (d["ms_per_launch"] * 1e-3) / 1e9
     launches_per_step = sum(len(kernel_names(eff_codec(c), args.schedule, N, f32)) for c in w.codecs)
 
-    # (3) parity and accuracy of this step's outputs on sampled tiles (outside the timed region)
+    # (3) accuracy of this step's outputs on sampled tiles (outside the timed region)
     accuracy = {}
     if not f32:
         T = n // TILE
@@ -304,7 +304,7 @@ def run_ours(args, rank, world, device):
         for codec in w.codecs:
             allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
             torch.cuda.synchronize(device)
-            accuracy[codec] = sample_check(xs, outs, codec, sample.numpy(), w.min_quant_bytes)
+            accuracy[codec] = sample_check(xs, outs, sample.numpy())
 
     # (4) end to end through the public API with host buffers
     e2e = None
@@ -433,24 +433,20 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def sample_check(xs, outs, codec, tiles, min_quant_bytes=0):
-    """Bit-exact comparison of sampled output tiles with the oracle, the error
-    of those tiles against the exact (binary64) sum of the inputs, and a hash of
-    the sampled input bytes.  Tiles are independent, so a sample is exact."""
-    from oracle import oracle as O
+def sample_check(xs, outs, tiles):
+    """The error of sampled output tiles against the exact (binary64) sum of the
+    inputs, and a hash of the sampled input bytes.  Bit-exact parity with the
+    oracle on the same points is the business of tests/test_gpu_parity.py
+    (test_workload_large_sampled_tiles, test_sweep_sampled_tiles)."""
     idx = torch.from_numpy((tiles[:, None] * TILE + torch.arange(TILE).numpy()[None, :]).reshape(-1)).to(xs[0].device)
-    ins = [x[idx].view(torch.int16).cpu().numpy().view("uint16") for x in xs]
-    got = [o[idx].view(torch.int16).cpu().numpy().view("uint16") for o in outs]
-    ref, _ = O.allreduce(ins, codec, min_quant_bytes)
-    parity = all((g == ref[0]).all() for g in got)
-    exact = sum(O.bf16_bits_to_f32(x).astype("float64") for x in ins)
-    err = O.bf16_bits_to_f32(got[0]).astype("float64") - exact
+    ins = [x[idx].float().cpu().numpy().astype("float64") for x in xs]     # BF16 -> binary64 is exact
+    got = outs[0][idx].float().cpu().numpy().astype("float64")
+    err = got - sum(ins)
     h = hashlib.blake2b(digest_size=8)
-    for x in ins:
-        h.update(x.tobytes())
-    return {"parity_bit_exact": bool(parity), "sampled_tiles": int(len(tiles)),
-            "max_abs_err_vs_exact": float(abs(err).max()), "rms_err_vs_exact": float((err ** 2).mean() ** 0.5),
-            "input_sample_blake2b": h.hexdigest()}
+    for x in xs:
+        h.update(x[idx].view(torch.int16).cpu().numpy().tobytes())
+    return {"sampled_tiles": int(len(tiles)), "max_abs_err_vs_exact": float(abs(err).max()),
+            "rms_err_vs_exact": float((err ** 2).mean() ** 0.5), "input_sample_blake2b": h.hexdigest()}
 
 
 def oracle_gbs(op, N, codec, tiles=64):
@@ -521,7 +517,7 @@ def run_sweep(args, device):
                                   "l2": "256 MiB buffer rewritten before every timed call",
                                   "note": "L2-resident / launch-bound" if N * mb < (16 << 20) else "",
                                   "peak": peak, "cpu_baseline": cpu[(N, codec)], "seed": w.seed,
-                                  **sample_check(xs, outs, codec, sample.numpy())})
+                                  **sample_check(xs, outs, sample.numpy())})
                 print(row, flush=True)
                 if sink:
                     sink.write(row + "\n")
