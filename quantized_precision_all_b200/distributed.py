@@ -11,9 +11,12 @@ links, compute stays in FP32):
      [jT/N, (j+1)T/N), the same floor partition as the emulation) of every
      rank's wire, in rank order;
   3. rank j reduces its shard from the N received wires and requantises it
-     (``lpar_reduce``: FP32 sum in ascending rank order from +0.0f);
-  4. all-gather of the requantised shards;
-  5. every rank decodes the gathered wire (``lpar_decode``).
+     (``lpar_reduce``: FP32 sum in ascending rank order from +0.0f), straight
+     into its slot of the all-gather buffer;
+  4. all-gather of the requantised shards into one buffer (slots padded to the
+     largest shard);
+  5. every rank decodes each shard from its slot into its place of the output
+     (``lpar_decode``): no concatenation or other copy of the gathered wire.
 
 The result is bit-identical to ``lpar_allreduce`` on the N messages in one GPU.
 The exchanges use ``torch.distributed`` collectives on the wire bytes (NCCL on
@@ -33,8 +36,9 @@ TILE_ELEMS = L.TILE_ELEMS
 
 @dataclass
 class Stages:
-    """quantize(x, codec) -> wire; reduce(wires, tiles, codec) -> reduced wire of
-    `tiles` tiles; decode(wire, n, codec) -> n BF16 values; tile_bytes(codec)."""
+    """quantize(x, codec) -> wire; reduce(wires, tiles, codec, out) writes the
+    reduced wire of `tiles` tiles into `out`; decode(wire, n, codec, out) writes
+    n BF16 values into `out`; tile_bytes(codec)."""
     quantize: Callable
     reduce: Callable
     decode: Callable
@@ -48,16 +52,12 @@ def cuda_stages(stream: Optional[torch.cuda.Stream] = None) -> Stages:
         L.lpar_quantize(x, x.numel(), codec, wire, stream)
         return wire
 
-    def reduce(wires, tiles, codec):
-        out = torch.empty(tiles * L.lpar_tile_bytes(codec), dtype=torch.uint8, device=wires[0].device)
+    def reduce(wires, tiles, codec, out):
         if tiles:
             L.lpar_reduce(list(wires), 0, tiles, codec, out, stream)
-        return out
 
-    def decode(wire, n, codec):
-        out = torch.empty(n, dtype=torch.bfloat16, device=wire.device)
+    def decode(wire, n, codec, out):
         L.lpar_decode(wire, n, codec, out, stream)
-        return out
 
     return Stages(quantize, reduce, decode, L.lpar_tile_bytes)
 
@@ -76,7 +76,8 @@ class DistributedAllreduce:
         self.rank = dist.get_rank(group)
         self.stages = stages if stages is not None else cuda_stages()
 
-    def allreduce(self, x: torch.Tensor, codec: str, min_quant_bytes: int = 0) -> torch.Tensor:
+    def allreduce(self, x: torch.Tensor, codec: str, min_quant_bytes: int = 0,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
         n = x.numel()
         if n % TILE_ELEMS:
             raise ValueError("the message must be a whole number of 2048-element tiles")
@@ -94,12 +95,19 @@ class DistributedAllreduce:
         dist.all_to_all_single(recv, wire, output_split_sizes=[my_tiles * tb] * N,
                                input_split_sizes=send_sizes, group=self.group)
         received = [recv[r * my_tiles * tb:(r + 1) * my_tiles * tb] for r in range(N)]
-        shard = st.reduce(received, my_tiles, codec)        # 3. stage 2 of my shard
-        # 4. all-gather of the shards (padded to the largest shard)
+        # 3. stage 2 of my shard, straight into my slot of the all-gather (padded
+        #    to the largest shard; the padding is never decoded)
         width = max(t1 - t0 for t0, t1 in shards) * tb
-        padded = torch.zeros(width, dtype=torch.uint8, device=wire.device)
-        padded[:shard.numel()] = shard
-        gathered = [torch.empty(width, dtype=torch.uint8, device=wire.device) for _ in range(N)]
-        dist.all_gather(gathered, padded, group=self.group)
-        full = torch.cat([g[:(t1 - t0) * tb] for g, (t0, t1) in zip(gathered, shards)])
-        return st.decode(full, n, codec)                    # 5. stage 3
+        send = torch.empty(width, dtype=torch.uint8, device=wire.device)
+        st.reduce(received, my_tiles, codec, send[:my_tiles * tb])
+        # 4. all-gather of the shards into one buffer, rank j's slot at j * width
+        gathered = torch.empty(N * width, dtype=torch.uint8, device=wire.device)
+        dist.all_gather(list(gathered.view(N, width).unbind(0)), send, group=self.group)
+        # 5. stage 3: each shard decoded from its slot into its place of the output
+        if out is None:
+            out = torch.empty(n, dtype=torch.bfloat16, device=x.device)
+        for j, (t0, t1) in enumerate(shards):
+            if t1 > t0:
+                st.decode(gathered[j * width:j * width + (t1 - t0) * tb], (t1 - t0) * TILE_ELEMS, codec,
+                          out[t0 * TILE_ELEMS:t1 * TILE_ELEMS])
+        return out

@@ -1,7 +1,8 @@
 """The cross-process all-reduce (quantized_precision_all_b200.distributed) on CPU
 with gloo, world sizes 2 to 4: the host orchestration (shard partition, the
 all-to-all split sizes, rank order of the received wires, the padded
-all-gather) runs with the oracle's stage functions, and every rank's result
+all-gather into one buffer and the per-shard decode) runs with the oracle's
+stage functions, and every rank's result
 must equal the oracle's all-reduce of all ranks' messages bit for bit."""
 import os
 import socket
@@ -24,13 +25,13 @@ def oracle_stages():
     def quantize(x, codec):
         return torch.from_numpy(O.quantize(bits(x), codec).copy())
 
-    def reduce(wires, tiles, codec):
-        if tiles == 0:
-            return torch.empty(0, dtype=torch.uint8)
-        return torch.from_numpy(O.reduce([w.numpy() for w in wires], 0, tiles, codec)[:tiles * O.tile_bytes(codec)].copy())
+    def reduce(wires, tiles, codec, out):
+        if tiles:
+            red = O.reduce([w.numpy() for w in wires], 0, tiles, codec)[:tiles * O.tile_bytes(codec)]
+            out.copy_(torch.from_numpy(red.copy()))
 
-    def decode(wire, n, codec):
-        return torch.from_numpy(O.decode(wire.numpy(), n, codec).view(np.int16).copy()).view(torch.bfloat16)
+    def decode(wire, n, codec, out):
+        out.copy_(torch.from_numpy(O.decode(wire.numpy(), n, codec).view(np.int16).copy()).view(torch.bfloat16))
 
     return Stages(quantize, reduce, decode, O.tile_bytes)
 
