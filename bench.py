@@ -42,7 +42,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 REF_TILES_PER_STEP = 256            # reference arm: 0.5 Mi elements per rank per core per step
 CPU_BASELINE_TILES = 16384          # cpu_baseline: 32 Mi elements (64 MiB) per rank
 PAR_TILES_PER_CORE = 2048           # cpu_baseline on every core: 4 Mi elements per rank per core
-HOST_CHUNK_ELEMS = 8 << 20          # e2e: 16 MiB of BF16 per rank per chunk of the host all-reduce
+HOST_CHUNK_BYTES = 32 << 20         # e2e: bytes of one chunk of the host all-reduce, all ranks together
 
 
 def log(*a):
@@ -315,31 +315,23 @@ def run_ours(args, rank, world, device):
             h.copy_(x)
         h_out = [torch.empty(n, dtype=xs[0].dtype, pin_memory=True) for _ in range(N)]
 
+        # the host all-reduce: chunks uploaded, reduced and downloaded on three
+        # streams of the library, overlapped; one call per codec
+        chunk = min(n, max(TILE, HOST_CHUNK_BYTES // (N * w.elem_bytes) // TILE * TILE))
         if f32:
-            # binary32 messages: the copies and the call in order on one stream
-            def e2e_step():
-                for x, h in zip(xs, h_in):
-                    x.copy_(h, non_blocking=True)
-                for codec in w.codecs:
-                    allreduce(xs, n, codec, outs, ws, ws_bytes, w.min_quant_bytes, args.schedule, stream)
-                    for h, o in zip(h_out, outs):
-                        h.copy_(o, non_blocking=True)
-            h2d = N * w.elem_bytes * n
-            api = "lpar_allreduce_f32 with pinned host buffers copied in and out on the same stream"
+            host_call, staging_bytes = L.lpar_allreduce_f32_host, L.lpar_host_staging_bytes_f32
         else:
-            # the host all-reduce: chunks uploaded, reduced and downloaded on
-            # three streams of the library, overlapped; one call per codec
-            chunk = min(n, HOST_CHUNK_ELEMS)
-            staging = torch.empty(max(L.lpar_host_staging_bytes(N, chunk, eff_codec(c)) for c in w.codecs),
-                                  dtype=torch.uint8, device=device)
+            host_call, staging_bytes = L.lpar_allreduce_host, L.lpar_host_staging_bytes
+        staging = torch.empty(max(staging_bytes(N, chunk, eff_codec(c)) for c in w.codecs), dtype=torch.uint8,
+                              device=device)
 
-            def e2e_step():
-                for codec in w.codecs:
-                    L.lpar_allreduce_host(h_in, n, codec, h_out, chunk, staging, staging.numel(), w.min_quant_bytes,
-                                          args.schedule, stream)
-            h2d = N * w.elem_bytes * n * len(w.codecs)
-            api = ("lpar_allreduce_host with pinned host buffers: chunks of %d elements per rank uploaded, "
-                   "reduced and downloaded on three streams, overlapped; one call per codec" % chunk)
+        def e2e_step():
+            for codec in w.codecs:
+                host_call(h_in, n, codec, h_out, chunk, staging, staging.numel(), w.min_quant_bytes, args.schedule,
+                          stream)
+        h2d = N * w.elem_bytes * n * len(w.codecs)
+        api = ("%s with pinned host buffers: chunks of %d elements per rank uploaded, reduced and downloaded on "
+               "three streams, overlapped; one call per codec" % (host_call.__name__, chunk))
 
         e2e_step()
         torch.cuda.synchronize(device)

@@ -300,6 +300,16 @@ lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N, size_t 
                                   void *const *host_out, size_t chunk, void *device, size_t device_bytes,
                                   const lpar_options_t *opts, cudaStream_t stream);
 
+/* The same for binary32 messages: lpar_allreduce_f32 chunk by chunk.  Staging:
+ * lpar_host_staging_bytes_f32(N, min(chunk, n), effective codec), the
+ * threshold deciding on the binary32 message (4n bytes) as in
+ * lpar_allreduce_f32; schedules LPAR_SCHEDULE_AUTO and
+ * LPAR_SCHEDULE_SINGLE_PASS; otherwise as lpar_allreduce_host. */
+size_t lpar_host_staging_bytes_f32(int N, size_t chunk, lpar_codec_t codec);
+lpar_status_t lpar_allreduce_f32_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
+                                      void *const *host_out, size_t chunk, void *device, size_t device_bytes,
+                                      const lpar_options_t *opts, cudaStream_t stream);
+
 /* The codec lpar_allreduce runs for these arguments after the threshold. */
 lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts);
 

@@ -33,7 +33,8 @@ MAX_RANKS = 8
 EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_quantize", "lpar_reduce",
            "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string",
            "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all",
-           "lpar_allreduce_f32", "lpar_host_staging_bytes", "lpar_allreduce_host")
+           "lpar_allreduce_f32", "lpar_host_staging_bytes", "lpar_allreduce_host", "lpar_host_staging_bytes_f32",
+           "lpar_allreduce_f32_host")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -70,6 +71,8 @@ def _load():
         "lpar_allreduce_f32": (i32, [vpp, i32, sz, i32, vpp, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_host_staging_bytes": (sz, [i32, sz, i32]),
         "lpar_allreduce_host": (i32, [vpp, i32, sz, i32, vpp, sz, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_host_staging_bytes_f32": (sz, [i32, sz, i32]),
+        "lpar_allreduce_f32_host": (i32, [vpp, i32, sz, i32, vpp, sz, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -214,6 +217,23 @@ def lpar_status_string(status):
 
 def lpar_host_staging_bytes(N, chunk, codec):
     return _lib.lpar_host_staging_bytes(N, chunk, _codec(codec))
+
+
+def lpar_host_staging_bytes_f32(N, chunk, codec):
+    return _lib.lpar_host_staging_bytes_f32(N, chunk, _codec(codec))
+
+
+def lpar_allreduce_f32_host(host_inputs, n, codec, host_out, chunk, device, device_bytes, min_quant_bytes=0,
+                            schedule="auto", stream=None, N=None, stage_events=None):
+    """All-reduce of N binary32 messages in host memory, chunk by chunk through
+    `device` staging of lpar_host_staging_bytes_f32 bytes."""
+    ins = _ptr_array(host_inputs, _host_ptr)
+    outs = _ptr_array(host_out, _host_ptr)
+    N = len(host_inputs) if N is None else N
+    opts = _options(min_quant_bytes, schedule, stage_events)
+    _check(_lib.lpar_allreduce_f32_host(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+                                        chunk, _ptr(device), device_bytes, ctypes.byref(opts), _stream(stream)),
+           "lpar_allreduce_f32_host")
 
 
 def lpar_allreduce_host(host_inputs, n, codec, host_out, chunk, device, device_bytes, min_quant_bytes=0,

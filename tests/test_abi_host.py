@@ -235,6 +235,29 @@ def test_argument_errors_allreduce_host(L):
     assert status_of(f, [H, H], n, "int4", [H, H], 2048 * 64, A, small - 16, stream=0) == 3
 
 
+def test_host_staging_bytes_f32(L):
+    c = 2048 * 8
+    assert L.lpar_host_staging_bytes_f32(8, c, "fp8") == 3 * 8 * 4 * c + \
+        L.lpar_collective_workspace_bytes("allreduce_f32", 8, c, "fp8")
+    assert L.lpar_host_staging_bytes_f32(2, c, "bf16") == 3 * 2 * 4 * c + 4 * c
+    assert L.lpar_host_staging_bytes_f32(0, c, "fp8") == 0
+    assert L.lpar_host_staging_bytes_f32(2, c + 2, "fp8") == 0
+
+
+def test_argument_errors_allreduce_f32_host(L):
+    H = 0x10000
+    n, c = 2048 * 6, 2048 * 4
+    need = L.lpar_host_staging_bytes_f32(2, c, "fp8")
+    f = L.lpar_allreduce_f32_host
+    assert status_of(f, [H, H], n, "fp8", [H, H], c, A, need - 16, stream=0) == 3
+    assert status_of(f, [H, H], n, "fp8", [H, H], c, M, need, stream=0) == 2
+    assert status_of(f, [H, 0], n, "fp8", [H, H], c, A, need, stream=0) == 1
+    assert status_of(f, [H, H], n + 2, "fp8", [H, H], c, A, need, stream=0) == 1
+    assert status_of(f, [H, H], n, 12, [H, H], c, A, need, stream=0) == 4
+    assert status_of(f, [H, H], n, "fp8", [H, H], c, A, need, schedule="fused", stream=0) == 4
+    assert status_of(f, [H, H], 0, "fp8", [H, H], c, A, 0, stream=0) == 0
+
+
 def test_status_strings(L):
     for s in range(6):
         assert L.lpar_status_string(s)

@@ -116,3 +116,39 @@ def test_helper_and_stream_order(L):
     for o in outs:
         assert o.is_pinned()
         assert np.array_equal(o.view(torch.int16).numpy().view(np.uint16), ref[0])
+
+
+# ---- binary32 messages: lpar_allreduce_f32_host ------------------------------------
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("N,tiles,chunk_tiles", [(2, 7, 2), (8, 5, 3)])
+def test_f32_host_matches_oracle(L, codec, N, tiles, chunk_tiles):
+    from tests.test_gpu_f32 import adversarial_f32
+    n = tiles * 2048
+    xs = [adversarial_f32(n, 3800 + 10 * N + r) for r in range(N)]
+    hin = [torch.from_numpy(x.copy()).pin_memory() for x in xs]
+    hout = [torch.zeros(n, dtype=torch.float32).pin_memory() for _ in range(N)]
+    eff = L.lpar_effective_codec(2 * n, codec, 0)
+    c = chunk_tiles * 2048
+    dev = torch.empty(L.lpar_host_staging_bytes_f32(N, c, eff), dtype=torch.uint8, device="cuda")
+    L.lpar_allreduce_f32_host(hin, n, codec, hout, c, dev, dev.numel())
+    torch.cuda.current_stream().synchronize()
+    ref, used = O.allreduce_f32(xs, codec)
+    assert used == codec
+    for o in hout:
+        assert np.array_equal(o.numpy().view(np.uint32), ref[0].view(np.uint32)), (codec, N)
+
+
+def test_f32_host_threshold_on_the_whole_message(L):
+    from tests.test_gpu_f32 import adversarial_f32
+    n = 2048 * 6
+    xs = [adversarial_f32(n, 3900 + r) for r in range(2)]
+    hin = [torch.from_numpy(x.copy()).pin_memory() for x in xs]
+    hout = [torch.zeros(n, dtype=torch.float32).pin_memory() for _ in range(2)]
+    thr = 4 * n                                       # the whole binary32 message qualifies, a chunk would not
+    dev = torch.empty(L.lpar_host_staging_bytes_f32(2, 2048 * 2, "fp8"), dtype=torch.uint8, device="cuda")
+    L.lpar_allreduce_f32_host(hin, n, "fp8", hout, 2048 * 2, dev, dev.numel(), min_quant_bytes=thr)
+    torch.cuda.current_stream().synchronize()
+    ref, used = O.allreduce_f32(xs, "fp8", thr)
+    assert used == "fp8"
+    assert np.array_equal(hout[0].numpy().view(np.uint32), ref[0].view(np.uint32))
+
