@@ -426,7 +426,15 @@ static bool launch_gather_c(const InPtrs &in, const OutPtrs &wire, const OutPtrs
     constexpr int smem = gather_smem<C, A2A>();
     if (!allow_dynamic_smem<k_gather_single<C, A2A>>(smem)) return false;
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
-    const unsigned grid = persistent_grid(chunks, resident_ctas<k_gather_single<C, A2A>>(smem));
+    unsigned grid = persistent_grid(chunks, resident_ctas<k_gather_single<C, A2A>>(smem));
+    // The all-gather writes N outputs per item: from 64 MiB of input, fewer
+    // CTAs (fewer concurrent output streams) write faster -- two per SM up to
+    // three ranks, one from four (measured on B200, 4-8% at 64-256 MiB); with
+    // eight ranks the counts measured alike (within 2%) and all CTAs stay.
+    if (!A2A && N < 8 && (size_t)N * tiles * (kTileElems * 2) >= ((size_t)64 << 20)) {
+        const unsigned sms = sm_count();
+        if (sms) grid = std::min<unsigned>(grid, sms * (N <= 3 ? 2u : 1u));
+    }
     k_gather_single<C, A2A><<<grid, kThreads, smem, st>>>(in, wire, out, tiles, seg_tiles, chunks, N);
     return true;
 }

@@ -397,6 +397,19 @@ static unsigned resident_ctas(int smem = 0) {
     return v;
 }
 
+// SM count of the current device, cached per device; 0 when the query fails.
+static inline unsigned sm_count() {
+    static std::atomic<unsigned> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    unsigned v = cache[dev].load(std::memory_order_relaxed);
+    if (v) return v;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 0;
+    cache[dev].store((unsigned)sms, std::memory_order_relaxed);
+    return (unsigned)sms;
+}
+
 // The opt-in to more than 48 KiB of dynamic shared memory, made once per
 // device and per kernel; false when it fails.
 template <auto Kernel>
