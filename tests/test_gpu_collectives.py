@@ -202,6 +202,36 @@ def test_large_sampled_tiles(L, op):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("N", [3, 5])
+def test_all_gather_reduced_grid_ragged(L, N):
+    """The all-gather from 64 MiB of input runs on fewer CTAs (2 per SM for
+    N <= 3, 1 for N = 4..7); here with a ragged last chunk (tiles % 4 == 3),
+    sampled tiles against the oracle's round trip at every destination."""
+    mt = -(-(64 << 20) // (N * 4096))
+    mt += (3 - mt % 4) % 4
+    m = mt * 2048
+    assert N * m * 2 >= (64 << 20) and mt % 4 == 3
+    w = W.Workload("capped_all_gather", N=N, n=m, dist="student_t", nu=3, seed=11, codecs=("int4",))
+    xs = W.make_inputs(w, "cuda")
+    rng = np.random.default_rng(12)
+    stiles = np.unique(np.concatenate([np.arange(mt - 5, mt), rng.choice(mt, 64, replace=False)]))
+    idx = torch.from_numpy((stiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
+    for codec in ("int4", "fp8"):
+        outs = [torch.empty(N * m, dtype=torch.bfloat16, device="cuda") for _ in range(N)]
+        ws = torch.empty(L.lpar_collective_workspace_bytes("all_gather", N, m, codec), dtype=torch.uint8,
+                         device="cuda")
+        L.lpar_all_gather(xs, m, codec, outs, ws, ws.numel())
+        torch.cuda.synchronize()
+        for r in range(N):
+            sample = xs[r][idx].view(torch.int16).cpu().numpy().view(np.uint16)
+            trip = O.decode(O.quantize(sample, codec), sample.size, codec)
+            for j in range(N):
+                got = outs[j][r * m:(r + 1) * m][idx].view(torch.int16).cpu().numpy().view(np.uint16)
+                assert np.array_equal(got, trip), (codec, N, r, j)
+        del outs, ws
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------------------
 # The cross-process all-reduce on the GPU: the library's stages with NCCL
 # collectives.  Only one GPU is available, so this runs one process (the
