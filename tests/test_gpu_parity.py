@@ -434,6 +434,34 @@ def test_allreduce_matches_oracle(L, codec, N, schedule):
         assert np.array_equal(host[N * wb:(N + 1) * wb], O.reduce(wires, 0, tiles, codec))
 
 
+# Seeded random cases over the whole argument space: codec, N in 1..8, 1..40
+# tiles, every schedule (one-shot against its own oracle), a threshold either
+# side of the message, in place or not; adversarial or random inputs per rank.
+N_RANDOM_CASES = 48
+
+
+@pytest.mark.parametrize("case", range(N_RANDOM_CASES))
+def test_allreduce_random_cases(L, case):
+    rng = np.random.default_rng(9000 + case)
+    codec = CODECS[rng.integers(len(CODECS))]
+    N = int(rng.integers(1, 9))
+    tiles = int(rng.integers(1, 41))
+    n = tiles * 2048
+    schedule = ["auto", "fused", "three_stage", "single_pass", "one_shot"][rng.integers(5)]
+    thr = [0, 2 * n, 2 * n + 2][rng.integers(3)]
+    inplace = bool(rng.integers(2))
+    xs = [adversarial_bf16(n, int(rng.integers(1 << 30))) if rng.integers(2)
+          else random_bf16(n, int(rng.integers(1 << 30)), float(2.0 ** rng.integers(-8, 9))) for _ in range(N)]
+    outs, _ = run_allreduce(L, xs, codec, schedule, thr, inplace)
+    if schedule == "one_shot":
+        ref, used = O.allreduce_oneshot(xs, codec, thr)
+    else:
+        ref, used = O.allreduce(xs, codec, thr)
+    assert used == L.lpar_effective_codec(n, codec, thr)
+    for o in outs:
+        assert np.array_equal(o, ref[0]), (codec, N, tiles, schedule, thr, inplace)
+
+
 @pytest.mark.parametrize("codec", CODECS)
 def test_allreduce_in_place(L, codec):
     n = 2048 * 6
