@@ -49,6 +49,34 @@ def run(L, op, xs, size, codec, out_sizes, min_quant_bytes=0):
     return [host_u16(g) for g in outs], eff
 
 
+# Seeded random cases: operation, codec, N in 1..8, 1..24 tiles, a threshold
+# either side of the message; adversarial and random inputs.
+@pytest.mark.parametrize("case", range(36))
+def test_collectives_random_cases(L, case):
+    rng = np.random.default_rng(9500 + case)
+    op = ("reduce_scatter", "all_gather", "all_to_all")[rng.integers(3)]
+    codec = CODECS[rng.integers(len(CODECS))]
+    N = int(rng.integers(1, 9))
+    tiles = int(rng.integers(1, 25))
+    size = tiles * 2048
+    n_msg = N * size if op == "all_to_all" else size
+    thr = (0, 2 * n_msg, 2 * n_msg + 2)[rng.integers(3)]
+    xs = inputs(N, n_msg, int(rng.integers(1 << 20)))
+    if op == "reduce_scatter":
+        sizes = [(t1 - t0) * 2048 for t0, t1 in O.shard_tiles(N, tiles)]
+        ref, used = O.reduce_scatter(xs, codec, thr)
+    elif op == "all_gather":
+        sizes = [N * size] * N
+        ref, used = O.all_gather(xs, codec, thr)
+    else:
+        sizes = [N * size] * N
+        ref, used = O.all_to_all(xs, codec, thr)
+    outs, eff = run(L, op, xs, size, codec, sizes, thr)
+    assert eff == used
+    for j, (o, r) in enumerate(zip(outs, ref)):
+        assert np.array_equal(o, r), (op, codec, N, tiles, thr, j)
+
+
 @pytest.mark.parametrize("codec", CODECS)
 @pytest.mark.parametrize("N,tiles", [(1, 5), (2, 9), (3, 13), (5, 3), (8, 21)])
 def test_reduce_scatter_matches_oracle(L, codec, N, tiles):
