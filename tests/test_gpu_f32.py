@@ -136,3 +136,23 @@ def test_allreduce_f32_prefill_shape_sampled(L):
     ref, _ = O.allreduce_f32(sample, "fp8")
     for o in outs:
         assert np.array_equal(o[idx].cpu().numpy().view(np.uint32), ref[0].view(np.uint32))
+
+
+# Seeded random cases: codec, N in 1..8, 1..30 tiles, a threshold either side
+# of the binary32 message, in place or not.
+@pytest.mark.parametrize("case", range(24))
+def test_allreduce_f32_random_cases(L, case):
+    rng = np.random.default_rng(9700 + case)
+    codec = CODECS[rng.integers(len(CODECS))]
+    N = int(rng.integers(1, 9))
+    tiles = int(rng.integers(1, 31))
+    n = tiles * 2048
+    thr = (0, 4 * n, 4 * n + 4)[rng.integers(3)]
+    inplace = bool(rng.integers(2))
+    xs = [adversarial_f32(n, int(rng.integers(1 << 20))) for _ in range(N)]
+    outs, eff = run(L, xs, codec, min_quant_bytes=thr, inplace=inplace)
+    ref, used = O.allreduce_f32(xs, codec, thr)
+    assert eff == used
+    for o in outs:
+        assert np.array_equal(o.view(np.uint32), ref[0].view(np.uint32)), (codec, N, tiles, thr, inplace)
+
