@@ -17,7 +17,9 @@
 // The BF16 passthrough (below the threshold, or codec BF16) moves the BF16
 // values themselves.  Each quantising collective is one persistent kernel of
 // the single-pass shape (see lpar_kernels.cu): a CTA quantises a 4-tile chunk,
-// then reduces or decodes it while cp.async prefetches the next chunk.
+// then reduces or decodes it while cp.async prefetches the next chunk.  The
+// reductions come in a warp-local and a CTA-wide form (picked by codec, N and
+// size), the all-gather and all-to-all send their outputs by bulk copies.
 #include "lpar.h"
 #include "lpar_codec.cuh"
 #include "lpar_tiles.cuh"

@@ -10,8 +10,10 @@
 //   K23 k_reduce<.., true>   K2 plus the decode of the gathered block straight
 //                        from registers into every rank's BF16 output
 //   K3  k_decode        gathered wire -> BF16 into every rank's output
-//   K123 k_allreduce_single  all three stages in one persistent kernel (the
-//                        default schedule)
+//   K123 all three stages in one persistent kernel (the default schedule), in
+//        two forms: k_allreduce_single_warp (warp-local, no CTA barrier) and
+//        k_allreduce_single (CTA-wide, output by bulk copies from 128 MiB of
+//        input); launch_single_cn picks one by codec, N and size
 // The BF16 passthrough uses k_bf16_reduce (FP32 sum, one BF16 rounding) and
 // k_broadcast (plain copies).  The one-shot schedule's kernel lives with the
 // standalone collectives (lpar_collectives.cu), the binary32 all-reduce in

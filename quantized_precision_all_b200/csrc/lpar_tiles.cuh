@@ -8,6 +8,8 @@
 // so packed loads/stores are coalesced as they are.  The BF16 side (64 B per
 // thread) is staged through shared memory with an XOR swizzle so both the
 // coalesced global access and the per-thread 64-B access are bank-conflict free.
+// The warp-local kernels stage per warp: warp w copies, reads and stores only
+// its half tile (bytes [2048w, 2048w + 2048) of a stage).
 #pragma once
 
 #include "lpar.h"
