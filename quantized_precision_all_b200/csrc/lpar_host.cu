@@ -21,6 +21,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #define LPAR_API extern "C" __attribute__((visibility("default")))
 
@@ -30,6 +31,14 @@ constexpr size_t kTile = 2048;   // elements per tile
 constexpr int kSlots = 3;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around the call (host-side enqueue), as for every C ABI call.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 
 size_t round16(size_t b) { return (b + 15) & ~(size_t)15; }
 
@@ -171,6 +180,7 @@ LPAR_API size_t lpar_host_staging_bytes_f32(int N, size_t chunk, lpar_codec_t co
 LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
                                            void *const *host_out, size_t chunk, void *device, size_t device_bytes,
                                            const lpar_options_t *opts, cudaStream_t stream) {
+    Range trace("lpar_allreduce_host");
     const lpar_status_t st = check_host_args(host_inputs, N, n, codec, host_out, chunk, device, opts);
     if (st != LPAR_OK || n == 0) return st;
     const lpar_codec_t eff = lpar_effective_codec(n, codec, opts);    // decided on the whole message
@@ -188,6 +198,7 @@ LPAR_API lpar_status_t lpar_allreduce_host(const void *const *host_inputs, int N
 LPAR_API lpar_status_t lpar_allreduce_f32_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
                                                void *const *host_out, size_t chunk, void *device,
                                                size_t device_bytes, const lpar_options_t *opts, cudaStream_t stream) {
+    Range trace("lpar_allreduce_f32_host");
     const lpar_status_t st = check_host_args(host_inputs, N, n, codec, host_out, chunk, device, opts);
     if (st != LPAR_OK || n == 0) return st;
     const int schedule = opts ? (int)opts->schedule : (int)LPAR_SCHEDULE_AUTO;

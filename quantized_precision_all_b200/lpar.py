@@ -317,6 +317,24 @@ def allreduce_host(host_inputs, codec, out=None, chunk=HOST_CHUNK_ELEMS, device_
     return out
 
 
+def allreduce_f32_host(host_inputs, codec, out=None, chunk=HOST_CHUNK_ELEMS // 2, device_buffer=None,
+                       min_quant_bytes=0, stream=None, device=None):
+    """All-reduce a list of N equal-size binary32 host tensors (pin them for
+    overlap) through the device in chunks; returns the N host outputs."""
+    import torch
+    n = host_inputs[0].numel()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in host_inputs]
+    c = max(2048, min(chunk, n))
+    need = lpar_host_staging_bytes_f32(len(host_inputs), c, lpar_effective_codec(2 * n, codec, min_quant_bytes))
+    if device_buffer is None:
+        device_buffer = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    lpar_allreduce_f32_host(host_inputs, n, codec, out, c, device_buffer, device_buffer.numel(), min_quant_bytes,
+                            "auto", stream)
+    return out
+
+
 def shard_tiles(N, T):
     """Tile range [t0, t1) of reduce-scatter shard j, j = 0..N-1 (floor partition)."""
     return [(j * T // N, (j + 1) * T // N) for j in range(N)]

@@ -152,3 +152,15 @@ def test_f32_host_threshold_on_the_whole_message(L):
     assert used == "fp8"
     assert np.array_equal(hout[0].numpy().view(np.uint32), ref[0].view(np.uint32))
 
+
+def test_f32_helper(L):
+    from tests.test_gpu_f32 import adversarial_f32
+    n = 2048 * 12
+    xs = [adversarial_f32(n, 3950 + r) for r in range(3)]
+    outs = L.allreduce_f32_host([torch.from_numpy(x.copy()).pin_memory() for x in xs], "int4", chunk=2048 * 4)
+    torch.cuda.current_stream().synchronize()
+    ref, _ = O.allreduce_f32(xs, "int4")
+    for o in outs:
+        assert o.is_pinned()
+        assert np.array_equal(o.numpy().view(np.uint32), ref[0].view(np.uint32))
+
