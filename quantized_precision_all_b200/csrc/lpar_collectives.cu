@@ -372,54 +372,56 @@ static inline bool rs_warp_form(int C, int N, bool ALL, size_t in_bytes) {
 }
 
 template <int C, int N, bool ALL>
-static void launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
+static bool launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
     if (rs_warp_form(C, N, ALL, (size_t)N * tiles * (kTileElems * 2))) {
         constexpr int smem = 3 * kStageBytes;
-        if (!allow_dynamic_smem<k_reduce_bf16_warp<C, N, ALL>>(smem)) return;   // reported by launch_status
+        if (!allow_dynamic_smem<k_reduce_bf16_warp<C, N, ALL>>(smem)) return false;
         const unsigned grid = persistent_grid(chunks, resident_ctas<k_reduce_bf16_warp<C, N, ALL>>(smem));
         k_reduce_bf16_warp<C, N, ALL><<<grid, kThreads, smem, st>>>(in, wire, out, tiles, chunks);
-        return;
+        return true;
     }
     const unsigned grid = persistent_grid(chunks, resident_ctas<k_reduce_bf16_single<C, N, ALL>>());
     k_reduce_bf16_single<C, N, ALL><<<grid, kThreads, 0, st>>>(in, wire, out, tiles, chunks);
+    return true;
 }
 
 template <int N, bool ALL>
-static void launch_rb_na(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles,
+static bool launch_rb_na(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles,
                          cudaStream_t st) {
     switch (codec) {
-    case kINT4: launch_rb_cna<kINT4, N, ALL>(in, wire, out, tiles, st); break;
-    case kINT3: launch_rb_cna<kINT3, N, ALL>(in, wire, out, tiles, st); break;
-    case kFP8: launch_rb_cna<kFP8, N, ALL>(in, wire, out, tiles, st); break;
-    case kMXFP4: launch_rb_cna<kMXFP4, N, ALL>(in, wire, out, tiles, st); break;
+    case kINT4: return launch_rb_cna<kINT4, N, ALL>(in, wire, out, tiles, st);
+    case kINT3: return launch_rb_cna<kINT3, N, ALL>(in, wire, out, tiles, st);
+    case kFP8: return launch_rb_cna<kFP8, N, ALL>(in, wire, out, tiles, st);
+    case kMXFP4: return launch_rb_cna<kMXFP4, N, ALL>(in, wire, out, tiles, st);
     default: {
         const unsigned grid = (unsigned)std::min<size_t>(tiles, (size_t)1 << 20);
         k_bf16_reduce_to<N, ALL><<<grid, kThreads, 0, st>>>(in, out, tiles);
+        return true;
     }
     }
 }
 
 template <bool ALL>
-static void launch_rb_a(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
+static bool launch_rb_a(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N, size_t tiles,
                         cudaStream_t st) {
     switch (N) {
-    case 1: launch_rb_na<1, ALL>(codec, in, wire, out, tiles, st); break;
-    case 2: launch_rb_na<2, ALL>(codec, in, wire, out, tiles, st); break;
-    case 3: launch_rb_na<3, ALL>(codec, in, wire, out, tiles, st); break;
-    case 4: launch_rb_na<4, ALL>(codec, in, wire, out, tiles, st); break;
-    case 5: launch_rb_na<5, ALL>(codec, in, wire, out, tiles, st); break;
-    case 6: launch_rb_na<6, ALL>(codec, in, wire, out, tiles, st); break;
-    case 7: launch_rb_na<7, ALL>(codec, in, wire, out, tiles, st); break;
-    case 8: launch_rb_na<8, ALL>(codec, in, wire, out, tiles, st); break;
-    default: break;
+    case 1: return launch_rb_na<1, ALL>(codec, in, wire, out, tiles, st);
+    case 2: return launch_rb_na<2, ALL>(codec, in, wire, out, tiles, st);
+    case 3: return launch_rb_na<3, ALL>(codec, in, wire, out, tiles, st);
+    case 4: return launch_rb_na<4, ALL>(codec, in, wire, out, tiles, st);
+    case 5: return launch_rb_na<5, ALL>(codec, in, wire, out, tiles, st);
+    case 6: return launch_rb_na<6, ALL>(codec, in, wire, out, tiles, st);
+    case 7: return launch_rb_na<7, ALL>(codec, in, wire, out, tiles, st);
+    case 8: return launch_rb_na<8, ALL>(codec, in, wire, out, tiles, st);
+    default: return false;
     }
 }
 
-void launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
+bool launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
                            size_t tiles, bool all, cudaStream_t st) {
-    if (all) launch_rb_a<true>(codec, in, wire, out, N, tiles, st);
-    else launch_rb_a<false>(codec, in, wire, out, N, tiles, st);
+    return all ? launch_rb_a<true>(codec, in, wire, out, N, tiles, st)
+               : launch_rb_a<false>(codec, in, wire, out, N, tiles, st);
 }
 
 template <int C, bool A2A>
@@ -524,7 +526,7 @@ LPAR_API lpar_status_t lpar_reduce_scatter(const void *const *inputs, int N, siz
                                               workspace_bytes, opts, in, o, wires, eff, n_msg);
     if (st != LPAR_OK || n_msg == 0) return st;
     mark(opts, 0, stream);
-    launch_reduce_to_bf16(eff, in, wires, o, N, n / kTileElems, false, stream);
+    if (!launch_reduce_to_bf16(eff, in, wires, o, N, n / kTileElems, false, stream)) return LPAR_ERR_CUDA;
     mark(opts, 1, stream);
     return launch_status();
 }

@@ -649,7 +649,7 @@ LPAR_API lpar_status_t lpar_allreduce(const void *const *inputs, int N, size_t n
         const size_t wb1 = eff == LPAR_CODEC_BF16 ? 0 : lpar_wire_bytes(eff, n);
         for (int r = 0; r < N; ++r) w1.p[r] = ws + (size_t)r * wb1;
         if (opts && opts->stage_events[0]) cudaEventRecord(opts->stage_events[0], stream);
-        launch_reduce_to_bf16(eff, in, w1, o, N, tiles, true, stream);
+        if (!launch_reduce_to_bf16(eff, in, w1, o, N, tiles, true, stream)) return LPAR_ERR_CUDA;
         if (opts && opts->stage_events[1]) cudaEventRecord(opts->stage_events[1], stream);
         return launch_status();
     }

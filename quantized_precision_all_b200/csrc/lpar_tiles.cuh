@@ -445,8 +445,8 @@ static inline lpar_status_t launch_status() {
 // once to BF16, no requantisation), defined in lpar_collectives.cu: into every
 // out[r] (all = true: the one-shot all-reduce) or into the shard owners
 // (all = false: the reduce-scatter).  `wire` holds N stage-1 wires (unused
-// for BF16).
-void launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
+// for BF16).  False when the launch could not be configured.
+bool launch_reduce_to_bf16(int codec, const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, int N,
                            size_t tiles, bool all, cudaStream_t st);
 
 }  // namespace lpar
