@@ -1,0 +1,91 @@
+"""bench.py's byte model on the host (no GPU): the algorithmic bytes behind every
+roofline fraction, checked against the per-element model they come from (stage-1
+wires written and read back, one gathered wire, N outputs), against the figures
+quoted in profiles/, and the kernel labels against the library's choice of form."""
+import os
+import random
+import re
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+C = bench.CODEC_C
+
+
+def test_wire_bytes_per_element_are_the_tile_sizes():
+    assert C["int4"] * 2048 == 1152 and C["int3"] * 2048 == 896
+    assert C["fp8"] * 2048 == 2304 and C["mxfp4"] * 2048 == 1088 and C["bf16"] == 2
+
+
+@pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4"])
+def test_single_pass_bytes_follow_the_per_element_model(codec):
+    # per N*n elements: 2 in + c wire out + c wire back in + c/N gathered wire + 2 out
+    rng = random.Random(1)
+    for _ in range(50):
+        N = rng.randint(1, 8)
+        n = 2048 * rng.randint(1, 1 << 18)
+        c = C[codec]
+        got = bench.algorithmic_bytes("k_allreduce_single<%s,N=%d>" % (codec, N), codec, N, n)
+        assert got == pytest.approx(N * n * (4 + 2 * c + c / N))
+        assert bench.algorithmic_bytes("k_allreduce_single_warp<%s,N=%d>" % (codec, N), codec, N, n) == got
+
+
+def test_schedules_move_the_same_bytes_as_single_pass():
+    N, n = 4, 2048 * 1000
+    for codec in ("int4", "int3", "fp8", "mxfp4"):
+        single = bench.algorithmic_bytes("k_allreduce_single<x>", codec, N, n)
+        fused = sum(bench.algorithmic_bytes(k, codec, N, n) for k in bench.kernel_names(codec, "fused", N))
+        three = sum(bench.algorithmic_bytes(k, codec, N, n) for k in bench.kernel_names(codec, "three_stage", N))
+        assert fused == pytest.approx(single)
+        assert three == pytest.approx(single + n * C[codec])  # K3 also reads the gathered wire
+
+
+def test_binary32_bytes():
+    N, n = 8, 2048 * 8192
+    c = C["fp8"]
+    assert bench.algorithmic_bytes("k_allreduce_single_f32<fp8,N=8>", "fp8", N, n) == \
+        pytest.approx(N * n * (4 + c) + n * (N * c + c + 4 * N))
+    assert bench.algorithmic_bytes("k_f32_reduce<N=8>", "bf16", N, n) == n * (8 * N + 4)
+
+
+def test_profiles_quote_the_model():
+    """The algorithmic bytes printed in profiles/dram_traffic.txt are the model's."""
+    text = open(os.path.join(ROOT, "profiles", "dram_traffic.txt")).read()
+    n = 512 * 1024 * 1024
+    assert "5469372416" in text and "5804916736" in text and "5721030656" in text
+    assert bench.algorithmic_bytes("k_allreduce_single_warp<int3,N=2>", "int3", 2, n) == 5469372416
+    assert bench.algorithmic_bytes("k_allreduce_single<int4,N=2>", "int4", 2, n) == 5804916736
+    assert bench.algorithmic_bytes("k_allreduce_single<mxfp4,N=2>", "mxfp4", 2, n) == 5721030656
+    for line in re.findall(r"^kernel=.*$", text, re.M):
+        kv = dict(f.split("=", 1) for f in line.split())
+        assert int(kv["bytes_per_launch"]) == int(kv["read"]) + int(kv["write"])
+
+
+def test_collective_bytes():
+    N, m = 4, 2048 * 100
+    c = C["int3"]
+    assert bench.collective_bytes("reduce_scatter", "int3", N, m) == pytest.approx(N * m * (2 + c) + N * m * c + 2 * m)
+    assert bench.collective_bytes("one_shot", "int3", N, m) == pytest.approx(N * m * (2 + 2 * c) + 2 * N * m)
+    assert bench.collective_bytes("all_gather", "int3", N, m) == pytest.approx(N * m * (2 + c) + 2 * N * N * m)
+    assert bench.collective_bytes("all_to_all", "int3", N, m) == pytest.approx(N * N * m * (2 + c) + 2 * N * N * m)
+    assert bench.collective_bytes("all_gather", "bf16", N, m) == N * 2 * m + 2 * N * N * m
+
+
+def test_single_pass_labels_follow_the_launcher_rule():
+    mib = 1 << 20
+    k = bench.single_pass_kernel
+    assert k("int3", 2, 512 * mib).startswith("k_allreduce_single_warp")        # INT3, N <= 2: always
+    assert k("int3", 8, 16 * mib).startswith("k_allreduce_single_warp")         # 256 MiB < 512 MiB of input
+    assert k("int3", 8, 64 * mib).startswith("k_allreduce_single<")             # 1 GiB of input
+    assert k("int4", 2, 16 * mib).startswith("k_allreduce_single_warp")         # 64 MiB < 128 MiB
+    assert k("int4", 2, 32 * mib).startswith("k_allreduce_single<")             # 128 MiB
+    assert k("mxfp4", 4, 8 * mib).startswith("k_allreduce_single_warp")
+    assert k("fp8", 2, 1024).startswith("k_allreduce_single<")                  # FP8: always CTA-wide
+    src = open(os.path.join(ROOT, "quantized_precision_all_b200", "csrc", "lpar_kernels.cu")).read()
+    assert "kBulkMinBytes = (size_t)128 << 20" in src and "kInt3WarpMaxBytes = (size_t)512 << 20" in src
+    assert bench.BULK_MIN_BYTES == 128 * mib and bench.INT3_WARP_MAX_BYTES == 512 * mib
