@@ -1,5 +1,6 @@
 """The oracle's all-reduce over tile ranges on all host cores.  TEST
-INFRASTRUCTURE ONLY (the CPU-baseline legs of ``bench.py`` call it).
+INFRASTRUCTURE ONLY (the CPU-baseline legs of ``bench.py`` time it; the GPU
+parity tests use `allreduce` to check whole messages against it).
 
 Every tile of the collective depends only on the same tile of every rank, so
 the oracle's all-reduce of a tile range is exactly its share of the whole call.
@@ -56,6 +57,71 @@ def _worker_main(argv=None):
             fn(xs, c, 0)
     b = time.perf_counter()
     print("done %.9f %.9f" % (a, b), flush=True)
+
+
+def _compute_main(argv=None):
+    """Worker of `allreduce`: the oracle's all-reduce of its tile range with
+    each codec in turn, written into the output file at that range (rank 0's
+    output: every rank receives the same values); prints `done`."""
+    in_path, out_path, N, n, t0, t1, codecs = (argv or sys.argv[1:])
+    N, n, t0, t1 = int(N), int(n), int(t0), int(t1)
+    codecs = codecs.split(",")
+    arr = np.memmap(in_path, dtype=np.uint16, mode="r", shape=(N, n))
+    xs = [np.array(arr[r, t0 * O.TILE_ELEMS:t1 * O.TILE_ELEMS]) for r in range(N)]
+    del arr
+    res = np.memmap(out_path, dtype=np.uint16, mode="r+", shape=(len(codecs), n))
+    for k, c in enumerate(codecs):
+        outs, _ = O.allreduce(xs, c, 0)
+        res[k, t0 * O.TILE_ELEMS:t1 * O.TILE_ELEMS] = outs[0]
+    res.flush()
+    del res
+    print("done 0 0", flush=True)
+
+
+def allreduce(xs, codecs, workers=None, timeout=1800.0):
+    """The oracle's all-reduce of the N host arrays `xs` (BF16 bits as uint16,
+    whole tiles) for every codec of `codecs` (each the codec the message runs
+    with: no threshold), over tile ranges on every host core.  Returns
+    {codec: the result every rank receives}."""
+    N, n = len(xs), xs[0].size
+    T = n // O.TILE_ELEMS
+    P = max(1, min(workers or host_cores(), T))
+    O.lib()
+    tmpdir = "/dev/shm" if os.path.isdir("/dev/shm") else None
+    paths = []
+    procs = []
+    try:
+        for suffix in (".in", ".out"):
+            fd, path = tempfile.mkstemp(prefix="lpar_oracle_", suffix=suffix, dir=tmpdir)
+            os.close(fd)
+            paths.append(path)
+        arr = np.memmap(paths[0], dtype=np.uint16, mode="w+", shape=(N, n))
+        for r, x in enumerate(xs):
+            arr[r] = np.asarray(x, dtype=np.uint16).reshape(-1)
+        arr.flush()
+        del arr
+        res = np.memmap(paths[1], dtype=np.uint16, mode="w+", shape=(len(codecs), n))
+        res.flush()
+        del res
+        env = dict(os.environ, PYTHONPATH=_ROOT + os.pathsep + os.environ.get("PYTHONPATH", ""))
+        for k in range(P):
+            t0, t1 = k * T // P, (k + 1) * T // P
+            args = [paths[0], paths[1], N, n, t0, t1, ",".join(codecs)]
+            procs.append(subprocess.Popen(
+                [sys.executable, "-c", "from oracle.parallel import _compute_main; _compute_main()"] + [str(a) for a in args],
+                stdin=subprocess.DEVNULL, stdout=subprocess.PIPE, text=True, env=env, cwd=_ROOT))
+        _read_lines(procs, "done", time.monotonic() + timeout)
+        for p in procs:
+            p.wait(timeout=60)
+        res = np.array(np.memmap(paths[1], dtype=np.uint16, mode="r", shape=(len(codecs), n)))
+        return {c: res[k] for k, c in enumerate(codecs)}
+    finally:
+        for p in procs:
+            if p.poll() is None:
+                p.kill()
+                p.wait()
+        for path in paths:
+            os.unlink(path)
 
 
 def _read_lines(procs, want, deadline):

@@ -60,6 +60,15 @@ def test_runner_splits_over_workers():
     assert used == 2 and dt > 0
 
 
+def test_whole_message_over_workers_equals_one_call():
+    xs = bf16_inputs(3, 11, 21)
+    codecs = ["int4", "int3", "fp8", "mxfp4", "bf16"]
+    got = OP.allreduce(xs, codecs, workers=4)
+    for c in codecs:
+        ref, _ = O.allreduce(xs, c)
+        assert np.array_equal(got[c], ref[0]), c
+
+
 def test_runner_reports_a_failing_worker():
     xs = bf16_inputs(2, 2, 3)
     with pytest.raises(RuntimeError):
