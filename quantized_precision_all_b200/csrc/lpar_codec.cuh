@@ -629,26 +629,28 @@ __device__ __forceinline__ void int4_word_to_h2(uint32_t w, uint32_t (&h)[4]) {
 
 // INT3 half-block (elements 16*half .. 16*half+15) -> eight packed binary16
 // pairs of q.  Codes are assembled one per nibble: the low two bits of the
-// even (odd) elements are q2w & 0x33333333 ((q2w >> 2) & 0x33333333), and the
-// q1w bits of the same elements are deposited at bit 2 of each nibble.  A
-// nibble code c (0..7) then indexes an 8-byte table with one PRMT: the binary16
-// value of q = c - 4 is -4, -3, ..., 3, whose low byte is always 0, so the
-// table holds only the high bytes and two more PRMTs interleave zero bytes.
+// even (odd) elements are q2w & 0x33333333 ((q2w >> 2) & 0x33333333).  The
+// sixteen q1w bits of the half are spread to every second bit (bit j -> bit
+// 2j), which puts the bit of element 2k at 4k and that of element 2k + 1 at
+// 4k + 2: the odd elements' high bits are then in place, the even elements'
+// two bits to the left.  A nibble code c (0..7) indexes an 8-byte table with
+// one PRMT: the binary16 value of q = c - 4 is -4, -3, ..., 3, whose low byte
+// is always 0, so the table holds only the high bytes and two more PRMTs
+// interleave zero bytes.
 // h[0..3] = (e0,e2) (e4,e6) (e8,e10) (e12,e14); h[4..7] = (e1,e3) (e5,e7)
 // (e9,e11) (e13,e15), indices relative to 16*half.
-__device__ __forceinline__ uint32_t deposit_even_bits(uint32_t x) {   // bit 2k of x (k < 8) -> bit 4k+2
-    uint32_t t = x & 0x5555u;
-    t = (t | (t << 8)) & 0x00550055u;
-    t = (t | (t << 4)) & 0x05050505u;
-    t = (t | (t << 2)) & 0x11111111u;
-    return t << 2;
+__device__ __forceinline__ uint32_t spread_half_bits(uint32_t q1w, int half) {   // bit 16*half + j -> bit 2j
+    uint32_t t = __byte_perm(q1w, 0u, half ? 0x4342 : 0x4140);              // byte k -> byte 2k
+    t = (t | (t << 4)) & 0x0F0F0F0Fu;
+    t = (t | (t << 2)) & 0x33333333u;
+    return (t | (t << 1)) & 0x55555555u;
 }
 
 __device__ __forceinline__ void int3_half_to_h2(const Packed<kINT3> &p, int half, uint32_t (&h)[8]) {
     const uint32_t w = p.q2w[half];
-    const uint32_t q1 = p.q1w >> (16 * half);
-    const uint32_t ce = (w & 0x33333333u) | deposit_even_bits(q1);          // even elements
-    const uint32_t co = ((w >> 2) & 0x33333333u) | deposit_even_bits(q1 >> 1);   // odd elements
+    const uint32_t d = spread_half_bits(p.q1w, half);
+    const uint32_t ce = (w & 0x33333333u) | ((d << 2) & 0xCCCCCCCCu);        // even elements
+    const uint32_t co = ((w >> 2) & 0x33333333u) | (d & 0xCCCCCCCCu);        // odd elements
     const uint32_t T0 = 0xBCC0C2C4u;       // high bytes of -1, -2, -3, -4 (codes 3..0)
     const uint32_t T1 = 0x42403C00u;       // high bytes of  3,  2,  1,  0 (codes 7..4)
     const uint32_t e0 = __byte_perm(T0, T1, ce), e1 = __byte_perm(T0, T1, ce >> 16);
