@@ -226,6 +226,45 @@ def test_reduce_matches_oracle_on_a_tile_range(L, codec, N):
     assert np.array_equal(out.host(), ref)            # tiles outside the range untouched
 
 
+def arbitrary_wire(codec, n, rng, tile_bytes):
+    """Random code bytes (every bit pattern is a code the decoder accepts, including
+    the INT codes -2^(b-1) that the encoder never writes) with random scales:
+    binary16 of either sign, subnormals and 65504 included; E8M0 bytes 0..249.
+    Non-finite values are outside the method's definition, so the E8M0 bytes stop
+    where a sum of eight decoded values stays finite (|e| 2^E <= 6 * 2^122)."""
+    wire = rng.integers(0, 256, (n // 2048) * tile_bytes, dtype=np.uint8)
+    for t in range(n // 2048):
+        if codec == "mxfp4":
+            wire[t * tile_bytes + 1024:(t + 1) * tile_bytes] = rng.integers(0, 250, 64).astype(np.uint8)
+        else:
+            sc = rng.integers(0, 0x7C00, 64).astype(np.uint16) | (rng.integers(0, 2, 64).astype(np.uint16) << 15)
+            wire[(t + 1) * tile_bytes - 128:(t + 1) * tile_bytes] = sc.view(np.uint8)
+    return wire
+
+
+@pytest.mark.parametrize("codec", ["int4", "int3", "mxfp4"])
+@pytest.mark.parametrize("N", [1, 2, 3, 8])
+def test_reduce_arbitrary_code_bytes(L, codec, N):
+    # stage 2 decodes every code pattern of N ranks, sums and requantises; the
+    # sums reach the saturated and subnormal scales
+    n = 2048 * 5
+    rng = np.random.default_rng(400 + N)
+    tb = L.lpar_tile_bytes(codec)
+    wires = [arbitrary_wire(codec, n, rng, tb) for _ in range(N)]
+    for w in wires:                                   # finite by construction
+        assert np.all((O.decode(w, n, codec) & 0x7FFF) < 0x7F80)
+    dws = []
+    for w in wires:
+        g = Guarded(w.size)
+        g.t.copy_(torch.from_numpy(w))
+        dws.append(g)
+    out = Guarded(wires[0].size)
+    L.lpar_reduce([g.ptr() for g in dws], 0, n // 2048, codec, out.ptr())
+    torch.cuda.synchronize()
+    out.check()
+    assert np.array_equal(out.host(), O.reduce(wires, 0, n // 2048, codec))
+
+
 @pytest.mark.parametrize("bits,codec", [(4, "int4"), (3, "int3")])
 def test_reduce_exact_ties_at_stage_two(L, bits, codec):
     # rank 0 holds q0 * S (absmax qmax * S), rank 1 holds odd multiples of S/2 with
