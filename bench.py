@@ -2,19 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--schedule fused|three_stage]
+    python bench.py --sweep | --collectives | --floor       (one JSON line per point)
 
 A step is one pass of the whole path (quantise -> reduce + requantise ->
-decode, all simulated ranks) for every codec of the workload, back to back.
-Default workload: ``large_int3_int4`` (N=2 simulated ranks x 1 GiB BF16 per
-rank, INT3 then INT4), the large-message configuration on which the HBM
-roofline target is defined; its inputs (2 GiB) are far larger than the 126 MB
-L2, so no flush is needed between steps.
+decode, all ranks) for every codec of the workload, back to back.  Default
+workload: ``large_int3_int4`` (2 ranks x 1 GiB BF16 per rank, INT3 then INT4),
+the large-message configuration on which the HBM roofline target is defined;
+its inputs (2 GiB) are far larger than the 126 MB L2, so no flush is needed
+between steps.
 
-Metric: GB/s = (simulated ranks x per-rank BF16 bytes x codecs) / time, plus
-the fraction of measured HBM bandwidth the dominant kernel reaches.  With
-``--gpus G`` (torchrun, one process per GPU) every GPU runs its own
-independent instance of the workload (weak scaling); there is no data-path
-collective -- the N simulated ranks of one instance live in one GPU's HBM.
+Metric: GB/s = (ranks x per-rank BF16 bytes x codecs) / time.  On one GPU the
+ranks are simulated in its HBM (the emulated reduce-scatter / all-gather) and
+the roofline is the fraction of measured HBM bandwidth the dominant kernel
+reaches.  With ``--gpus G > 1`` (torchrun, one process per GPU) the ranks are
+the G processes: every GPU holds one rank's message of the workload's size and
+the step is the real all-reduce across them (``distributed.DistributedAllreduce``:
+the library's stage kernels, NCCL all-to-all and all-gather of the wire bytes);
+its roofline is the NVLink bytes each rank sends.
 """
 import argparse
 import hashlib
@@ -43,6 +47,8 @@ REF_TILES_PER_STEP = 256            # reference arm: 0.5 Mi elements per rank pe
 CPU_BASELINE_TILES = 16384          # cpu_baseline: 32 Mi elements (64 MiB) per rank
 PAR_TILES_PER_CORE = 2048           # cpu_baseline on every core: 4 Mi elements per rank per core
 HOST_CHUNK_BYTES = 32 << 20         # e2e: bytes of one chunk of the host all-reduce, all ranks together
+ROTATE_BYTES = 512 << 20            # back-to-back timing: buffer sets rotated over at least this many bytes (4x L2)
+NVLINK_GBS = 770.0                  # measured peer copy per direction per GPU on this machine's B200s
 
 
 def log(*a):
@@ -128,6 +134,28 @@ def algorithmic_bytes(kernel, codec, N, n):
     if kernel == "k_broadcast":
         return n * (2 + 2 * N)
     raise ValueError(kernel)
+
+
+def min_dram_bytes(codec, N, n):
+    """The fewest DRAM bytes an emulated all-reduce call can move: every input
+    read, every stage-1 wire and the gathered wire written once (they are the
+    transmitted data), every output written; the wires' read-back may come from
+    L2.  ncu DRAM bytes of the large workloads sit at this figure."""
+    c = CODEC_C[codec]
+    if codec == "bf16":
+        return n * (2 * N + 2 + 2 * N)
+    return N * n * (4 + c) + n * c
+
+
+def min_dram_for(kernel, codec, N, n):
+    """min_dram_bytes for the single-pass kernels (whose stage-1 read-back may
+    hit L2); the algorithmic bytes for every other kernel."""
+    c = CODEC_C[codec]
+    if kernel.startswith("k_allreduce_single_f32"):
+        return N * n * (4 + c) + n * c + 4 * N * n
+    if kernel.startswith("k_allreduce_single"):
+        return min_dram_bytes(codec, N, n)
+    return algorithmic_bytes(kernel, codec, N, n)
 
 
 def traffic_for(kernel, workload):
@@ -293,6 +321,7 @@ def run_ours(args, rank, world, device):
         d["ms_per_launch"] = d["ms_total"] / d["launches"]
         d["algorithmic_bytes"] = algorithmic_bytes(name, d["codec"], N, n)
         d["achieved_gbs"] = d["algorithmic_bytes"] / (d["ms_per_launch"] * 1e-3) / 1e9
+        d["min_dram_bytes"] = min_dram_for(name, d["codec"], N, n)
     launches_per_step = sum(len(kernel_names(eff_codec(c), args.schedule, N, f32)) for c in w.codecs)
 
     # (3) accuracy of this step's outputs on sampled tiles (outside the timed region)
@@ -357,6 +386,97 @@ def run_ours(args, rank, world, device):
 
     return {"ms": ms_max, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
             "e2e": e2e, "cpu": cpu, "w": w, "accuracy": accuracy}
+
+
+def nvlink_bytes_sent(world, n, codec, chunks, rank=0):
+    """Wire bytes one rank sends in one real all-reduce: its wire minus its own
+    shard in the all-to-all, its padded send slot to every peer in the
+    all-gather, chunk by chunk."""
+    from quantized_precision_all_b200 import distributed as D
+    tb = int(round(CODEC_C[codec] * TILE))
+    total = 0
+    for t0, t1 in D.chunk_tiles(n // TILE, chunks):
+        shards = D.shard_tiles(world, t1 - t0)
+        width = max(b - a for a, b in shards) * tb
+        total += (t1 - t0) * tb - (shards[rank][1] - shards[rank][0]) * tb + (world - 1) * width
+    return total
+
+
+def run_distributed(args, rank, world, device):
+    """The real all-reduce across the `world` processes (one GPU each): rank r
+    holds rank r's message of the workload (same size, same seeded recipe);
+    each step runs every codec of the workload through DistributedAllreduce."""
+    from quantized_precision_all_b200.distributed import DistributedAllreduce
+    w = W.WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        raise SystemExit("the cross-GPU all-reduce takes BF16 messages")
+    n = w.n
+    x = W.make_rank_input(w, rank, device)
+    out = torch.empty_like(x)
+    ar = DistributedAllreduce(chunks=args.chunks)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for codec in w.codecs:
+            ar.allreduce(x, codec, w.min_quant_bytes, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    torch.distributed.barrier()
+    ms_max = max_over_ranks(start.elapsed_time(end), world, device)
+
+    def eff(c):
+        return c if c == "bf16" or 2 * n >= w.min_quant_bytes else "bf16"
+
+    sent = sum(nvlink_bytes_sent(world, n, eff(c), args.chunks, rank) for c in w.codecs)
+    launches = 0
+    from quantized_precision_all_b200 import distributed as D
+    for c in w.codecs:
+        for t0, t1 in D.chunk_tiles(n // TILE, args.chunks):
+            launches += 2 + sum(1 for a, b in D.shard_tiles(world, t1 - t0) if b > a)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 5))
+        h_in = torch.empty(n, dtype=x.dtype, pin_memory=True)
+        h_in.copy_(x)
+        h_out = torch.empty(n, dtype=x.dtype, pin_memory=True)
+
+        def e2e_step():
+            for codec in w.codecs:
+                x.copy_(h_in, non_blocking=True)
+                ar.allreduce(x, codec, w.min_quant_bytes, out=out)
+                h_out.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = max_over_ranks(s0.elapsed_time(s1), world, device)
+        per = 2 * n * len(w.codecs)
+        e2e = {"value": aggregate_gbs(world, per, e2e_steps, e_ms), "unit": "GB/s", "h2d_bytes_per_step": per,
+               "d2h_bytes_per_step": per, "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
+               "api": "DistributedAllreduce.allreduce, each rank's message uploaded from pinned host memory and "
+                      "its result downloaded, per codec"}
+        del h_in, h_out
+    ar.release()
+    return {"ms": ms_max, "clocks": clocks.summary(), "sent": sent, "launches_per_step": launches, "e2e": e2e,
+            "w": w}
 
 
 def oracle_codecs(w):
@@ -456,14 +576,90 @@ def oracle_gbs(op, N, codec, tiles=64):
             "sample": "%d tiles per rank, N=%d, %s, %s" % (tiles, N, codec, op)}
 
 
+class BufferSets:
+    """R copies of one call's buffers (inputs, outputs, workspace) at distinct
+    addresses, R chosen so that the sets span at least ROTATE_BYTES (4x L2):
+    calls that rotate over them find their inputs outside L2 even when timed
+    back to back."""
+
+    def __init__(self, xs, out_elems, ws_bytes, device, rotate=ROTATE_BYTES):
+        N, n = len(xs), xs[0].numel()
+        wsb = -(-max(ws_bytes, 16) // 256) * 256
+        set_bytes = N * n * xs[0].element_size() + N * out_elems * 2 + wsb
+        self.R = max(1, -(-rotate // set_bytes))
+        if self.R == 1:
+            self.inputs = [list(xs)]
+        else:
+            pool = torch.empty((self.R, N, n), dtype=xs[0].dtype, device=device)
+            pool[:] = torch.stack(list(xs))
+            self.inputs = [list(pool[i].unbind(0)) for i in range(self.R)]
+        outs = torch.empty((self.R, N, out_elems), dtype=torch.bfloat16, device=device)
+        self.outputs = [list(outs[i].unbind(0)) for i in range(self.R)]
+        ws = torch.empty((self.R, wsb), dtype=torch.uint8, device=device)
+        self.ws = [ws[i] for i in range(self.R)]
+        self.ws_bytes = wsb
+
+
+def time_call(call, R, flush, device, single_iters=20, batches=3):
+    """Per-call time of call(i, stream) for buffer set i, in microseconds, two ways:
+    single: one call between two CUDA events after a 256 MiB write (cold L2),
+    median of single_iters; graph: K calls rotating over the R sets captured in
+    one CUDA graph and replayed (launches pipelined, no host enqueue cost in the
+    timed region), replay time / K, median of `batches` replays.  CUDA events on
+    this pool tick in steps of about 2.05 us, so the single-call figure carries
+    that resolution and the graph figure resolves it away."""
+    stream = torch.cuda.current_stream(device)
+    for i in range(min(R, 3)):
+        call(i, stream)
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(single_iters)]
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        call(0, stream)
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    single = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+    K = min(max(2 * R, 20), 4000)
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for k in range(K):
+            call(k % R, side)
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize(device)
+    per = []
+    for _ in range(batches):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        per.append(e0.elapsed_time(e1) * 1e3 / K)
+    del g
+    return {"us_single": single, "us": statistics.median(per), "us_min": min(per), "calls_per_graph": K}
+
+
+def _fractions(alg, dram, N, mb, us, peak):
+    t = us * 1e-6
+    return {"GBps": N * mb / t / 1e9, "hbm_fraction": alg / t / 1e9 / peak, "dram_fraction": dram / t / 1e9 / peak}
+
+
 def run_sweep(args, device):
     """One JSON line per sweep point (N, message size, codec): GB/s and the
-    fraction of measured HBM peak the whole call reaches (its algorithmic
-    bytes over its time)."""
+    fraction of measured HBM peak the whole call reaches, per call back to back
+    (CUDA graph over rotating buffer sets) and as a single cold call, with the
+    SM clock record of the (N, size) group."""
     from quantized_precision_all_b200 import lpar as L
     peak, peak_src = measured_peaks()
-    stream = torch.cuda.current_stream(device)
-    cpu = {(N, c): oracle_gbs("allreduce", N, c) for N in W.SWEEP_RANKS for c in W.SWEEP_CODECS}
+    ranks = [args.sweep_n] if args.sweep_n else list(W.SWEEP_RANKS)
+    sizes = [args.sweep_mib << 20] if args.sweep_mib else list(W.SWEEP_SIZES_BYTES)
+    codecs = [args.sweep_codec] if args.sweep_codec else list(W.SWEEP_CODECS)
+    cpu = {(N, c): oracle_gbs("allreduce", N, c) for N in ranks for c in codecs}
     done = set()
     if args.resume and os.path.exists(args.resume):   # restart: skip the points already written
         with open(args.resume) as f:
@@ -472,50 +668,102 @@ def run_sweep(args, device):
                     d = json.loads(line)
                     done.add((d["N"], d["message_bytes"], d["codec"]))
     sink = open(args.resume, "a") if args.resume else None
-    for N in W.SWEEP_RANKS:
-        for mb in W.SWEEP_SIZES_BYTES:
-            if all((N, mb, c) in done for c in W.SWEEP_CODECS):
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # > L2, rewritten before single calls
+    for N in ranks:
+        for mb in sizes:
+            todo = [c for c in codecs if (N, mb, c) not in done]
+            if not todo:
                 continue
             w = W.sweep_workload(N, mb, "bf16")
             xs = W.make_inputs(w, device)
-            outs = [torch.empty_like(x) for x in xs]
-            wsb = max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS)
-            ws = torch.empty(wsb, dtype=torch.uint8, device=device)
-            flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # > L2, rewritten between calls
+            wsb = max(L.lpar_workspace_bytes(N, w.n, c) for c in todo)
+            sets = BufferSets(xs, w.n, wsb, device)
             T = w.n // TILE
             rng = torch.Generator().manual_seed(5000 + N)
             sample = torch.unique(torch.cat([torch.tensor([0, T - 1]), torch.randint(0, T, (2,), generator=rng)]))
-            for codec in W.SWEEP_CODECS:
-                if (N, mb, codec) in done:
-                    continue
-                iters = max(3, min(50, int(2e9 / (N * mb))))
-                for _ in range(3):
-                    L.lpar_allreduce(xs, w.n, codec, outs, ws, wsb, schedule=args.schedule, stream=stream)
-                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                       for _ in range(iters)]
-                for e0, e1 in evs:
-                    flush.fill_(1)
-                    e0.record(stream)
-                    L.lpar_allreduce(xs, w.n, codec, outs, ws, wsb, schedule=args.schedule, stream=stream)
-                    e1.record(stream)
-                torch.cuda.synchronize(device)
-                ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
-                names = kernel_names(codec, args.schedule, N)
-                alg = sum(algorithmic_bytes(k, codec, N, w.n) for k in names)
-                row = json.dumps({"sweep": True, "N": N, "message_bytes": mb, "codec": codec,
-                                  "schedule": args.schedule, "ms": ms,
-                                  "GBps": N * mb / (ms * 1e-3) / 1e9, "algorithmic_bytes": alg,
-                                  "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
-                                  "l2": "256 MiB buffer rewritten before every timed call",
-                                  "note": "L2-resident / launch-bound" if N * mb < (16 << 20) else "",
-                                  "peak": peak, "cpu_baseline": cpu[(N, codec)], "seed": w.seed,
-                                  **sample_check(xs, outs, sample.numpy())})
-                print(row, flush=True)
+            rows = []
+            with ClockSampler(device) as clocks:
+                for codec in todo:
+                    def call(i, st, codec=codec):
+                        L.lpar_allreduce(sets.inputs[i], w.n, codec, sets.outputs[i], sets.ws[i], sets.ws_bytes,
+                                         schedule=args.schedule, stream=st)
+                    tm = time_call(call, sets.R, flush, device)
+                    names = kernel_names(codec, args.schedule, N, n=w.n)
+                    alg = sum(algorithmic_bytes(k, codec, N, w.n) for k in names)
+                    dram = min_dram_bytes(codec, N, w.n)
+                    graph = _fractions(alg, dram, N, mb, tm["us"], peak)
+                    single = _fractions(alg, dram, N, mb, tm["us_single"], peak)
+                    call(0, torch.cuda.current_stream(device))
+                    torch.cuda.synchronize(device)
+                    rows.append({"sweep": True, "N": N, "message_bytes": mb, "codec": codec,
+                                 "schedule": args.schedule, "kernel": names[0],
+                                 "us": tm["us"], "us_single": tm["us_single"], "ms": tm["us"] * 1e-3,
+                                 **graph, **{k + "_single": v for k, v in single.items()},
+                                 "algorithmic_bytes": alg, "min_dram_bytes": dram,
+                                 "rotated_sets": sets.R, "calls_per_graph": tm["calls_per_graph"],
+                                 "timing": "us: K calls over the rotated buffer sets in one CUDA graph, replay "
+                                           "time / K (inputs outside L2); us_single: one call after a 256 MiB "
+                                           "write, median of 20",
+                                 "peak": peak, "cpu_baseline": cpu[(N, codec)], "seed": w.seed,
+                                 **sample_check(xs, sets.outputs[0], sample.numpy())})
+            clk = clocks.summary()
+            for row in rows:
+                row["clocks"] = clk
+                line = json.dumps(row)
+                print(line, flush=True)
                 if sink:
-                    sink.write(row + "\n")
+                    sink.write(line + "\n")
                     sink.flush()
-            del xs, outs, ws, flush
+            del xs, sets
             torch.cuda.empty_cache()
+
+
+def run_floor(args, device):
+    """Small messages against the per-call floor: the same call with a one-tile
+    BF16 message on one rank (one tiny kernel through lpar_allreduce), then the
+    all-reduce of 128 KiB - 2 MiB per rank; each timed single (cold) and back to
+    back (CUDA graph), and back to back from Python (eager enqueue)."""
+    from quantized_precision_all_b200 import lpar as L
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def eager(call, R, K=200):
+        for i in range(3):
+            call(i % R, stream)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(K):
+            call(k % R, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) * 1e3 / K
+
+    points = [(1, 2048 * 2, "bf16", "floor: one tile on one rank, BF16")]
+    for N in (2, 4, 8):
+        for mb in (128 << 10, 256 << 10, 512 << 10, 1 << 20, 2 << 20):
+            for codec in W.SWEEP_CODECS:
+                points.append((N, mb, codec, ""))
+    with ClockSampler(device) as clocks:
+        rows = []
+        for N, mb, codec, note in points:
+            w = W.sweep_workload(N, mb, "bf16")
+            xs = W.make_inputs(w, device)
+            wsb = L.lpar_workspace_bytes(N, w.n, codec)
+            sets = BufferSets(xs, w.n, wsb, device)
+
+            def call(i, st):
+                L.lpar_allreduce(sets.inputs[i], w.n, codec, sets.outputs[i], sets.ws[i], sets.ws_bytes,
+                                 schedule=args.schedule, stream=st)
+            tm = time_call(call, sets.R, flush, device)
+            rows.append({"floor": True, "N": N, "message_bytes": mb, "codec": codec, "note": note,
+                         "us_graph": tm["us"], "us_single": tm["us_single"], "us_eager": eager(call, sets.R),
+                         "GBps_graph": N * mb / (tm["us"] * 1e-6) / 1e9})
+            del xs, sets
+    clk = clocks.summary()
+    for row in rows:
+        row["clocks"] = clk
+        print(json.dumps(row), flush=True)
 
 
 COLL_OPS = ("reduce_scatter", "one_shot", "all_gather", "all_to_all")
@@ -543,18 +791,17 @@ def collective_bytes(op, codec, N, size):
 def run_collectives(args, device):
     """One JSON line per (op, N, message size, codec) of the standalone
     collectives and the one-shot all-reduce: GB/s (N x per-rank message bytes
-    / time) and the fraction of measured HBM peak (algorithmic bytes / time)."""
+    / time) and the fraction of measured HBM peak (algorithmic bytes / time),
+    back to back (CUDA graph over rotating buffer sets) and as a single cold
+    call, with the SM clock record of the (op, N, size) group."""
     from quantized_precision_all_b200 import lpar as L
     peak, _ = measured_peaks()
-    stream = torch.cuda.current_stream(device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    cpu = {(op, N, c): oracle_gbs(op, N, c) for op in (args.coll_op and [args.coll_op] or COLL_OPS)
-           for N in (args.coll_n and [args.coll_n] or (2, 4, 8))
-           for c in (args.coll_codec and [args.coll_codec] or W.SWEEP_CODECS)}
     ops = [args.coll_op] if args.coll_op else COLL_OPS
     ranks = [args.coll_n] if args.coll_n else (2, 4, 8)
     sizes = [args.coll_mib << 20] if args.coll_mib else COLL_SIZES_BYTES
     codecs = [args.coll_codec] if args.coll_codec else W.SWEEP_CODECS
+    cpu = {(op, N, c): oracle_gbs(op, N, c) for op in ops for N in ranks for c in codecs}
     for op in ops:
         for N in ranks:
             for mb in sizes:
@@ -562,48 +809,53 @@ def run_collectives(args, device):
                 size = msg // N if op == "all_to_all" else msg
                 w = W.Workload("collective", N=N, n=msg, dist="student_t", nu=3, seed=9, codecs=("bf16",))
                 xs = W.make_inputs(w, device)
+                if op == "all_gather":
+                    xs = [x[:size] for x in xs]
                 out_elems = N * size if op in ("all_gather", "all_to_all") else msg
-                outs = [torch.empty(out_elems, dtype=torch.bfloat16, device=device) for _ in range(N)]
-                ws = torch.empty(max(L.lpar_workspace_bytes(N, msg, c) for c in W.SWEEP_CODECS),
-                                 dtype=torch.uint8, device=device)
-
-                def call(codec):
-                    if op == "one_shot":
-                        L.lpar_allreduce(xs, msg, codec, outs, ws, ws.numel(), schedule="one_shot", stream=stream)
-                    else:
-                        src = [x[:size] for x in xs] if op == "all_gather" else xs
-                        getattr(L, "lpar_" + op)(src, size, codec, outs, ws, ws.numel(), stream=stream)
-
-                for codec in codecs:
-                    for _ in range(3):
-                        call(codec)
-                    iters = 10
-                    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                           for _ in range(iters)]
-                    for e0, e1 in evs:
-                        flush.fill_(1)
-                        e0.record(stream)
-                        call(codec)
-                        e1.record(stream)
-                    torch.cuda.synchronize(device)
-                    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
-                    alg = collective_bytes(op, codec, N, size)
-                    print(json.dumps({"collective": op, "N": N, "message_bytes": mb, "codec": codec, "ms": ms,
-                                      "GBps": N * mb / (ms * 1e-3) / 1e9,
-                                      "hbm_fraction": alg / (ms * 1e-3) / 1e9 / peak,
-                                      "algorithmic_bytes": alg, "peak": peak, "cpu_baseline": cpu[(op, N, codec)],
-                                      "l2": "256 MiB buffer rewritten before every timed call"}), flush=True)
-                del xs, outs, ws
+                wsb = max(L.lpar_workspace_bytes(N, msg, c) for c in codecs)
+                sets = BufferSets(xs, out_elems, wsb, device)
+                rows = []
+                with ClockSampler(device) as clocks:
+                    for codec in codecs:
+                        def call(i, st, codec=codec):
+                            if op == "one_shot":
+                                L.lpar_allreduce(sets.inputs[i], msg, codec, sets.outputs[i], sets.ws[i],
+                                                 sets.ws_bytes, schedule="one_shot", stream=st)
+                            else:
+                                getattr(L, "lpar_" + op)(sets.inputs[i], size, codec, sets.outputs[i], sets.ws[i],
+                                                         sets.ws_bytes, stream=st)
+                        tm = time_call(call, sets.R, flush, device, single_iters=10)
+                        alg = collective_bytes(op, codec, N, size)
+                        rows.append({"collective": op, "N": N, "message_bytes": mb, "codec": codec,
+                                     "us": tm["us"], "us_single": tm["us_single"], "ms": tm["us"] * 1e-3,
+                                     "GBps": N * mb / (tm["us"] * 1e-6) / 1e9,
+                                     "GBps_single": N * mb / (tm["us_single"] * 1e-6) / 1e9,
+                                     "hbm_fraction": alg / (tm["us"] * 1e-6) / 1e9 / peak,
+                                     "hbm_fraction_single": alg / (tm["us_single"] * 1e-6) / 1e9 / peak,
+                                     "algorithmic_bytes": alg, "peak": peak, "cpu_baseline": cpu[(op, N, codec)],
+                                     "rotated_sets": sets.R, "calls_per_graph": tm["calls_per_graph"]})
+                clk = clocks.summary()
+                for row in rows:
+                    row["clocks"] = clk
+                    print(json.dumps(row), flush=True)
+                del xs, sets
                 torch.cuda.empty_cache()
 
 
-def workload_config(w, args):
-    return {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n, "message_dtype": w.dtype,
-            "message_bytes_per_rank": w.message_bytes, "codecs": list(w.codecs), "schedule": args.schedule,
-            "distribution": w.note, "min_quant_bytes": w.min_quant_bytes,
-            "l2": "inputs %d MiB > 126 MB L2: no flush between steps" % (w.N * w.message_bytes >> 20)
-            if w.N * w.message_bytes > 126e6 else "inputs fit in L2",
-            "parallelism": "one independent instance per GPU"}
+def workload_config(w, args, world=1):
+    cfg = {"workload": w.name, "simulated_ranks": w.N, "elements_per_rank": w.n, "message_dtype": w.dtype,
+           "message_bytes_per_rank": w.message_bytes, "codecs": list(w.codecs), "schedule": args.schedule,
+           "distribution": w.note, "min_quant_bytes": w.min_quant_bytes,
+           "l2": "inputs %d MiB > 126 MB L2: no flush between steps" % (w.N * w.message_bytes >> 20)
+           if w.N * w.message_bytes > 126e6 else "inputs fit in L2",
+           "parallelism": "the %d ranks simulated in one GPU's HBM (emulated reduce-scatter / all-gather)" % w.N}
+    if world > 1:
+        cfg.update({"simulated_ranks": None, "ranks": world,
+                    "l2": "message %d MiB per rank > 126 MB L2: no flush between steps" % (w.message_bytes >> 20),
+                    "parallelism": "real all-reduce across %d GPUs, one rank per GPU: the library's stage kernels "
+                                   "with NCCL all-to-all and all-gather of the wire bytes, %d chunk(s) pipelined"
+                                   % (world, args.chunks)})
+    return cfg
 
 
 def main():
@@ -614,9 +866,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_int3_int4", choices=sorted(W.WORKLOADS))
     ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_stage", "single_pass"])
+    ap.add_argument("--chunks", type=int, default=4,
+                    help="with --gpus > 1: tile ranges pipelined through the cross-GPU all-reduce")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
+    ap.add_argument("--sweep-n", type=int, default=None, help="with --sweep: only this N")
+    ap.add_argument("--sweep-mib", type=int, default=None, help="with --sweep: only this per-rank MiB size")
+    ap.add_argument("--sweep-codec", default=None, help="with --sweep: only this codec")
     ap.add_argument("--resume", default=None,
                     help="with --sweep: append rows to this JSONL file and skip the points it already holds")
     ap.add_argument("--collectives", action="store_true",
@@ -626,8 +883,11 @@ def main():
     ap.add_argument("--coll-n", type=int, default=None, help="with --collectives: only this N")
     ap.add_argument("--coll-mib", type=int, default=None, help="with --collectives: only this per-rank MiB size")
     ap.add_argument("--coll-codec", default=None, help="with --collectives: only this codec")
+    ap.add_argument("--floor", action="store_true",
+                    help="small messages against the per-call floor, one JSON line per point")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.chunks = max(1, args.chunks)
     if args.schedule == "auto":                # what the library picks for LPAR_SCHEDULE_AUTO
         args.schedule = "single_pass"
 
@@ -648,48 +908,83 @@ def main():
     if args.collectives:
         run_collectives(args, device)
         return
+    if args.floor:
+        run_floor(args, device)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
+        try:
+            res = run_distributed(args, rank, world, device)
+            if rank == 0:
+                print(json.dumps(distributed_line(args, world, res)), flush=True)
+            torch.distributed.barrier()
+        finally:
+            torch.distributed.destroy_process_group()
+        return
     res = run_ours(args, rank, world, device)
+    print(json.dumps(emulation_line(args, res)), flush=True)
+
+
+def distributed_line(args, world, res):
     w = res["w"]
-    if rank == 0:
-        peak, peak_src = measured_peaks()
-        step_bytes = w.N * w.message_bytes * len(w.codecs)
-        ms_per_step = res["ms"] / args.steps
-        value = aggregate_gbs(world, step_bytes, args.steps, res["ms"])
-        kern = res["kern"]
-        dom = max(kern, key=lambda k: kern[k]["ms_total"])
-        total_ms = sum(d["ms_total"] for d in kern.values())
-        alg_step = sum(d["algorithmic_bytes"] * d["launches"] for d in kern.values()) / (
-            max(d["launches"] for d in kern.values()))
-        d = kern[dom]
-        traffic = traffic_for(dom, w.name)
-        line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(w, args),
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": d["achieved_gbs"], "peak": peak,
-                         "unit": "GB/s", "frac": d["achieved_gbs"] / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": d["algorithmic_bytes"],
-                         "ms_per_launch": d["ms_per_launch"], "share_of_step": d["ms_total"] / total_ms,
-                         "peak_source": peak_src},
-            "step_hbm_fraction": alg_step / (ms_per_step * 1e-3) / 1e9 / peak,
-            "kernels": {k: {"ms_per_launch": v["ms_per_launch"], "achieved_gbs": v["achieved_gbs"],
-                            "frac": v["achieved_gbs"] / peak, "share": v["ms_total"] / total_ms,
-                            "algorithmic_bytes": v["algorithmic_bytes"]} for k, v in kern.items()},
-            "gpu_launches": res["launches_per_step"] * args.steps,
-            "clocks": res["clocks"],
-            "e2e": res["e2e"],
-            "cpu_baseline": res["cpu"],
-            "accuracy": res["accuracy"],
-            "source_sha": source_sha(),
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    ms_per_step = res["ms"] / args.steps
+    achieved = res["sent"] / (ms_per_step * 1e-3) / 1e9
+    return {
+        "metric": METRIC, "value": aggregate_gbs(world, w.message_bytes * len(w.codecs), args.steps, res["ms"]),
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, args, world),
+        "roofline": {"bound": "nvlink", "kernel": "whole step (stage kernels and NCCL exchanges)",
+                     "achieved": achieved, "peak": NVLINK_GBS, "unit": "GB/s", "frac": achieved / NVLINK_GBS,
+                     "traffic": None, "algorithmic_bytes_per_step": res["sent"],
+                     "peak_source": "measured peer copy per direction per GPU on this pool (not MEASURED_PEAKS.json)"},
+        "gpu_launches": res["launches_per_step"] * args.steps, "clocks": res["clocks"], "e2e": res["e2e"],
+        "cpu_baseline": None, "source_sha": source_sha(),
+    }
+
+
+def emulation_line(args, res):
+    w = res["w"]
+    peak, peak_src = measured_peaks()
+    step_bytes = w.N * w.message_bytes * len(w.codecs)
+    ms_per_step = res["ms"] / args.steps
+    value = aggregate_gbs(1, step_bytes, args.steps, res["ms"])
+    kern = res["kern"]
+    dom = max(kern, key=lambda k: kern[k]["ms_total"])
+    total_ms = sum(d["ms_total"] for d in kern.values())
+    alg_step = sum(d["algorithmic_bytes"] * d["launches"] for d in kern.values()) / (
+        max(d["launches"] for d in kern.values()))
+    d = kern[dom]
+    traffic = traffic_for(dom, w.name)
+    sec = d["ms_per_launch"] * 1e-3
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(w, args),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": d["achieved_gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": d["achieved_gbs"] / peak, "traffic": traffic,
+                     "frac_dram": None if traffic is None else traffic / sec / 1e9 / peak,
+                     "frac_min_dram": d["min_dram_bytes"] / sec / 1e9 / peak,
+                     "algorithmic_bytes_per_launch": d["algorithmic_bytes"],
+                     "min_dram_bytes_per_launch": d["min_dram_bytes"],
+                     "ms_per_launch": d["ms_per_launch"], "share_of_step": d["ms_total"] / total_ms,
+                     "peak_source": peak_src,
+                     "basis": "frac: the schedule's algorithmic bytes (stage-1 wires written and read back); "
+                              "frac_dram: ncu DRAM bytes per launch (null unless captured on these sources); "
+                              "frac_min_dram: the fewest DRAM bytes a call can move (wire read-back from L2)"},
+        "step_hbm_fraction": alg_step / (ms_per_step * 1e-3) / 1e9 / peak,
+        "kernels": {k: {"ms_per_launch": v["ms_per_launch"], "achieved_gbs": v["achieved_gbs"],
+                        "frac": v["achieved_gbs"] / peak, "share": v["ms_total"] / total_ms,
+                        "algorithmic_bytes": v["algorithmic_bytes"]} for k, v in kern.items()},
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "clocks": res["clocks"],
+        "e2e": res["e2e"],
+        "cpu_baseline": res["cpu"],
+        "accuracy": res["accuracy"],
+        "source_sha": source_sha(),
+    }
 
 
 if __name__ == "__main__":

@@ -251,14 +251,18 @@ lpar_status_t lpar_allreduce_f32(const void *const *inputs, int N, size_t n, lpa
  * device memory, or a loop held to a fixed memory budget).  The pages have no
  * counterpart: this is a deployment convenience, not part of the method.
  * Inputs, outputs, options and stream are as for lpar_allreduce; the workspace
- * is a 16 MiB array reserved inside the library on every device that loads it
- * and held until the process exits.  Returns LPAR_ERR_WORKSPACE_TOO_SMALL when
- * lpar_workspace_bytes(N, n, effective codec) exceeds
- * LPAR_STATIC_WORKSPACE_BYTES (e.g. INT3 with N = 2 up to n = 12.8 Mi), and
- * never calls cudaMalloc/cudaFree.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and caches it: make that call
- * before any stream capture.  All calls share the one array: calls whose work
- * overlaps on the GPU race on it and must be serialised by the caller. */
+ * is a 16 MiB array inside the library, reserved on a device when the
+ * library's code is loaded there (with CUDA's lazy module loading, no later
+ * than the first call on that device) and held until the process exits.
+ * Returns LPAR_ERR_WORKSPACE_TOO_SMALL when lpar_workspace_bytes(N, n,
+ * effective codec) exceeds LPAR_STATIC_WORKSPACE_BYTES (e.g. INT3 with N = 2
+ * up to n = 12.8 Mi), and never calls cudaMalloc/cudaFree.  The first call in
+ * a device context looks up the array's device address (cudaGetSymbolAddress)
+ * and caches it with that context; a call in another context (another context
+ * on the device, or the new primary context after cudaDeviceReset) looks it up
+ * again.  Make the first call before any stream capture.  All calls share the
+ * one array: calls whose work overlaps on the GPU race on it and must be
+ * serialised by the caller. */
 lpar_status_t lpar_allreduce_static(const void *const *inputs, int N, size_t n, lpar_codec_t codec,
                                     void *const *out, const lpar_options_t *opts, cudaStream_t stream);
 
@@ -291,8 +295,11 @@ size_t lpar_host_staging_bytes(int N, size_t chunk, lpar_codec_t codec);
  * effective codec) bytes of device memory, 16-byte aligned, owned by the
  * caller.  The work is ordered after earlier work on `stream`, and later work
  * on `stream` runs after the last result has reached host memory; the call
- * returns once everything is enqueued.  Not for stream capture (the library
- * creates and releases its streams inside the call).  Argument errors are
+ * returns once everything is enqueued.  The copies and kernels run on three
+ * streams of the library's own, created on a device's first call (in the
+ * current context, normally the primary one) and kept until the process
+ * exits; calls from several host threads are serialised while they enqueue.
+ * Not for stream capture.  Argument errors are
  * returned before anything is enqueued; after an error returned once copies
  * or kernels were enqueued, later work on `stream` still runs after them, so
  * the buffers may be released once `stream` has passed the call. */

@@ -15,12 +15,18 @@
 // chunk k - 1 run at the same time: with page-locked host buffers the time is
 // bound by the slower PCIe direction instead of the sum of both.  The
 // threshold is decided once, on the whole message, and every chunk runs with
-// the codec it selects.  The streams and events are created per call and
-// released when their work is done; the library keeps nothing.
+// the codec it selects.  The three streams and their events are created on a
+// device's first call and kept for the life of the process (one set per
+// device, in the device's primary context); a per-device lock makes each
+// call's enqueue complete before another thread's begins, so concurrent
+// callers never interleave their event records.  Every call starts after
+// the work already on the caller's stream and ends by making that stream wait
+// for all of its own work.
 #include "lpar.h"
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <mutex>
 #include <nvtx3/nvToolsExt.h>
 
 #define LPAR_API extern "C" __attribute__((visibility("default")))
@@ -59,19 +65,24 @@ struct Pipeline {
             ok = ok && cudaEventCreateWithFlags(&down[k], cudaEventDisableTiming) == cudaSuccess;
         }
     }
-    // Destroying a stream or an event with work pending returns at once; the
-    // resources are released when the work completes.
-    ~Pipeline() {
-        for (auto &s : st)
-            if (s) cudaStreamDestroy(s);
-        if (start) cudaEventDestroy(start);
-        for (int k = 0; k < kSlots; ++k) {
-            if (up[k]) cudaEventDestroy(up[k]);
-            if (comp[k]) cudaEventDestroy(comp[k]);
-            if (down[k]) cudaEventDestroy(down[k]);
-        }
-    }
 };
+
+constexpr int kMaxDevices = 64;
+
+// The current device's pipeline and its lock; created on first use and never
+// destroyed (the process's exit releases them).  Null when the device cannot
+// be queried or the streams cannot be created.
+struct DevicePipeline {
+    std::mutex lock;
+    Pipeline *p = nullptr;
+};
+
+DevicePipeline *device_pipeline() {
+    static DevicePipeline per_device[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    return &per_device[dev];
+}
 
 // Device bytes of the pipeline: three slots of N chunks of `elem` bytes per
 // element, then the workspace `ws` of one chunk.
@@ -93,8 +104,15 @@ lpar_status_t host_pipeline(const void *const *host_inputs, int N, size_t n, voi
     uint8_t *const ws = base + (size_t)kSlots * N * cb;
     const size_t ws_bytes = device_bytes - (size_t)kSlots * N * cb;
 
-    Pipeline p;
-    if (!p.ok) return LPAR_ERR_CUDA;
+    DevicePipeline *dp = device_pipeline();
+    if (!dp) return LPAR_ERR_CUDA;
+    std::lock_guard<std::mutex> held(dp->lock);
+    if (!dp->p) {
+        Pipeline *fresh = new Pipeline();
+        if (!fresh->ok) return LPAR_ERR_CUDA;      // a failed set is dropped, not released
+        dp->p = fresh;
+    }
+    Pipeline &p = *dp->p;
     cudaStream_t up = p.st[0], comp = p.st[1], down = p.st[2];
     if (opts && opts->stage_events[0]) cudaEventRecord(opts->stage_events[0], stream);
     if (cudaEventRecord(p.start, stream) != cudaSuccess) return LPAR_ERR_CUDA;

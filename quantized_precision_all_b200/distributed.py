@@ -4,27 +4,36 @@ This is the two-shot schedule of the single-GPU emulation with the exchange
 steps made real ("RCCLX: Innovating GPU communications on AMD platforms",
 Direct Data Access: the tree all-reduce is a reduce-scatter followed by an
 all-gather; Low-Precision Collectives: the quantised wire is what crosses the
-links, compute stays in FP32):
+links, compute stays in FP32).  For each chunk of the message (a range of
+whole tiles; tiles are independent, so chunking changes no result):
 
-  1. every rank quantises its message into its wire (``lpar_quantize``);
-  2. all-to-all of wire shards: rank j receives shard j (tiles
-     [jT/N, (j+1)T/N), the same floor partition as the emulation) of every
-     rank's wire, in rank order;
+  1. every rank quantises its chunk into its wire (``lpar_quantize``);
+  2. all-to-all of wire shards: rank j receives shard j of the chunk (tiles
+     [jT/N, (j+1)T/N) of its T tiles, the emulation's floor partition) of
+     every rank's wire, in rank order;
   3. rank j reduces its shard from the N received wires and requantises it
-     (``lpar_reduce``: FP32 sum in ascending rank order from +0.0f), straight
-     into its slot of the all-gather buffer;
-  4. all-gather of the requantised shards into one buffer (slots padded to the
-     largest shard);
+     (``lpar_reduce``: FP32 sum in ascending rank order from +0.0f) into its
+     send slot;
+  4. all-gather of the requantised shards into one buffer (slots padded to
+     the largest shard);
   5. every rank decodes each shard from its slot into its place of the output
      (``lpar_decode``): no concatenation or other copy of the gathered wire.
 
-The result is bit-identical to ``lpar_allreduce`` on the N messages in one GPU.
-The exchanges use ``torch.distributed`` collectives on the wire bytes (NCCL on
-GPUs); the arithmetic runs in the library's kernels.  The stage functions are
-an argument so that the host orchestration can be exercised on its own.
+The exchanges of chunk k are issued asynchronously, so with NCCL they run on
+its own stream while the kernels of chunk k + 1 run on the compute stream:
+the all-to-all of chunk k overlaps the quantisation of chunk k + 1, and the
+all-gather of chunk k the reduction of chunk k + 1.
+
+The result is bit-identical to ``lpar_allreduce`` on the N messages in one
+GPU.  The exchanges use ``torch.distributed`` collectives on the wire bytes;
+the arithmetic runs in the library's kernels.  Buffers are allocated once per
+(message size, codec, device) and reused by later calls.  With a process group
+that cannot move device memory (gloo), the wire bytes travel through host
+copies of the exchange buffers.  The stage functions are an argument so that
+the host orchestration can also be exercised with other implementations.
 """
 from dataclasses import dataclass
-from typing import Callable, List, Optional
+from typing import Callable, Dict, List, Optional, Tuple
 
 import torch
 import torch.distributed as dist
@@ -36,21 +45,20 @@ TILE_ELEMS = L.TILE_ELEMS
 
 @dataclass
 class Stages:
-    """quantize(x, codec) -> wire; reduce(wires, tiles, codec, out) writes the
-    reduced wire of `tiles` tiles into `out`; decode(wire, n, codec, out) writes
-    n BF16 values into `out`; tile_bytes(codec)."""
+    """quantize(x, codec, wire) writes x's wire into `wire`; reduce(wires,
+    tiles, codec, out) writes the reduced wire of `tiles` tiles into `out`;
+    decode(wire, n, codec, out) writes n BF16 values into `out`;
+    tile_bytes(codec)."""
     quantize: Callable
     reduce: Callable
     decode: Callable
     tile_bytes: Callable
 
 
-def cuda_stages(stream: Optional[torch.cuda.Stream] = None) -> Stages:
+def cuda_stages(stream=None) -> Stages:
     """The library's kernels on the current device (the product path)."""
-    def quantize(x, codec):
-        wire = torch.empty(L.lpar_wire_bytes(codec, x.numel()), dtype=torch.uint8, device=x.device)
+    def quantize(x, codec, wire):
         L.lpar_quantize(x, x.numel(), codec, wire, stream)
-        return wire
 
     def reduce(wires, tiles, codec, out):
         if tiles:
@@ -62,19 +70,101 @@ def cuda_stages(stream: Optional[torch.cuda.Stream] = None) -> Stages:
     return Stages(quantize, reduce, decode, L.lpar_tile_bytes)
 
 
-def shard_tiles(N: int, T: int) -> List[tuple]:
+def shard_tiles(N: int, T: int) -> List[Tuple[int, int]]:
     """Tile range [t0, t1) of shard j, j = 0..N-1 (floor partition)."""
     return [(j * T // N, (j + 1) * T // N) for j in range(N)]
 
 
-class DistributedAllreduce:
-    """All-reduce of one BF16 tensor per process across a process group."""
+def chunk_tiles(T: int, chunks: int) -> List[Tuple[int, int]]:
+    """The message's tiles split into at most `chunks` contiguous ranges."""
+    k = max(1, min(chunks, T))
+    return [(c * T // k, (c + 1) * T // k) for c in range(k)]
 
-    def __init__(self, group=None, stages: Optional[Stages] = None):
+
+class _Buffers:
+    """Exchange buffers of one (tiles per chunk, codec, device): the rank's
+    wire, the received shards, the send slot and the gathered slots, one set per
+    chunk in flight; plus host copies when the group moves host memory only."""
+
+    def __init__(self, N, me, chunk_ranges, tb, device, host):
+        self.plans = []
+        for t0, t1 in chunk_ranges:
+            T = t1 - t0
+            shards = shard_tiles(N, T)
+            mine = shards[me][1] - shards[me][0]
+            width = max(b - a for a, b in shards) * tb
+            plan = {
+                "T": T, "shards": shards, "mine": mine, "width": width,
+                "wire": torch.empty(T * tb, dtype=torch.uint8, device=device),
+                "recv": torch.empty(N * mine * tb, dtype=torch.uint8, device=device),
+                "send": torch.empty(width, dtype=torch.uint8, device=device),
+                "gathered": torch.empty(N * width, dtype=torch.uint8, device=device),
+            }
+            if host:
+                for k in ("wire", "recv", "send", "gathered"):
+                    plan["h_" + k] = torch.empty(plan[k].numel(), dtype=torch.uint8,
+                                                 pin_memory=torch.cuda.is_available() and device.type == "cuda")
+            self.plans.append(plan)
+
+
+class DistributedAllreduce:
+    """All-reduce of one BF16 tensor per process across a process group.
+
+    chunks: the message is processed in up to this many tile ranges, so that
+    the exchange of one overlaps the kernels of the next.  exchange_on_host:
+    route the wire bytes through host buffers (default: when the group's
+    backend is gloo and the data lives on a GPU)."""
+
+    def __init__(self, group=None, stages: Optional[Stages] = None, chunks: int = 1,
+                 exchange_on_host: Optional[bool] = None):
         self.group = group
         self.N = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.stages = stages if stages is not None else cuda_stages()
+        self.chunks = max(1, int(chunks))
+        self.exchange_on_host = exchange_on_host
+        self._cache: Dict[tuple, _Buffers] = {}
+
+    def _host(self, device) -> bool:
+        if self.exchange_on_host is not None:
+            return bool(self.exchange_on_host)
+        return device.type == "cuda" and dist.get_backend(self.group) == "gloo"
+
+    def buffers(self, n: int, codec: str, device) -> _Buffers:
+        key = (n, codec, str(device))
+        b = self._cache.get(key)
+        if b is None:
+            T = n // TILE_ELEMS
+            b = _Buffers(self.N, self.rank, chunk_tiles(T, self.chunks), self.stages.tile_bytes(codec), device,
+                         self._host(device))
+            self._cache[key] = b
+        return b
+
+    def release(self):
+        """Drop the cached exchange buffers."""
+        self._cache.clear()
+
+    # -- the two exchanges, on device buffers or through their host copies ----
+    def _all_to_all(self, p, tb, host):
+        N, mine = self.N, p["mine"]
+        in_splits = [(t1 - t0) * tb for t0, t1 in p["shards"]]
+        out_splits = [mine * tb] * N
+        if host:
+            p["h_wire"].copy_(p["wire"])
+            dist.all_to_all_single(p["h_recv"], p["h_wire"], output_split_sizes=out_splits,
+                                   input_split_sizes=in_splits, group=self.group)
+            p["recv"].copy_(p["h_recv"])
+            return None
+        return dist.all_to_all_single(p["recv"], p["wire"], output_split_sizes=out_splits,
+                                      input_split_sizes=in_splits, group=self.group, async_op=True)
+
+    def _all_gather(self, p, host):
+        if host:
+            p["h_send"].copy_(p["send"])
+            dist.all_gather_into_tensor(p["h_gathered"], p["h_send"], group=self.group)
+            p["gathered"].copy_(p["h_gathered"])
+            return None
+        return dist.all_gather_into_tensor(p["gathered"], p["send"], group=self.group, async_op=True)
 
     def allreduce(self, x: torch.Tensor, codec: str, min_quant_bytes: int = 0,
                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -83,31 +173,32 @@ class DistributedAllreduce:
             raise ValueError("the message must be a whole number of 2048-element tiles")
         if codec != "bf16" and 2 * n < min_quant_bytes:
             codec = "bf16"                                  # the threshold on the per-rank message
-        N, me, st = self.N, self.rank, self.stages
-        T = n // TILE_ELEMS
-        tb = st.tile_bytes(codec)
-        shards = shard_tiles(N, T)
-        wire = st.quantize(x, codec)                        # 1. stage 1
-        # 2. all-to-all: my shard's tiles from every rank, in rank order
-        send_sizes = [(t1 - t0) * tb for t0, t1 in shards]
-        my_tiles = shards[me][1] - shards[me][0]
-        recv = torch.empty(N * my_tiles * tb, dtype=torch.uint8, device=wire.device)
-        dist.all_to_all_single(recv, wire, output_split_sizes=[my_tiles * tb] * N,
-                               input_split_sizes=send_sizes, group=self.group)
-        received = [recv[r * my_tiles * tb:(r + 1) * my_tiles * tb] for r in range(N)]
-        # 3. stage 2 of my shard, straight into my slot of the all-gather (padded
-        #    to the largest shard; the padding is never decoded)
-        width = max(t1 - t0 for t0, t1 in shards) * tb
-        send = torch.empty(width, dtype=torch.uint8, device=wire.device)
-        st.reduce(received, my_tiles, codec, send[:my_tiles * tb])
-        # 4. all-gather of the shards into one buffer, rank j's slot at j * width
-        gathered = torch.empty(N * width, dtype=torch.uint8, device=wire.device)
-        dist.all_gather(list(gathered.view(N, width).unbind(0)), send, group=self.group)
-        # 5. stage 3: each shard decoded from its slot into its place of the output
         if out is None:
             out = torch.empty(n, dtype=torch.bfloat16, device=x.device)
-        for j, (t0, t1) in enumerate(shards):
-            if t1 > t0:
-                st.decode(gathered[j * width:j * width + (t1 - t0) * tb], (t1 - t0) * TILE_ELEMS, codec,
-                          out[t0 * TILE_ELEMS:t1 * TILE_ELEMS])
+        if n == 0:
+            return out
+        st, tb = self.stages, self.stages.tile_bytes(codec)
+        bufs = self.buffers(n, codec, x.device)
+        host = self._host(x.device)
+        ranges = chunk_tiles(n // TILE_ELEMS, self.chunks)
+        a2a = []
+        for (t0, t1), p in zip(ranges, bufs.plans):         # 1. stage 1, then 2. its all-to-all
+            st.quantize(x[t0 * TILE_ELEMS:t1 * TILE_ELEMS], codec, p["wire"])
+            a2a.append(self._all_to_all(p, tb, host))
+        ag = []
+        for h, p in zip(a2a, bufs.plans):                    # 3. stage 2 of my shard, 4. all-gather
+            if h is not None:
+                h.wait()
+            mine = p["mine"]
+            received = [p["recv"][r * mine * tb:(r + 1) * mine * tb] for r in range(self.N)]
+            st.reduce(received, mine, codec, p["send"][:mine * tb])
+            ag.append(self._all_gather(p, host))
+        for (t0, t1), h, p in zip(ranges, ag, bufs.plans):   # 5. stage 3 of every shard
+            if h is not None:
+                h.wait()
+            w = p["width"]
+            for j, (s0, s1) in enumerate(p["shards"]):
+                if s1 > s0:
+                    a, b = (t0 + s0) * TILE_ELEMS, (t0 + s1) * TILE_ELEMS
+                    st.decode(p["gathered"][j * w:j * w + (s1 - s0) * tb], b - a, codec, out[a:b])
         return out

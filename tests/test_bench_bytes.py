@@ -1,10 +1,9 @@
 """bench.py's byte model on the host (no GPU): the algorithmic bytes behind every
 roofline fraction, checked against the per-element model they come from (stage-1
-wires written and read back, one gathered wire, N outputs), against the figures
-quoted in profiles/, and the kernel labels against the library's choice of form."""
+wires written and read back, one gathered wire, N outputs), and the kernel labels
+against the library's choice of form."""
 import os
 import random
-import re
 import sys
 
 import pytest
@@ -53,17 +52,12 @@ def test_binary32_bytes():
     assert bench.algorithmic_bytes("k_f32_reduce<N=8>", "bf16", N, n) == n * (8 * N + 4)
 
 
-def test_profiles_quote_the_model():
-    """The algorithmic bytes printed in profiles/dram_traffic.txt are the model's."""
-    text = open(os.path.join(ROOT, "profiles", "dram_traffic.txt")).read()
+def test_bench_workload_bytes():
+    """The per-launch algorithmic bytes of the default bench workload (N = 2 x 512 Mi)."""
     n = 512 * 1024 * 1024
-    assert "5469372416" in text and "5804916736" in text and "5721030656" in text
     assert bench.algorithmic_bytes("k_allreduce_single_warp<int3,N=2>", "int3", 2, n) == 5469372416
     assert bench.algorithmic_bytes("k_allreduce_single<int4,N=2>", "int4", 2, n) == 5804916736
     assert bench.algorithmic_bytes("k_allreduce_single<mxfp4,N=2>", "mxfp4", 2, n) == 5721030656
-    for line in re.findall(r"^kernel=.*$", text, re.M):
-        kv = dict(f.split("=", 1) for f in line.split())
-        assert int(kv["bytes_per_launch"]) == int(kv["read"]) + int(kv["write"])
 
 
 def test_collective_bytes():

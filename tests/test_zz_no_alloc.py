@@ -3,7 +3,9 @@ memory (for example a plugin whose host application owns all device memory),
 using the workspace the library keeps for itself.
 
 Its results must equal those of lpar_allreduce with a caller-provided workspace,
-on two calls in a row (the shared workspace keeps the previous call's contents).
+on two calls in a row (the shared workspace keeps the previous call's contents),
+and once a first call has run on the device, later calls must leave the
+device's free memory unchanged.
 This file is named to be collected last, and must pass both alone in a fresh
 process and after the other tests.
 """
@@ -37,6 +39,20 @@ def test_static_workspace_equals_caller_workspace_on_two_calls(L, codec, N):
         torch.cuda.synchronize()
         for o, r in zip(out, ref_out):
             assert torch.equal(o.view(torch.int16), r.view(torch.int16)), (codec, call)
+
+
+def test_static_calls_allocate_nothing(L):
+    N, n = 4, 2048 * 200
+    xs = [torch.randn(n, device="cuda").to(torch.bfloat16) for _ in range(N)]
+    out = [torch.empty_like(x) for x in xs]
+    L.lpar_allreduce_static(xs, n, "int4", out)          # the first call may load the library's module
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for codec in ("int4", "int3", "fp8", "mxfp4", "bf16", "int4"):
+        L.lpar_allreduce_static(xs, n, codec, out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_static_workspace_rejects_messages_beyond_its_size(L):

@@ -128,6 +128,14 @@ def make_inputs(w: Workload, device="cpu", n: Optional[int] = None) -> List[torc
     return [_draw_f32(w, r, n, device).to(torch.bfloat16) for r in range(w.N)]
 
 
+def make_rank_input(w: Workload, r: int, device="cpu", n: Optional[int] = None) -> torch.Tensor:
+    """Rank r's message alone (the same values as ``make_inputs(w)[r]``; r may
+    exceed w.N when the ranks are real processes)."""
+    n = w.n if n is None else n
+    x = _draw_f32(w, r, n, device)
+    return x if w.dtype == "f32" else x.to(torch.bfloat16)
+
+
 def bf16_bits(t: torch.Tensor):
     """BF16 tensor -> numpy uint16 bit patterns on the host."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view("uint16")
