@@ -79,14 +79,20 @@ def measured_peaks():
 
 # ---- algorithmic bytes per launch (reads + writes the definition requires) ------
 # The library's choice of the single-pass kernel form (lpar_kernels.cu,
-# launch_single_cn): warp-local for INT3 with N <= 2 or below 512 MiB of input
+# launch_single_cn): the rank-parallel tile form up to 256 tiles per rank (512
+# for FP8); above, warp-local for INT3 with N <= 2 or below 512 MiB of input
 # and for INT4 / MXFP4 below 128 MiB of input, CTA-wide otherwise and for FP8.
 BULK_MIN_BYTES = 128 << 20
 INT3_WARP_MAX_BYTES = 512 << 20
 
 
+TILE_FORM_MAX_TILES = {"fp8": 512}           # others: 256
+
+
 def single_pass_kernel(codec, N, n):
     in_bytes = N * 2 * n
+    if n // TILE <= TILE_FORM_MAX_TILES.get(codec, 256):
+        return "k_allreduce_tile<%s,N=%d>" % (codec, N)
     if codec == "fp8":
         warp = False
     elif codec == "int3":
@@ -116,7 +122,7 @@ def algorithmic_bytes(kernel, codec, N, n):
         return N * n * (4 + c) + n * (N * c + c + 4 * N)
     if kernel.startswith("k_f32_reduce"):
         return n * (4 * N + 4 + 4 * N)
-    if kernel.startswith("k_allreduce_single"):
+    if kernel.startswith("k_allreduce_single") or kernel.startswith("k_allreduce_tile"):
         # N BF16 messages in, N wires out and back in, gathered wire out, N outputs out
         return N * n * (2 + c) + n * (N * c + c + 2 * N)
     if kernel.startswith("k_quantize"):
@@ -153,7 +159,7 @@ def min_dram_for(kernel, codec, N, n):
     c = CODEC_C[codec]
     if kernel.startswith("k_allreduce_single_f32"):
         return N * n * (4 + c) + n * c + 4 * N * n
-    if kernel.startswith("k_allreduce_single"):
+    if kernel.startswith("k_allreduce_single") or kernel.startswith("k_allreduce_tile"):
         return min_dram_bytes(codec, N, n)
     return algorithmic_bytes(kernel, codec, N, n)
 
@@ -176,6 +182,8 @@ def max_over_ranks(ms, world, device):
     """The slowest rank's time: every rank contributes, all receive the max."""
     if world <= 1:
         return float(ms)
+    if torch.distributed.get_backend() == "gloo":
+        device = torch.device("cpu")                  # gloo reduces host tensors
     t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
@@ -853,8 +861,8 @@ def workload_config(w, args, world=1):
         cfg.update({"simulated_ranks": None, "ranks": world,
                     "l2": "message %d MiB per rank > 126 MB L2: no flush between steps" % (w.message_bytes >> 20),
                     "parallelism": "real all-reduce across %d GPUs, one rank per GPU: the library's stage kernels "
-                                   "with NCCL all-to-all and all-gather of the wire bytes, %d chunk(s) pipelined"
-                                   % (world, args.chunks)})
+                                   "with %s all-to-all and all-gather of the wire bytes, %d chunk(s) pipelined"
+                                   % (world, args.backend.upper(), args.chunks)})
     return cfg
 
 
@@ -868,6 +876,9 @@ def main():
     ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_stage", "single_pass"])
     ap.add_argument("--chunks", type=int, default=4,
                     help="with --gpus > 1: tile ranges pipelined through the cross-GPU all-reduce")
+    ap.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
+                    help="with --gpus > 1: the process group's backend (gloo moves the wire bytes through host "
+                         "copies; for testing the multi-rank path on fewer GPUs than ranks)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point instead of the bench line")
@@ -900,7 +911,7 @@ def main():
             print(json.dumps(run_reference(args)), flush=True)
         return
 
-    device = torch.device("cuda", local_rank)
+    device = torch.device("cuda", local_rank % max(1, torch.cuda.device_count()))
     torch.cuda.set_device(device)
     if args.sweep:
         run_sweep(args, device)
@@ -913,8 +924,11 @@ def main():
         return
     if world > 1:
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+        if args.backend == "nccl":
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=device)
+        else:
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
         try:
             res = run_distributed(args, rank, world, device)
             if rank == 0:

@@ -199,6 +199,60 @@ __global__ void __launch_bounds__(kThreads, 4) k_reduce_bf16_warp(const __grid_c
     }
 }
 
+// The rank-parallel tile form of the reductions (small messages; see
+// k_allreduce_tile): one tile per CTA, the N ranks' tiles copied into shared
+// memory and their N x 64 block encodes spread over the threads; after one
+// barrier threads 0..63 read back the N wire blocks of their block, sum them in
+// rank order from +0.0f and round once to BF16 into rank 0's region, which all
+// threads store to the shard owner (ALL = false) or to every rank.
+template <int C, int N, bool ALL>
+__global__ void __launch_bounds__(kThreads) k_reduce_bf16_tile(const __grid_constant__ InPtrs in,
+                                                               const __grid_constant__ OutPtrs wire,
+                                                               const __grid_constant__ OutPtrs out, size_t tiles) {
+    constexpr int kTileBytesBf16 = kTileElems * 2;
+    __shared__ __align__(128) uint8_t stage[N * kTileBytesBf16];
+    const int t = threadIdx.x;
+    const size_t tile = blockIdx.x;
+#pragma unroll
+    for (int r = 0; r < N; ++r)
+        cp_async16(stage + r * kTileBytesBf16 + swz(t >> 2, t & 3), in.p[r] + tile * kTileBytesBf16 + 16 * t);
+    cp_async_commit();
+    cp_async_wait_all_groups();
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < (N + 3) / 4; ++k) {
+        const int idx = t + kThreads * k, r = idx >> 6, b = idx & 63;
+        if (r < N)
+            quantize_staged_block<C, false>(stage + r * kTileBytesBf16, wire.p[r] + tile * Layout<C>::kTileBytes, b,
+                                            NoSink{});
+    }
+    __syncthreads();                                             // wire blocks visible; rank 0's region free
+    if (t < kBlocksPerTile) {
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.0f;              // +0.0f, then ranks in ascending order
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            Packed<C> p;
+            load_block(wire.p[r] + tile * Layout<C>::kTileBytes, t, p);
+            accumulate<C>(p, acc);
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = pack_bf16x2(acc[2 * k], acc[2 * k + 1]);
+        stage_write(stage, t, o);
+    }
+    __syncthreads();
+    const uint4 d = *reinterpret_cast<const uint4 *>(stage + swz(t >> 2, t & 3));
+    if (ALL) {
+#pragma unroll
+        for (int r = 0; r < N; ++r) *reinterpret_cast<uint4 *>(out.p[r] + tile * kTileBytesBf16 + 16 * t) = d;
+    } else {
+        const int j = shard_of(tile, tiles, N);
+        *reinterpret_cast<uint4 *>(out.p[j] + (tile - shard_begin(j, tiles, N)) * kTileBytesBf16 + 16 * t) = d;
+    }
+}
+
 // BF16 passthrough of the reductions: one tile (256 x 16 B) per CTA step, the
 // FP32 sum in rank order rounded once.  The shard owner advances with the
 // tile index (tiles are visited in increasing order), so no division per tile.
@@ -359,7 +413,8 @@ static inline unsigned persistent_grid(unsigned chunks, unsigned resident) {
 }
 
 // Which form of the reductions runs (measured on B200, the forms timed
-// alternately in one process): the warp-local form below 128 MiB of input for
+// alternately in one process): the rank-parallel tile form up to
+// kTileFormMaxTiles tiles per rank; above, the warp-local form below 128 MiB of input for
 // every codec but FP8 (5-10% faster) and, for the reduce-scatter, for INT3 at
 // every size (6-9%) and for INT4 and MXFP4 from four ranks on (8% at N = 8);
 // the CTA-wide form for FP8, for the one-shot from 128 MiB (4-9%) and for the
@@ -373,6 +428,10 @@ static inline bool rs_warp_form(int C, int N, bool ALL, size_t in_bytes) {
 
 template <int C, int N, bool ALL>
 static bool launch_rb_cna(const InPtrs &in, const OutPtrs &wire, const OutPtrs &out, size_t tiles, cudaStream_t st) {
+    if (tiles <= kTileFormMaxTiles<C>()) {
+        k_reduce_bf16_tile<C, N, ALL><<<(unsigned)tiles, kThreads, 0, st>>>(in, wire, out, tiles);
+        return true;
+    }
     const unsigned chunks = (unsigned)((tiles + kTilesPerCta - 1) / kTilesPerCta);
     if (rs_warp_form(C, N, ALL, (size_t)N * tiles * (kTileElems * 2))) {
         constexpr int smem = 3 * kStageBytes;

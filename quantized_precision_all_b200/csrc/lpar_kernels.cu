@@ -10,8 +10,10 @@
 //   K23 k_reduce<.., true>   K2 plus the decode of the gathered block straight
 //                        from registers into every rank's BF16 output
 //   K3  k_decode        gathered wire -> BF16 into every rank's output
-//   K123 all three stages in one persistent kernel (the default schedule), in
-//        two forms: k_allreduce_single_warp (warp-local, no CTA barrier) and
+//   K123 all three stages in one kernel (the default schedule), in three
+//        forms: k_allreduce_tile (one tile per CTA, the ranks' stage 1 spread
+//        over the CTA's threads: small messages), and the persistent
+//        k_allreduce_single_warp (warp-local, no CTA barrier) and
 //        k_allreduce_single (CTA-wide, output by bulk copies from 128 MiB of
 //        input); launch_single_cn picks one by codec, N and size
 // The BF16 passthrough uses k_bf16_reduce (FP32 sum, one BF16 rounding) and
@@ -290,6 +292,57 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 // ---------------------------------------------------------------------------
+// K123, rank-parallel form for small messages: one tile per CTA, the N ranks'
+// stage 1 spread over the CTA's threads.  A small message fills few CTAs of
+// the persistent forms, each encoding the N ranks of its chunk one after
+// another; here every tile has its own CTA and the N x 64 block encodes of a
+// tile run side by side (thread t encodes block t % 64 of rank t / 64, then of
+// rank t / 64 + 4), so the call's dependent chain holds one or two encodes
+// instead of N.  The CTA copies the N BF16 tiles into shared memory (one
+// swizzled 4-KiB region per rank), writes the N stage-1 wire blocks, and after
+// one barrier (which makes the CTA's global writes visible to all its threads)
+// threads 0..63 read the N wire blocks of their block back, reduce, requantise
+// into the gathered wire and decode into rank 0's region, which all threads
+// then store to every output with coalesced 16-B stores.
+// ---------------------------------------------------------------------------
+template <int C, int N>
+__global__ void __launch_bounds__(kThreads) k_allreduce_tile(const __grid_constant__ InPtrs in,
+                                                             const __grid_constant__ OutPtrs wire, uint8_t *gather,
+                                                             const __grid_constant__ OutPtrs out) {
+    constexpr int kTileBytesBf16 = kTileElems * 2;               // 4 KiB: 64 blocks of 64 B
+    __shared__ __align__(128) uint8_t stage[N * kTileBytesBf16];
+    const int t = threadIdx.x;
+    const size_t tile = blockIdx.x;
+#pragma unroll
+    for (int r = 0; r < N; ++r)                                  // piece t of every rank's tile
+        cp_async16(stage + r * kTileBytesBf16 + swz(t >> 2, t & 3), in.p[r] + tile * kTileBytesBf16 + 16 * t);
+    cp_async_commit();
+    cp_async_wait_all_groups();
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < (N + 3) / 4; ++k) {                      // stage 1: block b of rank r
+        const int idx = t + kThreads * k, r = idx >> 6, b = idx & 63;
+        if (r < N) {
+            uint32_t x16[16];
+            stage_read(stage + r * kTileBytesBf16, b, x16);
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { x[2 * j] = bf16lo(x16[j]); x[2 * j + 1] = bf16hi(x16[j]); }
+            const float a = absmax_bf16x32(x16);
+            Packed<C> p;
+            encode<C, false, false>(x, a, p, NoSink{});
+            store_block(wire.p[r] + tile * Layout<C>::kTileBytes, b, p);
+        }
+    }
+    __syncthreads();                                             // wire blocks visible; rank 0's region free
+    if (t < kBlocksPerTile) reduce_block<C, N, true>(wire.p, tile, t, gather, StageSink{stage, t});
+    __syncthreads();
+    const uint4 d = *reinterpret_cast<const uint4 *>(stage + swz(t >> 2, t & 3));
+#pragma unroll
+    for (int r = 0; r < N; ++r) *reinterpret_cast<uint4 *>(out.p[r] + tile * kTileBytesBf16 + 16 * t) = d;
+}
+
+// ---------------------------------------------------------------------------
 // K3: gathered wire -> BF16 in every out[r].  grid = ceil(tiles / 4).
 // ---------------------------------------------------------------------------
 template <int C>
@@ -444,8 +497,16 @@ static bool launch_single_warp(const InPtrs &in, const OutPtrs &wire, uint8_t *g
     return true;
 }
 
+template <int C, int N>
+static bool launch_tile(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
+                        cudaStream_t st) {
+    k_allreduce_tile<C, N><<<(unsigned)tiles, kThreads, 0, st>>>(in, wire, g, o);
+    return true;
+}
+
 // Which form of K123 runs (measured on B200, the forms timed alternately in one
-// process): the warp-local kernel for INT3 with one or two ranks at any size
+// process): the rank-parallel tile kernel up to kTileFormMaxTiles tiles per
+// rank; above that the warp-local kernel for INT3 with one or two ranks at any size
 // (7-11% faster: its encode is issue-bound and the CTA barriers cost issue
 // slots) and for INT3 below kInt3WarpMaxBytes of input, and for INT4 and MXFP4
 // below kBulkMinBytes (up to 11% faster there); the CTA-wide kernel otherwise
@@ -453,10 +514,12 @@ static bool launch_single_warp(const InPtrs &in, const OutPtrs &wire, uint8_t *g
 // always for FP8.
 constexpr size_t kInt3WarpMaxBytes = (size_t)512 << 20;
 
+
 template <int C, int N>
 static bool launch_single_cn(const InPtrs &in, const OutPtrs &wire, uint8_t *g, const OutPtrs &o, size_t tiles,
                              cudaStream_t st) {
     const size_t in_bytes = (size_t)N * tiles * (kTileElems * 2);
+    if (tiles <= kTileFormMaxTiles<C>()) return launch_tile<C, N>(in, wire, g, o, tiles, st);
     if constexpr (C == kFP8) {
         if (in_bytes >= kBulkMinBytes) return launch_single_cnb<C, N, true>(in, wire, g, o, tiles, st);
         return launch_single_cnb<C, N, false>(in, wire, g, o, tiles, st);

@@ -326,6 +326,7 @@ __device__ __forceinline__ void stage_to_outputs(const uint8_t *stage, const Out
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all_groups() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void stage_load_chunk(uint8_t *stage, const uint8_t *src, int ntiles) {
@@ -375,6 +376,15 @@ __device__ __forceinline__ void warp_to_dst(const uint8_t *stage, uint8_t *dst, 
         *reinterpret_cast<uint4 *>(dst + 16 * (size_t)q) = *reinterpret_cast<const uint4 *>(stage + swz(g >> 2, g & 3));
     }
 }
+
+// The rank-parallel tile forms (one tile per CTA, the N ranks' stage 1 spread
+// over the CTA's threads) run up to 256 tiles per rank (1 MiB of BF16), 512
+// for FP8 (measured on B200 with the forms timed alternately in one process,
+// calls back to back and single: the all-reduce 25-48% faster at 128 KiB per
+// rank for N = 2..8, 11-35% at 1 MiB; from 2 MiB per rank slower for every
+// codec but FP8, which turns at 4 MiB).
+template <int C>
+__host__ __device__ constexpr size_t kTileFormMaxTiles() { return C == kFP8 ? 512 : 256; }
 
 // ---------------------------------------------------------------------------
 // Host-side helpers.

@@ -73,13 +73,18 @@ def test_collective_bytes():
 def test_single_pass_labels_follow_the_launcher_rule():
     mib = 1 << 20
     k = bench.single_pass_kernel
+    assert k("int4", 8, 256 * 2048).startswith("k_allreduce_tile")              # 256 tiles per rank
+    assert k("int4", 2, 257 * 2048).startswith("k_allreduce_single_warp")       # 257
+    assert k("fp8", 4, 512 * 2048).startswith("k_allreduce_tile")               # FP8: up to 512 tiles
+    assert k("fp8", 4, 513 * 2048).startswith("k_allreduce_single<")
     assert k("int3", 2, 512 * mib).startswith("k_allreduce_single_warp")        # INT3, N <= 2: always
     assert k("int3", 8, 16 * mib).startswith("k_allreduce_single_warp")         # 256 MiB < 512 MiB of input
     assert k("int3", 8, 64 * mib).startswith("k_allreduce_single<")             # 1 GiB of input
     assert k("int4", 2, 16 * mib).startswith("k_allreduce_single_warp")         # 64 MiB < 128 MiB
     assert k("int4", 2, 32 * mib).startswith("k_allreduce_single<")             # 128 MiB
     assert k("mxfp4", 4, 8 * mib).startswith("k_allreduce_single_warp")
-    assert k("fp8", 2, 1024).startswith("k_allreduce_single<")                  # FP8: always CTA-wide
+    assert k("fp8", 2, 2048 * 2048).startswith("k_allreduce_single<")           # FP8 above the tile form: CTA-wide
     src = open(os.path.join(ROOT, "quantized_precision_all_b200", "csrc", "lpar_kernels.cu")).read()
     assert "kBulkMinBytes = (size_t)128 << 20" in src and "kInt3WarpMaxBytes = (size_t)512 << 20" in src
+    assert "return C == kFP8 ? 512 : 256;" in src
     assert bench.BULK_MIN_BYTES == 128 * mib and bench.INT3_WARP_MAX_BYTES == 512 * mib

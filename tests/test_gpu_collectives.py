@@ -90,6 +90,35 @@ def test_reduce_scatter_matches_oracle(L, codec, N, tiles):
         assert np.array_equal(o, r), (codec, N, j)
 
 
+# The reductions' forms around the limit of the rank-parallel tile form (256
+# tiles per rank, 512 for FP8): at it the tile form, just above it the
+# persistent forms with a ragged last chunk.
+@pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4"])
+@pytest.mark.parametrize("N", [1, 3, 8])
+@pytest.mark.parametrize("extra", [0, 1, 3])
+def test_reductions_around_the_tile_limit(L, codec, N, extra):
+    tiles = (512 if codec == "fp8" else 256) + extra
+    n = tiles * 2048
+    xs = inputs(N, n, 1500 + 10 * N + extra)
+    sizes = [(t1 - t0) * 2048 for t0, t1 in O.shard_tiles(N, tiles)]
+    outs, _ = run(L, "reduce_scatter", xs, n, codec, sizes)
+    ref, used = O.reduce_scatter(xs, codec)
+    assert used == codec
+    for j, (o, r) in enumerate(zip(outs, ref)):
+        assert np.array_equal(o, r), (codec, N, tiles, j)
+    ins = [to_device(x) for x in xs]
+    outs1 = [Guarded(2 * n, fill=0x00) for _ in range(N)]
+    ws = Guarded(L.lpar_workspace_bytes(N, n, codec))
+    L.lpar_allreduce([g.ptr() for g in ins], n, codec, [g.ptr() for g in outs1], ws.ptr(), ws.nbytes,
+                     schedule="one_shot")
+    torch.cuda.synchronize()
+    for g in ins + outs1 + [ws]:
+        g.check()
+    ref1, _ = O.allreduce_oneshot(xs, codec)
+    for o in outs1:
+        assert np.array_equal(host_u16(o), ref1[0]), (codec, N, tiles)
+
+
 @pytest.mark.parametrize("codec", CODECS)
 @pytest.mark.parametrize("N,tiles", [(1, 5), (2, 9), (3, 6), (5, 2), (8, 7)])
 def test_all_gather_matches_oracle(L, codec, N, tiles):

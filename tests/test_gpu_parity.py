@@ -473,6 +473,36 @@ def test_allreduce_matches_oracle(L, codec, N, schedule):
         assert np.array_equal(host[N * wb:(N + 1) * wb], O.reduce(wires, 0, tiles, codec))
 
 
+# The single-pass kernel's forms around the limit of the rank-parallel tile
+# form (256 tiles per rank, 512 for FP8; one tile per CTA): at and below it
+# the tile form, just above it the persistent forms with a ragged last chunk
+# (T % 4 == 1 or 3).  Adversarial and random inputs; every output and the
+# workspace (stage-1 wires, gathered wire) against the oracle.
+def tile_form_limit(codec):
+    return 512 if codec == "fp8" else 256
+
+
+@pytest.mark.parametrize("codec", QCODECS)
+@pytest.mark.parametrize("N", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("where", ["one", "three", "limit", "limit+1", "limit+3"])
+def test_single_pass_forms_around_the_tile_limit(L, codec, N, where):
+    lim = tile_form_limit(codec)
+    tiles = {"one": 1, "three": 3, "limit": lim, "limit+1": lim + 1, "limit+3": lim + 3}[where]
+    n = tiles * 2048
+    xs = [adversarial_bf16(n, 7100 + 10 * N + r) if r % 2 == 0 else random_bf16(n, 7200 + r) for r in range(N)]
+    outs, ws = run_allreduce(L, xs, codec, "auto")
+    ref, used = O.allreduce(xs, codec)
+    assert used == codec
+    for o in outs:
+        assert np.array_equal(o, ref[0]), (codec, N, tiles)
+    wb = L.lpar_wire_bytes(codec, n)
+    host = ws.host()
+    wires = [O.quantize(x, codec) for x in xs]
+    for r in range(N):
+        assert np.array_equal(host[r * wb:(r + 1) * wb], wires[r])
+    assert np.array_equal(host[N * wb:(N + 1) * wb], O.reduce(wires, 0, tiles, codec))
+
+
 # Seeded random cases over the whole argument space: codec, N in 1..8, 1..40
 # tiles, every schedule (one-shot against its own oracle), a threshold either
 # side of the message, in place or not; adversarial or random inputs per rank.
