@@ -252,7 +252,8 @@ class ClockSampler:
 
 
 # ---- our arm -------------------------------------------------------------------------
-def run_ours(args, rank, world, device):
+def run_ours(args, device):
+    """One GPU: the workload's N ranks emulated in its HBM."""
     from quantized_precision_all_b200 import lpar as L
 
     w = W.WORKLOADS[args.workload]
@@ -283,8 +284,6 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
 
     # (1) the timed region: K steps, CUDA events on the launching stream
-    if world > 1:
-        torch.distributed.barrier()
     torch.cuda.synchronize(device)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(device) as clocks:
@@ -293,9 +292,7 @@ def run_ours(args, rank, world, device):
             step()
         end.record(stream)
         torch.cuda.synchronize(device)
-    if world > 1:
-        torch.distributed.barrier()
-    ms_max = max_over_ranks(start.elapsed_time(end), world, device)
+    ms_total = start.elapsed_time(end)
 
     # (2) per-kernel durations, live: stage events recorded between the kernels
     ksteps = max(1, min(args.steps, 200))
@@ -372,27 +369,23 @@ def run_ours(args, rank, world, device):
 
         e2e_step()
         torch.cuda.synchronize(device)
-        if world > 1:
-            torch.distributed.barrier()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         for _ in range(e2e_steps):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = max_over_ranks(s0.elapsed_time(s1), world, device)
+        e_ms = s0.elapsed_time(s1)
         eb = w.elem_bytes
-        e2e = {"value": aggregate_gbs(world, N * eb * n * len(w.codecs), e2e_steps, e_ms), "unit": "GB/s",
+        e2e = {"value": aggregate_gbs(1, N * eb * n * len(w.codecs), e2e_steps, e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": N * eb * n * len(w.codecs),
                "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps, "api": api}
         del h_in, h_out
 
-    # (5) the oracle on the host cores, rank 0 at N=1 only
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, xs)
+    # (5) the oracle on the host cores (one GPU, one process)
+    cpu = None if args.no_cpu_baseline else cpu_baseline(w, xs)
 
-    return {"ms": ms_max, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
+    return {"ms": ms_total, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
             "e2e": e2e, "cpu": cpu, "w": w, "accuracy": accuracy}
 
 
@@ -937,7 +930,7 @@ def main():
         finally:
             torch.distributed.destroy_process_group()
         return
-    res = run_ours(args, rank, world, device)
+    res = run_ours(args, device)
     print(json.dumps(emulation_line(args, res)), flush=True)
 
 

@@ -106,11 +106,18 @@ def _ptr(x):
     return x.data_ptr()
 
 
+_PTR_ARRAY_TYPES = [ctypes.c_void_p * k for k in range(MAX_RANKS + 1)]
+
+
 def _ptr_array(xs, conv=None):
+    """A ctypes array of the buffers' addresses; ctypes passes it where the C
+    function takes `void *const *`."""
     if xs is None:
         return None
-    arr = (ctypes.c_void_p * len(xs))(*[(conv or _ptr)(x) for x in xs])
-    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+    conv = conv or _ptr
+    k = len(xs)
+    typ = _PTR_ARRAY_TYPES[k] if k <= MAX_RANKS else ctypes.c_void_p * k
+    return typ(*[conv(x) for x in xs])
 
 
 def _host_ptr(x):
@@ -170,7 +177,7 @@ def lpar_quantize(in_bf16, n, codec, wire, stream=None):
 
 def lpar_reduce(wires, tile_begin, tile_count, codec, wire_out, stream=None):
     arr = _ptr_array(wires)
-    _check(_lib.lpar_reduce(arr[0] if arr else None, len(wires) if wires is not None else 0, tile_begin,
+    _check(_lib.lpar_reduce(arr, len(wires) if wires is not None else 0, tile_begin,
                             tile_count, _codec(codec), _ptr(wire_out), _stream(stream)), "lpar_reduce")
 
 
@@ -184,7 +191,7 @@ def lpar_allreduce(inputs, n, codec, out, workspace, workspace_bytes, min_quant_
     outs = _ptr_array(out)
     N = len(inputs) if N is None else N
     opts = _options(min_quant_bytes, schedule, stage_events)
-    _check(_lib.lpar_allreduce(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+    _check(_lib.lpar_allreduce(ins, N, n, _codec(codec), outs,
                                _ptr(workspace), workspace_bytes, ctypes.byref(opts), _stream(stream)),
            "lpar_allreduce")
 
@@ -195,7 +202,7 @@ def lpar_allreduce_static(inputs, n, codec, out, min_quant_bytes=0, schedule="au
     outs = _ptr_array(out)
     N = len(inputs) if N is None else N
     opts = _options(min_quant_bytes, schedule)
-    _check(_lib.lpar_allreduce_static(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+    _check(_lib.lpar_allreduce_static(ins, N, n, _codec(codec), outs,
                                       ctypes.byref(opts), _stream(stream)), "lpar_allreduce_static")
 
 
@@ -206,7 +213,7 @@ def lpar_allreduce_f32(inputs, n, codec, out, workspace, workspace_bytes, min_qu
     outs = _ptr_array(out)
     N = len(inputs) if N is None else N
     opts = _options(min_quant_bytes, schedule, stage_events)
-    _check(_lib.lpar_allreduce_f32(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+    _check(_lib.lpar_allreduce_f32(ins, N, n, _codec(codec), outs,
                                    _ptr(workspace), workspace_bytes, ctypes.byref(opts), _stream(stream)),
            "lpar_allreduce_f32")
 
@@ -231,7 +238,7 @@ def lpar_allreduce_f32_host(host_inputs, n, codec, host_out, chunk, device, devi
     outs = _ptr_array(host_out, _host_ptr)
     N = len(host_inputs) if N is None else N
     opts = _options(min_quant_bytes, schedule, stage_events)
-    _check(_lib.lpar_allreduce_f32_host(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None,
+    _check(_lib.lpar_allreduce_f32_host(ins, N, n, _codec(codec), outs,
                                         chunk, _ptr(device), device_bytes, ctypes.byref(opts), _stream(stream)),
            "lpar_allreduce_f32_host")
 
@@ -244,7 +251,7 @@ def lpar_allreduce_host(host_inputs, n, codec, host_out, chunk, device, device_b
     outs = _ptr_array(host_out, _host_ptr)
     N = len(host_inputs) if N is None else N
     opts = _options(min_quant_bytes, schedule, stage_events)
-    _check(_lib.lpar_allreduce_host(ins[0] if ins else None, N, n, _codec(codec), outs[0] if outs else None, chunk,
+    _check(_lib.lpar_allreduce_host(ins, N, n, _codec(codec), outs, chunk,
                                     _ptr(device), device_bytes, ctypes.byref(opts), _stream(stream)),
            "lpar_allreduce_host")
 
@@ -259,7 +266,7 @@ def _collective(fn, name, inputs, size, codec, out, workspace, workspace_bytes, 
     outs = _ptr_array(out)
     N = len(inputs) if N is None else N
     opts = _options(min_quant_bytes, "auto", stage_events)
-    _check(fn(ins[0] if ins else None, N, size, _codec(codec), outs[0] if outs else None, _ptr(workspace),
+    _check(fn(ins, N, size, _codec(codec), outs, _ptr(workspace),
               workspace_bytes, ctypes.byref(opts), _stream(stream)), name)
 
 

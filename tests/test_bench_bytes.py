@@ -86,5 +86,6 @@ def test_single_pass_labels_follow_the_launcher_rule():
     assert k("fp8", 2, 2048 * 2048).startswith("k_allreduce_single<")           # FP8 above the tile form: CTA-wide
     src = open(os.path.join(ROOT, "quantized_precision_all_b200", "csrc", "lpar_kernels.cu")).read()
     assert "kBulkMinBytes = (size_t)128 << 20" in src and "kInt3WarpMaxBytes = (size_t)512 << 20" in src
-    assert "return C == kFP8 ? 512 : 256;" in src
+    tiles_src = open(os.path.join(ROOT, "quantized_precision_all_b200", "csrc", "lpar_tiles.cuh")).read()
+    assert "return C == kFP8 ? 512 : 256;" in tiles_src
     assert bench.BULK_MIN_BYTES == 128 * mib and bench.INT3_WARP_MAX_BYTES == 512 * mib
