@@ -531,6 +531,26 @@ def test_allreduce_random_cases(L, case):
         assert np.array_equal(o, ref[0]), (codec, N, tiles, schedule, thr, inplace)
 
 
+# The same over 257..700 tiles per rank, where the persistent forms run (above
+# the tile form's limit), with ragged last chunks and every schedule.
+@pytest.mark.parametrize("case", range(16))
+def test_allreduce_random_cases_persistent(L, case):
+    rng = np.random.default_rng(9500 + case)
+    codec = CODECS[rng.integers(len(CODECS))]
+    N = int(rng.integers(1, 9))
+    tiles = int(rng.integers(257, 701))
+    n = tiles * 2048
+    schedule = ["auto", "fused", "three_stage", "single_pass", "one_shot"][rng.integers(5)]
+    inplace = bool(rng.integers(2))
+    xs = [adversarial_bf16(n, int(rng.integers(1 << 30))) if rng.integers(2)
+          else random_bf16(n, int(rng.integers(1 << 30)), float(2.0 ** rng.integers(-8, 9))) for _ in range(N)]
+    outs, _ = run_allreduce(L, xs, codec, schedule, 0, inplace)
+    ref, used = (O.allreduce_oneshot if schedule == "one_shot" else O.allreduce)(xs, codec)
+    assert used == codec
+    for o in outs:
+        assert np.array_equal(o, ref[0]), (codec, N, tiles, schedule, inplace)
+
+
 @pytest.mark.parametrize("codec", CODECS)
 def test_allreduce_in_place(L, codec):
     n = 2048 * 6
