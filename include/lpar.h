@@ -58,7 +58,8 @@
  *    LPAR_TILE_ELEMS, at most 2^44; n == 0 is a valid no-op.  N must be in
  *    [1, LPAR_MAX_RANKS].
  *  - Every data pointer must be 16-byte aligned.
- *  - The caller owns all memory.  The library allocates nothing, frees
+ *  - The caller owns all memory.  The library (lpar_peer_alloc and
+ *    lpar_peer_free aside, whose job it is) allocates nothing, frees
  *    nothing, never synchronises and keeps no pointer after a call returns.
  *    Work is enqueued on `stream` asynchronously; buffers must stay valid
  *    until the stream has passed the call.
@@ -316,6 +317,88 @@ size_t lpar_host_staging_bytes_f32(int N, size_t chunk, lpar_codec_t codec);
 lpar_status_t lpar_allreduce_f32_host(const void *const *host_inputs, int N, size_t n, lpar_codec_t codec,
                                       void *const *host_out, size_t chunk, void *device, size_t device_bytes,
                                       const lpar_options_t *opts, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The all-reduce as one kernel per rank over peer memory ("RCCLX: Innovating
+ * GPU communications on AMD platforms", Direct Data Access: ranks store into
+ * each other's memory directly, and the tree all-reduce is a reduce-scatter
+ * followed by an all-gather; Low-Precision Collectives: the quantised wire is
+ * what crosses the links).  Each rank's launch quantises its message and
+ * stores every wire tile straight into the mailbox of the tile's shard owner
+ * (shard j = tiles [jT/N, (j+1)T/N) of the T tiles), reduces and requantises
+ * its own shard once every rank's tiles have arrived and stores the reduced
+ * tiles into every rank's gathered wire, then decodes the gathered wire into
+ * its output.  Arrival is signalled by flag words that carry the call's epoch.
+ * The results equal lpar_allreduce's (same codec, schedule irrelevant) bit for
+ * bit.
+ *
+ * Per rank r, in memory the other ranks can reach (peer memory of another GPU
+ * opened with lpar_peer_import, or, when all ranks run in one launch, plain
+ * device memory):
+ *   mailboxes[r]  lpar_peer_mailbox_bytes(N, n, codec) bytes
+ *   gathered[r]   lpar_peer_gather_bytes(n, codec) bytes
+ *   flags[r]      lpar_peer_flag_bytes(N, n) bytes, all zero before the first
+ *                 call (lpar_peer_alloc zeroes) and left alone between calls
+ * and, for the ranks this launch runs only, inputs[r] / outputs[r] (n BF16
+ * values each, device memory of this GPU; an output may equal its input, as
+ * each output tile is written only after every launch has read that tile).
+ * All are host arrays of N pointers valid in the calling process, every
+ * pointer 16-byte aligned.
+ *
+ * The launch runs ranks [rank0, rank0 + ranks).  With ranks == N it is the
+ * whole all-reduce on this GPU (mailboxes and gathered wires in its HBM).
+ * With ranks < N the other ranks must be running their own launches on other
+ * GPUs (their buffers are memory of another device, or mapped host memory);
+ * a rank outside the launch whose buffers are memory of the current device is
+ * refused with LPAR_ERR_INVALID_ARG, because two launches on one GPU that
+ * wait on each other are not guaranteed to run at the same time.
+ *
+ * epoch: 1 for the first call on a set of buffers, one more for every later
+ * call; every rank passes the same epoch to the same call.  0 is refused.
+ * timeout_ns (> 0): a wait for another rank's tiles gives up when it has seen
+ * no arrival for this long (or after timeout_ns / 128 polls).
+ * status: LPAR_PEER_STATUS_WORDS uint32 words of this GPU's memory, 16-byte
+ * aligned, zero before the call.  The kernel leaves them zero on success; a
+ * wait that gives up writes [0] = 1, [1] = the phase (1: waiting for mailbox
+ * tiles, 2: waiting for gathered tiles), [2] = the waiting rank, [3] = the
+ * flag's index, and every other wait of the launch then returns too: the call
+ * ends with the outputs incomplete instead of hanging.  A launch that finds
+ * [0] != 0 does nothing.  After a failure the buffers' flags are in an
+ * unknown state: zero them (and the status) on every rank and restart the
+ * epochs at 1.
+ *
+ * The kernel is a cooperative launch (all its CTAs resident at once) on
+ * `stream`.  Argument errors return before the launch; LPAR_ERR_UNSUPPORTED
+ * for an unknown codec or a device without cooperative launch.
+ * ------------------------------------------------------------------------- */
+#define LPAR_PEER_STATUS_WORDS 4
+#define LPAR_PEER_HANDLE_BYTES 64
+
+/* Buffer sizes of lpar_allreduce_peer; 0 for N outside [1, LPAR_MAX_RANKS], an
+ * unknown codec, n not a multiple of 2048 or above 2^44, and for n == 0. */
+size_t lpar_peer_mailbox_bytes(int N, size_t n, lpar_codec_t codec);
+size_t lpar_peer_gather_bytes(size_t n, lpar_codec_t codec);
+size_t lpar_peer_flag_bytes(int N, size_t n);
+
+lpar_status_t lpar_allreduce_peer(const void *const *inputs, void *const *outputs, void *const *mailboxes,
+                                  void *const *gathered, void *const *flags, int N, int rank0, int ranks,
+                                  size_t n, lpar_codec_t codec, uint32_t epoch, uint64_t timeout_ns,
+                                  uint32_t *status, cudaStream_t stream);
+
+/* Buffers shared between processes (CUDA IPC), the one place the library
+ * allocates: lpar_peer_alloc reserves `bytes` of device memory on the current
+ * device, zeroes it and synchronises the device; lpar_peer_free releases it.
+ * lpar_peer_export writes the LPAR_PEER_HANDLE_BYTES-byte handle of an
+ * lpar_peer_alloc'd pointer; another process passes the handle to
+ * lpar_peer_import to map the memory (peer access enabled as needed) and
+ * unmaps it with lpar_peer_close.  A process cannot import its own handle.
+ * LPAR_ERR_INVALID_ARG for a null argument, LPAR_ERR_CUDA when the CUDA call
+ * fails. */
+lpar_status_t lpar_peer_alloc(size_t bytes, void **ptr);
+lpar_status_t lpar_peer_free(void *ptr);
+lpar_status_t lpar_peer_export(const void *ptr, unsigned char *handle);
+lpar_status_t lpar_peer_import(const unsigned char *handle, void **ptr);
+lpar_status_t lpar_peer_close(void *ptr);
 
 /* The codec lpar_allreduce runs for these arguments after the threshold. */
 lpar_codec_t lpar_effective_codec(size_t n, lpar_codec_t codec, const lpar_options_t *opts);

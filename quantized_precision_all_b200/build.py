@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "lpar_kernels.cu"), os.path.join(CSRC, "lpar_collectives.cu"),
            os.path.join(CSRC, "lpar_f32.cu"), os.path.join(CSRC, "lpar_static_ws.cu"),
-           os.path.join(CSRC, "lpar_host.cu")]
+           os.path.join(CSRC, "lpar_host.cu"), os.path.join(CSRC, "lpar_peer.cu")]
 HEADERS = [os.path.join(CSRC, "lpar_codec.cuh"), os.path.join(CSRC, "lpar_tiles.cuh"), os.path.join(ROOT, "include", "lpar.h")]
 LIB = os.path.join(HERE, "liblpar.so")
 PTXAS_LOG = os.path.join(HERE, "liblpar.ptxas.txt")

@@ -34,8 +34,12 @@ EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_q
            "lpar_decode", "lpar_allreduce", "lpar_allreduce_static", "lpar_effective_codec", "lpar_status_string",
            "lpar_collective_workspace_bytes", "lpar_reduce_scatter", "lpar_all_gather", "lpar_all_to_all",
            "lpar_allreduce_f32", "lpar_host_staging_bytes", "lpar_allreduce_host", "lpar_host_staging_bytes_f32",
-           "lpar_allreduce_f32_host")
+           "lpar_allreduce_f32_host", "lpar_peer_mailbox_bytes", "lpar_peer_gather_bytes", "lpar_peer_flag_bytes",
+           "lpar_allreduce_peer", "lpar_peer_alloc", "lpar_peer_free", "lpar_peer_export", "lpar_peer_import",
+           "lpar_peer_close")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
+LPAR_PEER_STATUS_WORDS = 4
+LPAR_PEER_HANDLE_BYTES = 64
 
 
 class LparError(RuntimeError):
@@ -73,6 +77,16 @@ def _load():
         "lpar_allreduce_host": (i32, [vpp, i32, sz, i32, vpp, sz, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
         "lpar_host_staging_bytes_f32": (sz, [i32, sz, i32]),
         "lpar_allreduce_f32_host": (i32, [vpp, i32, sz, i32, vpp, sz, vp, sz, ctypes.POINTER(lpar_options_t), vp]),
+        "lpar_peer_mailbox_bytes": (sz, [i32, sz, i32]),
+        "lpar_peer_gather_bytes": (sz, [sz, i32]),
+        "lpar_peer_flag_bytes": (sz, [i32, sz]),
+        "lpar_allreduce_peer": (i32, [vpp, vpp, vpp, vpp, vpp, i32, i32, i32, sz, i32, ctypes.c_uint32,
+                                      ctypes.c_uint64, vp, vp]),
+        "lpar_peer_alloc": (i32, [sz, vpp]),
+        "lpar_peer_free": (i32, [vp]),
+        "lpar_peer_export": (i32, [vp, ctypes.c_char_p]),
+        "lpar_peer_import": (i32, [ctypes.c_char_p, vpp]),
+        "lpar_peer_close": (i32, [vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -256,6 +270,71 @@ def lpar_allreduce_host(host_inputs, n, codec, host_out, chunk, device, device_b
            "lpar_allreduce_host")
 
 
+def lpar_peer_mailbox_bytes(N, n, codec):
+    return _lib.lpar_peer_mailbox_bytes(N, n, _codec(codec))
+
+
+def lpar_peer_gather_bytes(n, codec):
+    return _lib.lpar_peer_gather_bytes(n, _codec(codec))
+
+
+def lpar_peer_flag_bytes(N, n):
+    return _lib.lpar_peer_flag_bytes(N, n)
+
+
+def _addr(x):
+    """Address of a tensor (device or host) or a raw integer address."""
+    if x is None or isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("lpar: tensors must be contiguous")
+    return x.data_ptr()
+
+
+def lpar_allreduce_peer(inputs, outputs, mailboxes, gathered, flags, n, codec, epoch, timeout_ns, status,
+                        rank0=0, ranks=None, stream=None):
+    """inputs/outputs: N entries (None outside the launch's ranks); mailboxes,
+    gathered, flags: N buffers (tensors or addresses, on this GPU or reachable
+    from it); status: LPAR_PEER_STATUS_WORDS words of this GPU's memory."""
+    N = len(mailboxes)
+    ranks = N - rank0 if ranks is None else ranks
+    _check(_lib.lpar_allreduce_peer(_ptr_array(inputs, _addr), _ptr_array(outputs, _addr),
+                                    _ptr_array(mailboxes, _addr), _ptr_array(gathered, _addr),
+                                    _ptr_array(flags, _addr), N, rank0, ranks, n, _codec(codec), epoch,
+                                    int(timeout_ns), _ptr(status), _stream(stream)), "lpar_allreduce_peer")
+
+
+def lpar_peer_alloc(nbytes):
+    """Device address of `nbytes` of zeroed, IPC-exportable memory."""
+    p = ctypes.c_void_p()
+    _check(_lib.lpar_peer_alloc(nbytes, ctypes.byref(p)), "lpar_peer_alloc")
+    return p.value
+
+
+def lpar_peer_free(ptr):
+    _check(_lib.lpar_peer_free(ptr), "lpar_peer_free")
+
+
+def lpar_peer_export(ptr):
+    """The IPC handle of an lpar_peer_alloc'd address, as bytes."""
+    h = ctypes.create_string_buffer(LPAR_PEER_HANDLE_BYTES)
+    _check(_lib.lpar_peer_export(ptr, h), "lpar_peer_export")
+    return h.raw
+
+
+def lpar_peer_import(handle):
+    """Map another process's lpar_peer_alloc'd memory; returns its address here."""
+    if len(handle) != LPAR_PEER_HANDLE_BYTES:
+        raise ValueError("lpar: an IPC handle has %d bytes" % LPAR_PEER_HANDLE_BYTES)
+    p = ctypes.c_void_p()
+    _check(_lib.lpar_peer_import(handle, ctypes.byref(p)), "lpar_peer_import")
+    return p.value
+
+
+def lpar_peer_close(ptr):
+    _check(_lib.lpar_peer_close(ptr), "lpar_peer_close")
+
+
 def lpar_collective_workspace_bytes(op, N, size, codec):
     return _lib.lpar_collective_workspace_bytes(OPS[op] if isinstance(op, str) else int(op), N, size, _codec(codec))
 
@@ -384,6 +463,53 @@ def all_to_all(inputs, codec, min_quant_bytes=0, stream=None):
     ws = _workspace("all_to_all", N, m, codec, min_quant_bytes, inputs[0].device)
     lpar_all_to_all(inputs, m, codec, out, ws, ws.numel(), min_quant_bytes, stream)
     return out
+
+
+class PeerTimeout(RuntimeError):
+    """A wait of lpar_allreduce_peer gave up: (phase, waiting rank, flag index)."""
+
+
+class PeerBuffers:
+    """The buffers of lpar_allreduce_peer for N ranks that all live on one GPU
+    (mailboxes, gathered wires and flags as torch tensors, zeroed), the status
+    words and the epoch counter.  One set serves any number of calls of the
+    same (N, n, codec) in stream order."""
+
+    def __init__(self, N, n, codec, device=None):
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.N, self.n, self.codec = N, n, codec
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.mailboxes = [torch.zeros(max(lpar_peer_mailbox_bytes(N, n, codec), 16), **u8) for _ in range(N)]
+        self.gathered = [torch.zeros(max(lpar_peer_gather_bytes(n, codec), 16), **u8) for _ in range(N)]
+        self.flags = [torch.zeros(max(lpar_peer_flag_bytes(N, n), 16), **u8) for _ in range(N)]
+        self.status = torch.zeros(LPAR_PEER_STATUS_WORDS, dtype=torch.int32, device=dev)
+        self.epoch = 0
+
+    def allreduce(self, inputs, out, timeout_ns=1_000_000_000, stream=None):
+        self.epoch += 1
+        lpar_allreduce_peer(inputs, out, self.mailboxes, self.gathered, self.flags, self.n, self.codec, self.epoch,
+                            timeout_ns, self.status, 0, self.N, stream)
+        return out
+
+    def check(self):
+        """Synchronise and raise PeerTimeout if a wait gave up."""
+        w = [int(v) for v in self.status.cpu()]
+        if w[0]:
+            raise PeerTimeout("lpar_allreduce_peer: a wait gave up (phase %d, rank %d, flag %d)" % tuple(w[1:]))
+
+
+def allreduce_peer(inputs, codec, out=None, buffers=None, timeout_ns=1_000_000_000, stream=None):
+    """All-reduce of N equal-size BF16 CUDA tensors by the peer-memory kernel,
+    all ranks in one launch on this GPU; returns the N outputs (equal to
+    `allreduce`'s).  Pass `buffers` (a PeerBuffers) to reuse them across calls."""
+    import torch
+    N, n = len(inputs), inputs[0].numel()
+    if out is None:
+        out = [torch.empty_like(x) for x in inputs]
+    if buffers is None:
+        buffers = PeerBuffers(N, n, codec, inputs[0].device)
+    return buffers.allreduce(inputs, out, timeout_ns, stream)
 
 
 def allreduce_f32(inputs, codec, out=None, min_quant_bytes=0, stream=None):

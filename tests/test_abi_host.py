@@ -269,3 +269,61 @@ def test_python_binding_rejects_host_tensors(L):
     x = torch.zeros(2048, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         L.lpar_quantize(x, 2048, "int4", x)
+
+
+def test_peer_buffer_bytes(L):
+    n = 2048 * 10
+    assert L.lpar_peer_mailbox_bytes(3, n, "int4") == 3 * 4 * 1152        # 3 slots of ceil(10 / 3) tiles
+    assert L.lpar_peer_mailbox_bytes(2, n, "bf16") == 2 * 5 * 4096
+    assert L.lpar_peer_mailbox_bytes(1, n, "mxfp4") == 10 * 1088
+    assert L.lpar_peer_gather_bytes(n, "int3") == 10 * 896
+    assert L.lpar_peer_gather_bytes(n, "fp8") == 10 * 2304
+    assert L.lpar_peer_flag_bytes(3, n) == 2 * 3 * 4 * 4                  # P = ceil(10 / 3) chunks per shard
+    assert L.lpar_peer_flag_bytes(8, 2048 << 20) == 2 * 8 * 1024 * 4      # P capped at 1024
+    assert L.lpar_peer_flag_bytes(8, 2048 * 8 * 1024) == 2 * 8 * 1024 * 4
+    assert L.lpar_peer_flag_bytes(8, 2048 * (8 * 1024 - 8)) == 2 * 8 * 1023 * 4
+    for bad in (L.lpar_peer_mailbox_bytes(0, n, "int4"), L.lpar_peer_mailbox_bytes(9, n, "int4"),
+                L.lpar_peer_mailbox_bytes(2, n + 1, "int4"), L.lpar_peer_mailbox_bytes(2, n, 7),
+                L.lpar_peer_gather_bytes(n + 2, "int4"), L.lpar_peer_gather_bytes(n, 9),
+                L.lpar_peer_flag_bytes(0, n), L.lpar_peer_flag_bytes(2, n + 4), L.lpar_peer_flag_bytes(2, 0)):
+        assert bad == 0
+
+
+def test_argument_errors_allreduce_peer(L):
+    n = 2048 * 4
+
+    def call(inputs=(A, A), outputs=(A, A), mailboxes=(A, A), gathered=(A, A), flags=(A, A), n=n, codec="int4",
+             epoch=1, timeout_ns=10 ** 6, status=A, rank0=0, ranks=None):
+        return status_of(L.lpar_allreduce_peer, list(inputs), list(outputs), list(mailboxes), list(gathered),
+                         list(flags), n, codec, epoch, timeout_ns, status, rank0=rank0, ranks=ranks, stream=0)
+
+    assert call(epoch=0) == 1
+    assert call(timeout_ns=0) == 1
+    assert call(status=0) == 1
+    assert call(status=M) == 2
+    assert call(mailboxes=(A, M)) == 2
+    assert call(gathered=(M, A)) == 2
+    assert call(flags=(A, 0)) == 1
+    assert call(inputs=(A, 0)) == 1                      # rank 1 runs in this launch: it needs an input
+    assert call(outputs=(M, A)) == 2
+    assert call(n=n + 2048 // 2) == 1
+    assert call(codec=9) == 4
+    assert call(rank0=1, ranks=2) == 1
+    assert call(rank0=-1, ranks=1) == 1
+    assert call(ranks=0) == 1
+    assert call(inputs=[A] * 9, outputs=[A] * 9, mailboxes=[A] * 9, gathered=[A] * 9, flags=[A] * 9) == 1
+    assert call(n=0) == 0                                # a no-op, nothing launched
+    assert call(inputs=(A, None), outputs=(A, None), ranks=1, n=0) == 0   # rank 1 outside: no input needed
+    lib = L.library()
+    assert lib.lpar_allreduce_peer(None, None, None, None, None, 2, 0, 2, n, 2, 1, 10, A, None) == 1
+
+
+def test_peer_ipc_argument_errors(L):
+    lib = L.library()
+    assert lib.lpar_peer_alloc(0, None) == 1
+    assert lib.lpar_peer_free(None) == 1
+    assert lib.lpar_peer_export(None, None) == 1
+    assert lib.lpar_peer_import(None, None) == 1
+    assert lib.lpar_peer_close(None) == 1
+    with pytest.raises(ValueError):
+        L.lpar_peer_import(b"\0" * 10)

@@ -1,0 +1,337 @@
+"""The peer-memory all-reduce kernel (lpar_allreduce_peer) against the CPU
+oracle, bit for bit (needs a B200).
+
+All N ranks run in one launch on the one GPU, so every wait is on flags that
+the same launch raises.  Besides the outputs, the exchange buffers are checked
+against the oracle: rank j's mailbox slot s holds shard j of rank s's stage-1
+wire, and every rank's gathered wire holds the requantised wire of the whole
+message.  Every buffer the kernel writes has guard bands.  The failure path is
+tested with a rank whose buffers are mapped host memory and which never runs:
+its flags are never raised, the waits give up after the timeout and report it
+in the status words, and the context stays usable.  The CUDA IPC calls are
+tested across processes that share the GPU: each process exports its buffers,
+one process maps them all and runs the launch, the others only read their
+results afterwards (no kernel waits for another process)."""
+import os
+import socket
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import oracle as O
+from tests.test_gpu_parity import Guarded, adversarial_bf16, host_u16, random_bf16, to_device
+
+pytestmark = pytest.mark.gpu
+
+CODECS = ("int4", "int3", "fp8", "mxfp4", "bf16")
+TIMEOUT_NS = 2_000_000_000
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_precision_all_b200 import build
+    build.build()
+    from quantized_precision_all_b200 import lpar
+    return lpar
+
+
+class Bufs:
+    """Guarded mailboxes, gathered wires and flags of N ranks, and the status."""
+
+    def __init__(self, L, N, n, codec):
+        self.N, self.n, self.codec = N, n, codec
+        self.mbox = [Guarded(L.lpar_peer_mailbox_bytes(N, n, codec), fill=0) for _ in range(N)]
+        self.gath = [Guarded(L.lpar_peer_gather_bytes(n, codec), fill=0) for _ in range(N)]
+        self.flags = [Guarded(L.lpar_peer_flag_bytes(N, n), fill=0) for _ in range(N)]
+        self.status = torch.zeros(4, dtype=torch.int32, device="cuda")
+        self.epoch = 0
+
+    def call(self, L, ins, outs):
+        self.epoch += 1
+        L.lpar_allreduce_peer([g.ptr() for g in ins], [g.ptr() for g in outs], [g.ptr() for g in self.mbox],
+                              [g.ptr() for g in self.gath], [g.ptr() for g in self.flags], self.n, self.codec,
+                              self.epoch, TIMEOUT_NS, self.status)
+        torch.cuda.synchronize()
+        assert self.status.tolist() == [0, 0, 0, 0]
+        for g in self.mbox + self.gath + self.flags:
+            g.check()
+        flags = [g.host().view(np.uint32) for g in self.flags]
+        for f in flags:                                    # every flag of a non-empty chunk carries the epoch
+            assert np.all((f == self.epoch) | (f == 0))
+
+
+def inputs(N, n, seed):
+    return [adversarial_bf16(n, seed + r) if r % 2 else random_bf16(n, seed + 50 + r, 2.0 ** (r - 3))
+            for r in range(N)]
+
+
+def check_exchange(L, b, xs, codec):
+    """Mailbox slots and gathered wires against the oracle's wires."""
+    N, n = len(xs), xs[0].size
+    T = n // 2048
+    tb = L.lpar_tile_bytes(codec)
+    wires = [O.quantize(x, codec) for x in xs] if codec != "bf16" else [x.view(np.uint8) for x in xs]
+    slot = -(-T // N)
+    for j in range(N):
+        t0, t1 = j * T // N, (j + 1) * T // N
+        host = b.mbox[j].host()
+        for s in range(N):
+            got = host[s * slot * tb:(s * slot + t1 - t0) * tb]
+            assert np.array_equal(got, wires[s][t0 * tb:t1 * tb]), ("mailbox", j, s)
+    gathered = O.reduce(wires, 0, T, codec) if codec != "bf16" else None
+    for r in range(N):
+        if gathered is not None:
+            assert np.array_equal(b.gath[r].host(), gathered), ("gathered", r)
+
+
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("N", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("tiles", [1, 9, 37])
+def test_peer_matches_oracle(L, codec, N, tiles):
+    n = tiles * 2048
+    xs = inputs(N, n, 8100 + 10 * N + tiles)
+    ins = [to_device(x) for x in xs]
+    outs = [Guarded(2 * n, fill=0) for _ in range(N)]
+    b = Bufs(L, N, n, codec)
+    b.call(L, ins, outs)
+    ref, used = O.allreduce(xs, codec)
+    assert used == codec
+    for o in outs + ins:
+        o.check()
+    for r, o in enumerate(outs):
+        assert np.array_equal(host_u16(o), ref[0]), (codec, N, tiles, r)
+    check_exchange(L, b, xs, codec)
+
+
+@pytest.mark.parametrize("codec", CODECS)
+def test_peer_repeated_calls_reuse_the_buffers_and_in_place(L, codec):
+    """Epochs 1..4 on one set of buffers, new inputs every call; the last call
+    in place (outputs = inputs)."""
+    N, tiles = 3, 11
+    n = tiles * 2048
+    b = Bufs(L, N, n, codec)
+    for k in range(4):
+        xs = inputs(N, n, 8300 + 10 * k)
+        ins = [to_device(x) for x in xs]
+        outs = ins if k == 3 else [Guarded(2 * n, fill=0) for _ in range(N)]
+        b.call(L, ins, outs)
+        ref, _ = O.allreduce(xs, codec)
+        for o in outs:
+            o.check()
+            assert np.array_equal(host_u16(o), ref[0]), (codec, k)
+
+
+def sampled(xs_dev, tiles):
+    idx = torch.from_numpy((tiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
+    return idx, [x[idx].view(torch.int16).cpu().numpy().view(np.uint16) for x in xs_dev]
+
+
+@pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4", "bf16"])
+@pytest.mark.parametrize("N,T", [(2, 4099), (5, 5 * 3 * 1024 + 7), (8, 1024 * 8 + 2)])
+def test_peer_many_tile_chunks(L, codec, N, T):
+    """Shards of more than 1024 tiles (the chunk count's cap), so chunks hold
+    several tiles and are ragged; every chunk boundary of shard 0 and 1 and 256
+    random tiles compared with the oracle, and the whole of rank 0's output with
+    lpar_allreduce's."""
+    n = T * 2048
+    xs = [to_device(x) for x in inputs(N, n, 8400 + N)]
+    outs = [Guarded(2 * n, fill=0) for _ in range(N)]
+    b = Bufs(L, N, n, codec)
+    b.call(L, xs, outs)
+    P = min(-(-T // N), 1024)
+    bounds = []
+    for j in (0, 1):
+        base, S = j * T // N, (j + 1) * T // N - j * T // N
+        bounds += [base + c * S // P for c in range(P)] + [base + c * S // P - 1 for c in range(1, P + 1)]
+    rng = np.random.default_rng(8500 + N)
+    tiles = np.unique(np.concatenate([bounds, rng.choice(T, 256, replace=False), [T - 1]]))
+    idx, sample_in = sampled([x.t.view(torch.bfloat16) for x in xs], tiles)
+    ref, _ = O.allreduce(sample_in, codec)
+    for o in outs:
+        o.check()
+        assert np.array_equal(o.t.view(torch.bfloat16)[idx].view(torch.int16).cpu().numpy().view(np.uint16), ref[0])
+    ws = torch.empty(L.lpar_workspace_bytes(N, n, codec), dtype=torch.uint8, device="cuda")
+    want = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    L.lpar_allreduce([x.ptr() for x in xs], n, codec, [want] + [o.ptr() for o in outs[1:]], ws, ws.numel())
+    torch.cuda.synchronize()
+    assert torch.equal(want.view(torch.int16), outs[0].t.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["large_int3_int4"])
+def test_peer_full_size_sampled(L, name):
+    """1 GiB per rank, N = 2 (the large workload), every codec of it: 1024
+    seeded random tiles plus the first and last against the oracle."""
+    w = W.WORKLOADS[name]
+    xs = W.make_inputs(w, "cuda")
+    T = w.n // 2048
+    rng = np.random.default_rng(8600)
+    tiles = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 1024, replace=False)]))
+    idx, sample_in = sampled(xs, tiles)
+    for codec in w.codecs:
+        outs = [torch.empty_like(x) for x in xs]
+        buf = L.PeerBuffers(w.N, w.n, codec)
+        buf.allreduce(xs, outs)
+        buf.check()
+        ref, _ = O.allreduce(sample_in, codec)
+        for o in outs:
+            assert np.array_equal(o[idx].view(torch.int16).cpu().numpy().view(np.uint16), ref[0]), codec
+        del outs, buf
+    del xs
+    torch.cuda.empty_cache()
+
+
+def test_peer_wait_gives_up_on_a_rank_that_never_runs(L):
+    """N = 2, the launch runs rank 0 only; rank 1's buffers are pinned host
+    memory and nothing ever runs rank 1, so its flags are never raised.  Rank
+    0's waits for rank 1's mailbox tiles give up after the timeout, the status
+    words say so, and the context still runs a normal call afterwards."""
+    N, tiles, codec = 2, 6, "int4"
+    n = tiles * 2048
+    xs = inputs(N, n, 8700)
+    x0 = to_device(xs[0])
+    out0 = Guarded(2 * n, fill=0)
+    mb0 = Guarded(L.lpar_peer_mailbox_bytes(N, n, codec), fill=0)
+    ga0 = Guarded(L.lpar_peer_gather_bytes(n, codec), fill=0)
+    fl0 = Guarded(L.lpar_peer_flag_bytes(N, n), fill=0)
+    host = [torch.zeros(max(k, 16), dtype=torch.uint8, pin_memory=True)
+            for k in (L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
+                      L.lpar_peer_flag_bytes(N, n))]
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    timeout = 50_000_000                                  # 50 ms
+    t0 = time.perf_counter()
+    L.lpar_allreduce_peer([x0.ptr(), None], [out0.ptr(), None], [mb0.ptr(), host[0].data_ptr()],
+                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, 1, timeout,
+                          status, rank0=0, ranks=1)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    w = status.tolist()
+    P = min(-(-tiles // N), 1024)
+    assert w[0] == 1 and w[1] == 1 and w[2] == 0, w       # phase 1 (mailbox), waiting rank 0
+    assert P <= w[3] < 2 * P, w                            # a flag of source 1
+    assert elapsed < 5.0, elapsed
+    for g in (out0, mb0, ga0, fl0):
+        g.check()
+    # rank 0's phase A did reach rank 1: its tiles of shard 1 are in rank 1's mailbox, slot 0
+    wire0 = O.quantize(xs[0], codec)
+    tb, t1 = L.lpar_tile_bytes(codec), tiles // N
+    assert np.array_equal(host[0][:(tiles - t1) * tb].numpy(), wire0[t1 * tb:])
+    assert np.all(host[2].numpy().view(np.uint32)[:P] == 1)
+    # a launch that finds the status set does nothing
+    out1 = Guarded(2 * n, fill=0x33)
+    L.lpar_allreduce_peer([x0.ptr(), None], [out1.ptr(), None], [mb0.ptr(), host[0].data_ptr()],
+                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, 2, timeout,
+                          status, rank0=0, ranks=1)
+    torch.cuda.synchronize()
+    assert np.all(out1.host() == 0x33)
+    # the context is intact: a normal all-reduce of both ranks
+    out = L.allreduce_peer([torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in xs], codec)
+    torch.cuda.synchronize()
+    ref, _ = O.allreduce(xs, codec)
+    for o in out:
+        assert np.array_equal(o.view(torch.int16).cpu().numpy().view(np.uint16), ref[0])
+
+
+def test_peer_refuses_an_absent_rank_on_this_device(L):
+    """A rank outside the launch whose buffers are this GPU's memory would have
+    to be a second launch on the same GPU waiting on this one: refused before
+    anything is launched."""
+    N, n, codec = 2, 2048 * 4, "int4"
+    bufs = [torch.zeros(max(k, 16), dtype=torch.uint8, device="cuda")
+            for k in (L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
+                      L.lpar_peer_flag_bytes(N, n))] * 2
+    x = torch.zeros(n, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    with pytest.raises(L.LparError) as e:
+        L.lpar_allreduce_peer([x, None], [x, None], [bufs[0], bufs[3]], [bufs[1], bufs[4]], [bufs[2], bufs[5]], n,
+                              codec, 1, TIMEOUT_NS, status, rank0=0, ranks=1)
+    assert e.value.status == 1
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0, 0, 0]
+
+
+# ---------------------------------------------------------------------------
+# CUDA IPC across processes on the one GPU.
+# ---------------------------------------------------------------------------
+class _Raw:
+    def __init__(self, ptr, nbytes):
+        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1", "data": (ptr, False), "version": 3}
+
+
+def _layout(L, N, n, codec):
+    """Byte offsets of input, output, mailbox, gathered wire and flags in one
+    exported region (each 256-byte aligned)."""
+    sizes = [2 * n, 2 * n, L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
+             L.lpar_peer_flag_bytes(N, n)]
+    offs, o = [], 0
+    for s in sizes:
+        offs.append(o)
+        o += -(-s // 256) * 256
+    return offs, o
+
+
+def _ipc_worker(rank, world, port, n, codec, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        from quantized_precision_all_b200 import lpar as L
+        offs, total = _layout(L, world, n, codec)
+        region = L.lpar_peer_alloc(total)
+        view = torch.as_tensor(_Raw(region, total), device="cuda")
+        x = inputs(world, n, 8800)[rank]
+        view[offs[0]:offs[0] + 2 * n].copy_(torch.from_numpy(x.view(np.uint8)))
+        torch.cuda.synchronize()
+        handles = [None] * world
+        dist.all_gather_object(handles, L.lpar_peer_export(region))
+        if rank == 0:
+            bases = [region] + [L.lpar_peer_import(h) for h in handles[1:]]
+            status = torch.zeros(4, dtype=torch.int32, device="cuda")
+            ptr = lambda k: [b + offs[k] for b in bases]
+            L.lpar_allreduce_peer(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), n, codec, 1, TIMEOUT_NS, status)
+            torch.cuda.synchronize()
+            st = status.tolist()
+            for b in bases[1:]:
+                L.lpar_peer_close(b)
+        else:
+            st = None
+        dist.barrier()
+        out = view[offs[1]:offs[1] + 2 * n].cpu().numpy().copy()
+        dist.barrier()
+        L.lpar_peer_free(region)
+        q.put((rank, out, st))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world,tiles,codec", [(2, 7, "int3"), (3, 10, "fp8")])
+def test_peer_buffers_shared_by_ipc(world, tiles, codec):
+    import torch.multiprocessing as mp
+    n = tiles * 2048
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_worker, args=(r, world, port, n, codec, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r, out, st = q.get(timeout=300)
+        got[r] = (out, st)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert got[0][1] == [0, 0, 0, 0]
+    ref, _ = O.allreduce(inputs(world, n, 8800), codec)
+    for r in range(world):
+        assert np.array_equal(got[r][0].view(np.uint16), ref[0]), r
