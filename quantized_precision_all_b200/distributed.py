@@ -25,7 +25,11 @@ the all-to-all of chunk k overlaps the quantisation of chunk k + 1, and the
 all-gather of chunk k the reduction of chunk k + 1.
 
 The result is bit-identical to ``lpar_allreduce`` on the N messages in one
-GPU.  The exchanges use ``torch.distributed`` collectives on the wire bytes;
+GPU.  ``PeerAllreduce`` is the same all-reduce with the exchanges folded into
+the library's peer-memory kernel (``lpar_allreduce_peer``): one launch per
+rank stores its wire tiles straight into the owners' memory and the reduced
+shard into every rank's memory, over CUDA IPC mappings, with no separate
+collective on the data path.  The exchanges use ``torch.distributed`` collectives on the wire bytes;
 the arithmetic runs in the library's kernels.  Buffers are allocated once per
 (message size, codec, device) and reused by later calls.  With a process group
 that cannot move device memory (gloo), the wire bytes travel through host
@@ -202,3 +206,128 @@ class DistributedAllreduce:
                     a, b = (t0 + s0) * TILE_ELEMS, (t0 + s1) * TILE_ELEMS
                     st.decode(p["gathered"][j * w:j * w + (s1 - s0) * tb], b - a, codec, out[a:b])
         return out
+
+
+# ---------------------------------------------------------------------------
+# The peer-memory form: one kernel launch per rank, exchanges by stores into
+# the other ranks' memory.
+# ---------------------------------------------------------------------------
+@dataclass
+class PeerOps:
+    """The library calls PeerAllreduce makes: alloc(nbytes) -> address (zeroed,
+    exportable), free(addr), export(addr) -> handle bytes, import_(handle) ->
+    address, close(addr), mailbox_bytes(N, n, codec), gather_bytes(n, codec),
+    flag_bytes(N, n), and run(inputs, outputs, mailboxes, gathered, flags, n,
+    codec, epoch, timeout_ns, status, rank0, ranks) for lpar_allreduce_peer."""
+    alloc: Callable
+    free: Callable
+    export: Callable
+    import_: Callable
+    close: Callable
+    mailbox_bytes: Callable
+    gather_bytes: Callable
+    flag_bytes: Callable
+    run: Callable
+
+
+def cuda_peer_ops() -> PeerOps:
+    """The library's calls (the product path)."""
+    return PeerOps(L.lpar_peer_alloc, L.lpar_peer_free, L.lpar_peer_export, L.lpar_peer_import, L.lpar_peer_close,
+                   L.lpar_peer_mailbox_bytes, L.lpar_peer_gather_bytes, L.lpar_peer_flag_bytes,
+                   lambda *a, **k: L.lpar_allreduce_peer(*a, **k))
+
+
+def _align(x, a=256):
+    return -(-x // a) * a
+
+
+class _PeerRegion:
+    """One rank's exportable region for one (n, codec) -- mailbox, gathered
+    wire, flags -- and the addresses of every rank's region in this process."""
+
+    def __init__(self, ops, group, N, me, n, codec):
+        self.ops = ops
+        sizes = [ops.mailbox_bytes(N, n, codec), ops.gather_bytes(n, codec), ops.flag_bytes(N, n)]
+        self.offsets = [0, _align(sizes[0]), _align(sizes[0]) + _align(sizes[1])]
+        self.local = ops.alloc(self.offsets[2] + _align(sizes[2]))
+        handles = [None] * N
+        dist.all_gather_object(handles, ops.export(self.local), group=group)
+        self.bases = [self.local if r == me else ops.import_(handles[r]) for r in range(N)]
+        self.me = me
+        self.epoch = 0
+
+    def pointers(self, k):
+        return [b + self.offsets[k] for b in self.bases]
+
+    def release(self, group):
+        for r, b in enumerate(self.bases):
+            if r != self.me:
+                self.ops.close(b)
+        dist.barrier(group=group)                          # nobody maps our region any more
+        self.ops.free(self.local)
+
+
+class PeerAllreduce:
+    """All-reduce of one BF16 tensor per process, one GPU per process, by the
+    peer-memory kernel.  Each rank allocates an exportable region per (message
+    size, codec) on first use; the regions' handles are exchanged over the
+    process group and mapped in every process.  A call is one launch on this
+    rank's GPU that runs this rank only; every rank must make the same calls in
+    the same order (each call's epoch is counted per region).  The ranks' GPUs
+    must be distinct: the library refuses peers whose memory is this GPU's.
+    `check()` synchronises and raises when a wait for another rank gave up
+    (after timeout_ns without progress)."""
+
+    def __init__(self, group=None, ops: Optional[PeerOps] = None, timeout_ns: int = 2_000_000_000,
+                 device=None):
+        self.group = group
+        self.N = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.ops = ops if ops is not None else cuda_peer_ops()
+        self.timeout_ns = int(timeout_ns)
+        dev = device if device is not None else (torch.device("cuda", torch.cuda.current_device())
+                                                 if torch.cuda.is_available() else torch.device("cpu"))
+        self.status = torch.zeros(L.LPAR_PEER_STATUS_WORDS, dtype=torch.int32, device=dev)
+        self._regions: Dict[tuple, _PeerRegion] = {}
+
+    def region(self, n: int, codec: str) -> _PeerRegion:
+        key = (n, codec)
+        reg = self._regions.get(key)
+        if reg is None:
+            reg = _PeerRegion(self.ops, self.group, self.N, self.rank, n, codec)
+            self._regions[key] = reg
+        return reg
+
+    def allreduce(self, x: torch.Tensor, codec: str, min_quant_bytes: int = 0,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        n = x.numel()
+        if n % TILE_ELEMS:
+            raise ValueError("the message must be a whole number of 2048-element tiles")
+        if codec != "bf16" and 2 * n < min_quant_bytes:
+            codec = "bf16"
+        if out is None:
+            out = torch.empty(n, dtype=torch.bfloat16, device=x.device)
+        if n == 0:
+            return out
+        reg = self.region(n, codec)
+        reg.epoch += 1
+        ins = [x if r == self.rank else None for r in range(self.N)]
+        outs = [out if r == self.rank else None for r in range(self.N)]
+        self.ops.run(ins, outs, reg.pointers(0), reg.pointers(1), reg.pointers(2), n, codec, reg.epoch,
+                     self.timeout_ns, self.status, rank0=self.rank, ranks=1)
+        return out
+
+    def check(self):
+        w = [int(v) for v in self.status.cpu()]
+        if w[0]:
+            raise L.PeerTimeout("rank %d: a wait gave up (phase %d, waiting rank %d, flag %d)"
+                                % (self.rank, w[1], w[2], w[3]))
+
+    def release(self):
+        """Unmap the peers' regions and free this rank's (collective: every rank
+        calls it; no call may be in flight)."""
+        if torch.cuda.is_available() and self.status.is_cuda:
+            torch.cuda.synchronize(self.status.device)
+        for key in sorted(self._regions):
+            self._regions[key].release(self.group)
+        self._regions.clear()
