@@ -592,7 +592,7 @@ def oracle_gbs(op, N, codec, tiles=64):
     w = W.Workload("oracle_sample", N=N, n=tiles * TILE, dist="student_t", nu=3, seed=9, codecs=(codec,))
     xs = [x.view(torch.int16).numpy().view("uint16") for x in W.make_inputs(w, "cpu")]
     fn = {"allreduce": O.allreduce, "reduce_scatter": O.reduce_scatter, "one_shot": O.allreduce_oneshot,
-          "all_gather": O.all_gather, "all_to_all": O.all_to_all}[op]
+          "all_gather": O.all_gather, "all_to_all": O.all_to_all, "peer_allreduce": O.allreduce}[op]
     t0 = time.perf_counter()
     fn(xs, codec)
     dt = time.perf_counter() - t0
@@ -791,18 +791,24 @@ def run_floor(args, device):
         print(json.dumps(row), flush=True)
 
 
-COLL_OPS = ("reduce_scatter", "one_shot", "all_gather", "all_to_all")
+COLL_OPS = ("reduce_scatter", "one_shot", "all_gather", "all_to_all", "peer_allreduce")
 COLL_SIZES_BYTES = (16 << 20, 256 << 20)             # per-rank message
 
 
 def collective_bytes(op, codec, N, size):
     """Algorithmic HBM bytes of one collective call.  size = elements of the size
     argument (reduce-scatter / one-shot: n per rank; all-gather: m per rank;
-    all-to-all: m per segment, N * m per rank).  Quantising codecs: the N
-    messages are read and their wires written; reductions read the N wires back
-    and write one (reduce-scatter) or N (one-shot) BF16 results; all-gather and
-    all-to-all decode from the encoder's registers and write the outputs."""
+    all-to-all: m per segment, N * m per rank; the peer-memory all-reduce: n per
+    rank).  Quantising codecs: the N messages are read and their wires written;
+    reductions read the N wires back and write one (reduce-scatter) or N
+    (one-shot) BF16 results; all-gather and all-to-all decode from the encoder's
+    registers and write the outputs.  The peer-memory all-reduce with every rank
+    in one GPU moves each stage through memory: the N messages read, the N
+    wires written into the mailboxes and read back, the reduced wire written
+    into all N gathered wires and read back, the N outputs written."""
     c = CODEC_C[codec]
+    if op == "peer_allreduce":
+        return N * size * (4 + 4 * c)
     msg = N * size if op == "all_to_all" else size        # per-rank message, elements
     out = {"reduce_scatter": 2 * size, "one_shot": N * 2 * size,
            "all_gather": N * N * 2 * size, "all_to_all": N * N * 2 * size}[op]
@@ -837,13 +843,22 @@ def run_collectives(args, device):
                 if op == "all_gather":
                     xs = [x[:size] for x in xs]
                 out_elems = N * size if op in ("all_gather", "all_to_all") else msg
-                wsb = max(L.lpar_workspace_bytes(N, msg, c) for c in codecs)
+                if op == "peer_allreduce":                 # mailboxes + gathered wires of the N ranks
+                    wsb = max(N * (L.lpar_peer_mailbox_bytes(N, msg, c) + L.lpar_peer_gather_bytes(msg, c))
+                              for c in codecs)
+                else:
+                    wsb = max(L.lpar_workspace_bytes(N, msg, c) for c in codecs)
                 sets = BufferSets(xs, out_elems, wsb, device)
                 rows = []
                 with ClockSampler(device) as clocks:
                     for codec in codecs:
-                        def call(i, st, codec=codec):
-                            if op == "one_shot":
+                        peer = ([L.PeerBuffers(N, msg, codec, device) for _ in range(sets.R)]
+                                if op == "peer_allreduce" else None)
+
+                        def call(i, st, codec=codec, peer=peer):
+                            if op == "peer_allreduce":
+                                peer[i].allreduce(sets.inputs[i], sets.outputs[i], stream=st)
+                            elif op == "one_shot":
                                 L.lpar_allreduce(sets.inputs[i], msg, codec, sets.outputs[i], sets.ws[i],
                                                  sets.ws_bytes, schedule="one_shot", stream=st)
                             else:
@@ -859,6 +874,10 @@ def run_collectives(args, device):
                                      "hbm_fraction_single": alg / (tm["us_single"] * 1e-6) / 1e9 / peak,
                                      "algorithmic_bytes": alg, "peak": peak, "cpu_baseline": cpu[(op, N, codec)],
                                      "rotated_sets": sets.R, "calls_per_graph": tm["calls_per_graph"]})
+                        if peer:
+                            for b in peer:
+                                b.check()
+                            del peer
                 clk = clocks.summary()
                 for row in rows:
                     row["clocks"] = clk
@@ -919,7 +938,7 @@ def main():
                     help="with --sweep: append rows to this JSONL file and skip the points it already holds")
     ap.add_argument("--collectives", action="store_true",
                     help="one JSON line per standalone collective point instead of the bench line")
-    ap.add_argument("--coll-op", choices=["reduce_scatter", "one_shot", "all_gather", "all_to_all"], default=None,
+    ap.add_argument("--coll-op", choices=list(COLL_OPS), default=None,
                     help="with --collectives: only this collective")
     ap.add_argument("--coll-n", type=int, default=None, help="with --collectives: only this N")
     ap.add_argument("--coll-mib", type=int, default=None, help="with --collectives: only this per-rank MiB size")

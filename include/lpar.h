@@ -353,25 +353,28 @@ lpar_status_t lpar_allreduce_f32_host(const void *const *host_inputs, int N, siz
  * refused with LPAR_ERR_INVALID_ARG, because two launches on one GPU that
  * wait on each other are not guaranteed to run at the same time.
  *
- * epoch: 1 for the first call on a set of buffers, one more for every later
- * call; every rank passes the same epoch to the same call.  0 is refused.
  * timeout_ns (> 0): a wait for another rank's tiles gives up when it has seen
  * no arrival for this long (or after timeout_ns / 128 polls).
  * status: LPAR_PEER_STATUS_WORDS uint32 words of this GPU's memory, 16-byte
- * aligned, zero before the call.  The kernel leaves them zero on success; a
- * wait that gives up writes [0] = 1, [1] = the phase (1: waiting for mailbox
- * tiles, 2: waiting for gathered tiles), [2] = the waiting rank, [3] = the
- * flag's index, and every other wait of the launch then returns too: the call
- * ends with the outputs incomplete instead of hanging.  A launch that finds
- * [0] != 0 does nothing.  After a failure the buffers' flags are in an
- * unknown state: zero them (and the status) on every rank and restart the
- * epochs at 1.
+ * aligned, zero before the first call on a set of buffers and then left to
+ * the kernel (one status per set of buffers and launching rank).  Word [4] is
+ * the epoch of the last call: each launch reads it, uses one more as its own
+ * epoch (the value its flags carry) and stores that when its last CTA
+ * finishes, so calls captured in a CUDA graph stay correct on every replay;
+ * every rank must make the same calls on its buffers in the same order.  [5]
+ * counts finished CTAs during a launch.  A wait that gives up writes [0] = 1,
+ * [1] = the phase (1: waiting for mailbox tiles, 2: waiting for gathered
+ * tiles), [2] = the waiting rank, [3] = the flag's index, and every other wait
+ * of the launch then stops too: the call ends with the outputs incomplete
+ * instead of hanging.  A launch that finds [0] != 0 does nothing (it still
+ * advances [4]).  After a failure the flags are in an unknown state: zero the
+ * flags and the status words on every rank before the next call.
  *
  * The kernel is a cooperative launch (all its CTAs resident at once) on
  * `stream`.  Argument errors return before the launch; LPAR_ERR_UNSUPPORTED
  * for an unknown codec or a device without cooperative launch.
  * ------------------------------------------------------------------------- */
-#define LPAR_PEER_STATUS_WORDS 4
+#define LPAR_PEER_STATUS_WORDS 8
 #define LPAR_PEER_HANDLE_BYTES 64
 
 /* Buffer sizes of lpar_allreduce_peer; 0 for N outside [1, LPAR_MAX_RANKS], an
@@ -382,8 +385,8 @@ size_t lpar_peer_flag_bytes(int N, size_t n);
 
 lpar_status_t lpar_allreduce_peer(const void *const *inputs, void *const *outputs, void *const *mailboxes,
                                   void *const *gathered, void *const *flags, int N, int rank0, int ranks,
-                                  size_t n, lpar_codec_t codec, uint32_t epoch, uint64_t timeout_ns,
-                                  uint32_t *status, cudaStream_t stream);
+                                  size_t n, lpar_codec_t codec, uint64_t timeout_ns, uint32_t *status,
+                                  cudaStream_t stream);
 
 /* Buffers shared between processes (CUDA IPC), the one place the library
  * allocates: lpar_peer_alloc reserves `bytes` of device memory on the current

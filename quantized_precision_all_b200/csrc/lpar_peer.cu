@@ -32,7 +32,10 @@
 // thread issues a system-scope fence and a release store of the call's epoch
 // into the flag; a waiter polls the flag with system-scope acquire loads until
 // it reaches the epoch, then meets a CTA barrier before any thread reads the
-// data.  Epochs grow by one per call, so no flag needs resetting; a buffer is
+// data.  The epoch lives in the launching rank's status words: every CTA reads
+// the previous call's epoch when it starts and the last CTA to finish stores
+// the new one, so a call captured in a CUDA graph advances it on every replay.
+// Epochs grow by one per call, so no flag needs resetting; a buffer is
 // never rewritten before every reader of the previous call is done with it
 // (a rank enters call k+1 only after it has decoded every shard of call k,
 // and every shard of call k was reduced only after its mailbox chunks had been
@@ -40,9 +43,10 @@
 //
 // Waits are bounded: a wait that sees no progress for timeout_ns (or after
 // timeout_ns / 128 polls) records the failure in the caller's status words
-// and its CTA returns; every other wait of the launch then sees the status and
-// returns as well, so a missing rank ends the call with an error instead of a
-// hang.  Inside one launch every CTA finishes its phase-A work before its
+// and its CTA stops (the decision is taken at a CTA barrier, so all its
+// threads stop together); every other wait of the launch then sees the status
+// and stops as well, so a missing rank ends the call with an error instead of
+// a hang.  Inside one launch every CTA finishes its phase-A work before its
 // first wait and phase-B waits depend only on phase A, phase-C waits only on
 // phase B; the launch is cooperative, so all its CTAs are resident together.
 //
@@ -77,23 +81,42 @@ struct PeerGeom {
     unsigned long long timeout_ns;
     unsigned P;                        // chunks per shard
     int rank0, R;                      // the ranks this launch runs
-    uint32_t epoch;
+    int sys;                           // 1: other ranks run elsewhere (system-scope ordering)
 };
 
+// Status words (LPAR_PEER_STATUS_WORDS, in the launching GPU's memory).
+constexpr int kStFail = 0, kStPhase = 1, kStRank = 2, kStIndex = 3, kStEpoch = 4, kStDone = 5;
+
+// Chunks per shard: shards of up to ceil(T/N) tiles cut into chunks of at
+// least kPeerChunkTiles tiles, at most kPeerMaxChunks chunks.  Every flag costs
+// a CTA barrier, a fence and a wait, so a chunk should carry several tiles;
+// the ranks' shards should still give every CTA work.
 constexpr unsigned kPeerMaxChunks = 1024;
+constexpr unsigned kPeerChunkTiles = 16;
 
 inline unsigned peer_chunks(int N, size_t T) {
     const size_t s = (T + (size_t)N - 1) / (size_t)N;
-    return (unsigned)std::min<size_t>(std::max<size_t>(s, 1), kPeerMaxChunks);
+    const size_t c = (s + kPeerChunkTiles - 1) / kPeerChunkTiles;
+    return (unsigned)std::min<size_t>(std::max<size_t>(c, 1), kPeerMaxChunks);
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t *p) {
+// Flag accesses at the scope of the threads that take part: the whole system
+// when other ranks run on other GPUs, this GPU when every rank runs in this
+// launch (measured on B200: the system-scope fence makes the all-ranks launch
+// 3-4x slower at 16 MiB per rank, and buys nothing there).
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p, int sys) {
     uint32_t v;
-    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (sys) asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    else asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v, int sys) {
+    if (sys) asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    else asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence(int sys) {
+    if (sys) __threadfence_system();
+    else __threadfence();
 }
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
@@ -114,37 +137,51 @@ __device__ __forceinline__ void chunk_tiles(int j, unsigned c, int N, const Peer
 }
 
 // One thread waits until *flag has reached the epoch.  False when the wait
-// gave up (recorded in the status words: [0] = 1, [1] = phase, [2] = the
-// waiting rank, [3] = the flag's index) or another wait already had.
-__device__ bool wait_flag(const uint32_t *flag, const PeerGeom &g, uint32_t *status, uint32_t phase, int rank,
-                          uint32_t index) {
+// gave up (recorded in the status words: fail = 1, the phase, the waiting
+// rank, the flag's index) or another wait already had.
+__device__ bool wait_flag(const uint32_t *flag, uint32_t epoch, const PeerGeom &g, uint32_t *status, uint32_t phase,
+                          int rank, uint32_t index) {
     const unsigned long long t0 = globaltimer_ns();
     const unsigned long long polls = g.timeout_ns / 128 + 1024;
     for (unsigned long long k = 0; k < polls; ++k) {
-        if ((int32_t)(ld_acquire_sys(flag) - g.epoch) >= 0) return true;
+        if ((int32_t)(ld_acquire(flag, g.sys) - epoch) >= 0) return true;
         if (ld_status(status) != 0) return false;
         if (globaltimer_ns() - t0 > g.timeout_ns) break;
         __nanosleep(200);
     }
-    if (atomicCAS(status, 0u, 1u) == 0u) {
-        status[1] = phase;
-        status[2] = (uint32_t)rank;
-        status[3] = index;
+    if (atomicCAS(status + kStFail, 0u, 1u) == 0u) {
+        status[kStPhase] = phase;
+        status[kStRank] = (uint32_t)rank;
+        status[kStIndex] = index;
         __threadfence();
     }
     return false;
 }
 
+// Every CTA on every way out: the last one to finish (so every CTA has read
+// the old epoch) stores the call's epoch for the next call.
+__device__ __forceinline__ void finish(uint32_t *status, uint32_t epoch) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(status + kStDone, 1u) == gridDim.x - 1) {
+            status[kStDone] = 0;
+            *reinterpret_cast<volatile uint32_t *>(status + kStEpoch) = epoch;
+            __threadfence();
+        }
+    }
+}
+
 // After the CTA's stores: one thread publishes them with `count` flags
 // (flag k at base[k] + index).
 __device__ __forceinline__ void publish(uint32_t *const *flag_bases, int count, int first, size_t index,
-                                        uint32_t epoch) {
+                                        uint32_t epoch, int sys) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence_system();
+        fence(sys);
         for (int q = 0; q < count; ++q) {
             const int r = (first + q) % count;
-            st_release_sys(flag_bases[r] + index, epoch);
+            st_release(flag_bases[r] + index, epoch, sys);
         }
     }
 }
@@ -191,8 +228,8 @@ __device__ __forceinline__ void peer_reduce_block(const uint8_t *const *wp, size
 // Phase A: items (chunk c, owner j, rank r), c-major, so the first chunks of
 // every shard are published first.
 template <int C, int N>
-__device__ void peer_phase_a(const PeerPtrs &p, const PeerGeom &g, uint8_t (*stage)[C == kBF16 ? 16 : kStageBytes],
-                             uint8_t *wst) {
+__device__ void peer_phase_a(const PeerPtrs &p, const PeerGeom &g, uint32_t epoch,
+                             uint8_t (*stage)[C == kBF16 ? 16 : kStageBytes], uint8_t *wst) {
     constexpr size_t TB = Layout<C>::kTileBytes;
     const int t = threadIdx.x;
     const size_t per_c = (size_t)N * g.R;
@@ -237,13 +274,13 @@ __device__ void peer_phase_a(const PeerPtrs &p, const PeerGeom &g, uint8_t (*sta
                 buf ^= 1;
             }
         }
-        publish(p.flags + j, 1, 0, (size_t)r * g.P + c, g.epoch);
+        publish(p.flags + j, 1, 0, (size_t)r * g.P + c, epoch, g.sys);
     }
 }
 
 // Phase B: items (chunk c, owner j) for the launch's ranks j.
 template <int C, int N>
-__device__ bool peer_phase_b(const PeerPtrs &p, const PeerGeom &g, uint8_t *wst, uint32_t *status, int *s_fail) {
+__device__ bool peer_phase_b(const PeerPtrs &p, const PeerGeom &g, uint32_t epoch, uint8_t *wst, uint32_t *status) {
     constexpr size_t TB = Layout<C>::kTileBytes;
     const int t = threadIdx.x;
     const size_t items = (size_t)g.P * g.R;
@@ -253,10 +290,9 @@ __device__ bool peer_phase_b(const PeerPtrs &p, const PeerGeom &g, uint8_t *wst,
         size_t lo, hi, base;
         chunk_tiles(j, c, N, g, lo, hi, base);
         if (lo == hi) continue;
-        if (t < N && !wait_flag(p.flags[j] + (size_t)t * g.P + c, g, status, 1, j, (uint32_t)(t * g.P + c)))
-            *s_fail = 1;
-        __syncthreads();                                         // the N chunks are visible to every thread
-        if (*s_fail) return false;
+        const bool gave_up =
+            t < N && !wait_flag(p.flags[j] + (size_t)t * g.P + c, epoch, g, status, 1, j, (uint32_t)(t * g.P + c));
+        if (__syncthreads_or(gave_up)) return false;             // else the N chunks are visible to every thread
         const uint8_t *wp[N];
 #pragma unroll
         for (int s = 0; s < N; ++s) wp[s] = p.mbox[j] + (size_t)s * g.slot * TB;
@@ -295,14 +331,14 @@ __device__ bool peer_phase_b(const PeerPtrs &p, const PeerGeom &g, uint8_t *wst,
                     copy16(p.gath[(j + 1 + q) % N] + t0 * TB, wst, (size_t)ntl * TB);
             }
         }
-        publish(p.flags, N, j + 1, (size_t)(N + j) * g.P + c, g.epoch);
+        publish(p.flags, N, j + 1, (size_t)(N + j) * g.P + c, epoch, g.sys);
     }
     return true;
 }
 
 // Phase C: items (chunk c, owner j, rank r).
 template <int C, int N>
-__device__ void peer_phase_c(const PeerPtrs &p, const PeerGeom &g, uint8_t *stage, uint32_t *status, int *s_fail) {
+__device__ void peer_phase_c(const PeerPtrs &p, const PeerGeom &g, uint32_t epoch, uint8_t *stage, uint32_t *status) {
     constexpr size_t TB = Layout<C>::kTileBytes;
     const int t = threadIdx.x;
     const size_t per_c = (size_t)N * g.R;
@@ -314,9 +350,8 @@ __device__ void peer_phase_c(const PeerPtrs &p, const PeerGeom &g, uint8_t *stag
         chunk_tiles(j, c, N, g, lo, hi, base);
         if (lo == hi) continue;
         const size_t fi = (size_t)(N + j) * g.P + c;
-        if (t == 0 && !wait_flag(p.flags[r] + fi, g, status, 2, r, (uint32_t)fi)) *s_fail = 1;
-        __syncthreads();
-        if (*s_fail) return;
+        const bool gave_up = t == 0 && !wait_flag(p.flags[r] + fi, epoch, g, status, 2, r, (uint32_t)fi);
+        if (__syncthreads_or(gave_up)) return;
         const uint8_t *src = p.gath[r];
         uint8_t *dst = p.out[r];
         if constexpr (C == kBF16) {
@@ -345,19 +380,25 @@ __device__ void peer_phase_c(const PeerPtrs &p, const PeerGeom &g, uint8_t *stag
     }
 }
 
+// Four CTAs per SM (at most 64 registers a thread): measured on B200 with every
+// rank in one launch, 10-20% faster than the two or three CTAs per SM the
+// unbounded register counts allow, for every codec from 64 MiB per rank on.
 template <int C, int N>
-__global__ void __launch_bounds__(kThreads) k_allreduce_peer(const __grid_constant__ PeerPtrs p,
+__global__ void __launch_bounds__(kThreads, 4) k_allreduce_peer(const __grid_constant__ PeerPtrs p,
                                                              const __grid_constant__ PeerGeom g, uint32_t *status) {
     __shared__ __align__(128) uint8_t stage[2][C == kBF16 ? 16 : kStageBytes];
     __shared__ __align__(16) uint8_t wst[C == kBF16 ? 16 : kTilesPerCta * Layout<C>::kTileBytes];
-    __shared__ int s_fail;
-    if (threadIdx.x == 0) s_fail = ld_status(status) != 0;      // a failed earlier call: do nothing
-    __syncthreads();
-    if (s_fail) return;
-    peer_phase_a<C, N>(p, g, stage, wst);
-    if constexpr (C != kBF16) cp_async_wait_all_groups();
-    if (!peer_phase_b<C, N>(p, g, wst, status, &s_fail)) return;
-    peer_phase_c<C, N>(p, g, stage[0], status, &s_fail);
+    __shared__ uint32_t s_epoch;
+    if (threadIdx.x == 0) s_epoch = ld_status(status + kStEpoch) + 1u;
+    // a failed earlier call: do nothing
+    const bool failed = __syncthreads_or(threadIdx.x == 0 && ld_status(status + kStFail) != 0);
+    const uint32_t epoch = s_epoch;
+    if (!failed) {
+        peer_phase_a<C, N>(p, g, epoch, stage, wst);
+        if constexpr (C != kBF16) cp_async_wait_all_groups();
+        if (peer_phase_b<C, N>(p, g, epoch, wst, status)) peer_phase_c<C, N>(p, g, epoch, stage[0], status);
+    }
+    finish(status, epoch);
 }
 
 template <int C, int N>
@@ -424,12 +465,12 @@ LPAR_API size_t lpar_peer_flag_bytes(int N, size_t n) {
 
 LPAR_API lpar_status_t lpar_allreduce_peer(
     const void *const *inputs, void *const *outputs, void *const *mailboxes, void *const *gathered,
-    void *const *flags, int N, int rank0, int ranks, size_t n, lpar_codec_t codec, uint32_t epoch,
-    uint64_t timeout_ns, uint32_t *status, cudaStream_t stream) {
+    void *const *flags, int N, int rank0, int ranks, size_t n, lpar_codec_t codec, uint64_t timeout_ns,
+    uint32_t *status, cudaStream_t stream) {
     if (N < 1 || N > kMaxRanks || rank0 < 0 || ranks < 1 || rank0 + ranks > N) return LPAR_ERR_INVALID_ARG;
     if (!codec_ok(codec)) return LPAR_ERR_UNSUPPORTED;
     if (n % kTileElems || tiles_of(n) > kMaxTiles) return LPAR_ERR_INVALID_ARG;
-    if (!inputs || !outputs || !mailboxes || !gathered || !flags || !status || epoch == 0 || timeout_ns == 0)
+    if (!inputs || !outputs || !mailboxes || !gathered || !flags || !status || timeout_ns == 0)
         return LPAR_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(status) & 15u) return LPAR_ERR_MISALIGNED;
     PeerPtrs p{};
@@ -467,7 +508,7 @@ LPAR_API lpar_status_t lpar_allreduce_peer(
     g.P = peer_chunks(N, T);
     g.rank0 = rank0;
     g.R = ranks;
-    g.epoch = epoch;
+    g.sys = ranks < N;
     NvtxRange nvtx("lpar_allreduce_peer");
     switch (codec) {
         case LPAR_CODEC_BF16: return launch_peer_c<kBF16>(N, p, g, status, stream);

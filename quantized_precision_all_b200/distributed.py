@@ -218,7 +218,7 @@ class PeerOps:
     exportable), free(addr), export(addr) -> handle bytes, import_(handle) ->
     address, close(addr), mailbox_bytes(N, n, codec), gather_bytes(n, codec),
     flag_bytes(N, n), and run(inputs, outputs, mailboxes, gathered, flags, n,
-    codec, epoch, timeout_ns, status, rank0, ranks) for lpar_allreduce_peer."""
+    codec, timeout_ns, status, rank0, ranks) for lpar_allreduce_peer."""
     alloc: Callable
     free: Callable
     export: Callable
@@ -243,9 +243,10 @@ def _align(x, a=256):
 
 class _PeerRegion:
     """One rank's exportable region for one (n, codec) -- mailbox, gathered
-    wire, flags -- and the addresses of every rank's region in this process."""
+    wire, flags -- the addresses of every rank's region in this process, and
+    the status words of the calls on it (which carry their epoch)."""
 
-    def __init__(self, ops, group, N, me, n, codec):
+    def __init__(self, ops, group, N, me, n, codec, device):
         self.ops = ops
         sizes = [ops.mailbox_bytes(N, n, codec), ops.gather_bytes(n, codec), ops.flag_bytes(N, n)]
         self.offsets = [0, _align(sizes[0]), _align(sizes[0]) + _align(sizes[1])]
@@ -254,7 +255,7 @@ class _PeerRegion:
         dist.all_gather_object(handles, ops.export(self.local), group=group)
         self.bases = [self.local if r == me else ops.import_(handles[r]) for r in range(N)]
         self.me = me
-        self.epoch = 0
+        self.status = torch.zeros(L.LPAR_PEER_STATUS_WORDS, dtype=torch.int32, device=device)
 
     def pointers(self, k):
         return [b + self.offsets[k] for b in self.bases]
@@ -273,7 +274,7 @@ class PeerAllreduce:
     size, codec) on first use; the regions' handles are exchanged over the
     process group and mapped in every process.  A call is one launch on this
     rank's GPU that runs this rank only; every rank must make the same calls in
-    the same order (each call's epoch is counted per region).  The ranks' GPUs
+    the same order (the calls on a region are counted by its epoch).  The ranks' GPUs
     must be distinct: the library refuses peers whose memory is this GPU's.
     `check()` synchronises and raises when a wait for another rank gave up
     (after timeout_ns without progress)."""
@@ -285,16 +286,15 @@ class PeerAllreduce:
         self.rank = dist.get_rank(group)
         self.ops = ops if ops is not None else cuda_peer_ops()
         self.timeout_ns = int(timeout_ns)
-        dev = device if device is not None else (torch.device("cuda", torch.cuda.current_device())
-                                                 if torch.cuda.is_available() else torch.device("cpu"))
-        self.status = torch.zeros(L.LPAR_PEER_STATUS_WORDS, dtype=torch.int32, device=dev)
+        self.device = device if device is not None else (torch.device("cuda", torch.cuda.current_device())
+                                                         if torch.cuda.is_available() else torch.device("cpu"))
         self._regions: Dict[tuple, _PeerRegion] = {}
 
     def region(self, n: int, codec: str) -> _PeerRegion:
         key = (n, codec)
         reg = self._regions.get(key)
         if reg is None:
-            reg = _PeerRegion(self.ops, self.group, self.N, self.rank, n, codec)
+            reg = _PeerRegion(self.ops, self.group, self.N, self.rank, n, codec, self.device)
             self._regions[key] = reg
         return reg
 
@@ -310,24 +310,29 @@ class PeerAllreduce:
         if n == 0:
             return out
         reg = self.region(n, codec)
-        reg.epoch += 1
         ins = [x if r == self.rank else None for r in range(self.N)]
         outs = [out if r == self.rank else None for r in range(self.N)]
-        self.ops.run(ins, outs, reg.pointers(0), reg.pointers(1), reg.pointers(2), n, codec, reg.epoch,
-                     self.timeout_ns, self.status, rank0=self.rank, ranks=1)
+        self.ops.run(ins, outs, reg.pointers(0), reg.pointers(1), reg.pointers(2), n, codec, self.timeout_ns,
+                     reg.status, rank0=self.rank, ranks=1)
         return out
 
     def check(self):
-        w = [int(v) for v in self.status.cpu()]
-        if w[0]:
-            raise L.PeerTimeout("rank %d: a wait gave up (phase %d, waiting rank %d, flag %d)"
-                                % (self.rank, w[1], w[2], w[3]))
+        """Synchronise and raise PeerTimeout if a wait of any call gave up."""
+        for key in sorted(self._regions):
+            w = [int(v) for v in self._regions[key].status.cpu()]
+            if w[0]:
+                raise L.PeerTimeout("rank %d: a wait gave up (phase %d, waiting rank %d, flag %d)"
+                                    % (self.rank, w[1], w[2], w[3]))
+
+    def epochs(self):
+        """{(n, codec): epoch of the last call} (synchronises)."""
+        return {key: int(reg.status[4]) & 0xFFFFFFFF for key, reg in self._regions.items()}
 
     def release(self):
         """Unmap the peers' regions and free this rank's (collective: every rank
         calls it; no call may be in flight)."""
-        if torch.cuda.is_available() and self.status.is_cuda:
-            torch.cuda.synchronize(self.status.device)
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
         for key in sorted(self._regions):
             self._regions[key].release(self.group)
         self._regions.clear()

@@ -38,7 +38,7 @@ EXPORTS = ("lpar_tile_bytes", "lpar_wire_bytes", "lpar_workspace_bytes", "lpar_q
            "lpar_allreduce_peer", "lpar_peer_alloc", "lpar_peer_free", "lpar_peer_export", "lpar_peer_import",
            "lpar_peer_close")
 LPAR_STATIC_WORKSPACE_BYTES = 16 << 20
-LPAR_PEER_STATUS_WORDS = 4
+LPAR_PEER_STATUS_WORDS = 8
 LPAR_PEER_HANDLE_BYTES = 64
 
 
@@ -80,8 +80,7 @@ def _load():
         "lpar_peer_mailbox_bytes": (sz, [i32, sz, i32]),
         "lpar_peer_gather_bytes": (sz, [sz, i32]),
         "lpar_peer_flag_bytes": (sz, [i32, sz]),
-        "lpar_allreduce_peer": (i32, [vpp, vpp, vpp, vpp, vpp, i32, i32, i32, sz, i32, ctypes.c_uint32,
-                                      ctypes.c_uint64, vp, vp]),
+        "lpar_allreduce_peer": (i32, [vpp, vpp, vpp, vpp, vpp, i32, i32, i32, sz, i32, ctypes.c_uint64, vp, vp]),
         "lpar_peer_alloc": (i32, [sz, vpp]),
         "lpar_peer_free": (i32, [vp]),
         "lpar_peer_export": (i32, [vp, ctypes.c_char_p]),
@@ -291,17 +290,18 @@ def _addr(x):
     return x.data_ptr()
 
 
-def lpar_allreduce_peer(inputs, outputs, mailboxes, gathered, flags, n, codec, epoch, timeout_ns, status,
-                        rank0=0, ranks=None, stream=None):
+def lpar_allreduce_peer(inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0=0,
+                        ranks=None, stream=None):
     """inputs/outputs: N entries (None outside the launch's ranks); mailboxes,
     gathered, flags: N buffers (tensors or addresses, on this GPU or reachable
-    from it); status: LPAR_PEER_STATUS_WORDS words of this GPU's memory."""
+    from it); status: LPAR_PEER_STATUS_WORDS words of this GPU's memory (word 4
+    carries the epoch from call to call)."""
     N = len(mailboxes)
     ranks = N - rank0 if ranks is None else ranks
     _check(_lib.lpar_allreduce_peer(_ptr_array(inputs, _addr), _ptr_array(outputs, _addr),
                                     _ptr_array(mailboxes, _addr), _ptr_array(gathered, _addr),
-                                    _ptr_array(flags, _addr), N, rank0, ranks, n, _codec(codec), epoch,
-                                    int(timeout_ns), _ptr(status), _stream(stream)), "lpar_allreduce_peer")
+                                    _ptr_array(flags, _addr), N, rank0, ranks, n, _codec(codec), int(timeout_ns),
+                                    _ptr(status), _stream(stream)), "lpar_allreduce_peer")
 
 
 def lpar_peer_alloc(nbytes):
@@ -471,9 +471,9 @@ class PeerTimeout(RuntimeError):
 
 class PeerBuffers:
     """The buffers of lpar_allreduce_peer for N ranks that all live on one GPU
-    (mailboxes, gathered wires and flags as torch tensors, zeroed), the status
-    words and the epoch counter.  One set serves any number of calls of the
-    same (N, n, codec) in stream order."""
+    (mailboxes, gathered wires and flags as torch tensors, zeroed) and the
+    status words.  One set serves any number of calls of the same (N, n,
+    codec) in stream order, CUDA graph replays included."""
 
     def __init__(self, N, n, codec, device=None):
         import torch
@@ -484,19 +484,21 @@ class PeerBuffers:
         self.gathered = [torch.zeros(max(lpar_peer_gather_bytes(n, codec), 16), **u8) for _ in range(N)]
         self.flags = [torch.zeros(max(lpar_peer_flag_bytes(N, n), 16), **u8) for _ in range(N)]
         self.status = torch.zeros(LPAR_PEER_STATUS_WORDS, dtype=torch.int32, device=dev)
-        self.epoch = 0
 
     def allreduce(self, inputs, out, timeout_ns=1_000_000_000, stream=None):
-        self.epoch += 1
-        lpar_allreduce_peer(inputs, out, self.mailboxes, self.gathered, self.flags, self.n, self.codec, self.epoch,
-                            timeout_ns, self.status, 0, self.N, stream)
+        lpar_allreduce_peer(inputs, out, self.mailboxes, self.gathered, self.flags, self.n, self.codec, timeout_ns,
+                            self.status, 0, self.N, stream)
         return out
+
+    def epoch(self):
+        """Synchronise and return the epoch of the last call."""
+        return int(self.status[4].item()) & 0xFFFFFFFF
 
     def check(self):
         """Synchronise and raise PeerTimeout if a wait gave up."""
         w = [int(v) for v in self.status.cpu()]
         if w[0]:
-            raise PeerTimeout("lpar_allreduce_peer: a wait gave up (phase %d, rank %d, flag %d)" % tuple(w[1:]))
+            raise PeerTimeout("lpar_allreduce_peer: a wait gave up (phase %d, rank %d, flag %d)" % tuple(w[1:4]))
 
 
 def allreduce_peer(inputs, codec, out=None, buffers=None, timeout_ns=1_000_000_000, stream=None):

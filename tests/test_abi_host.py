@@ -278,10 +278,12 @@ def test_peer_buffer_bytes(L):
     assert L.lpar_peer_mailbox_bytes(1, n, "mxfp4") == 10 * 1088
     assert L.lpar_peer_gather_bytes(n, "int3") == 10 * 896
     assert L.lpar_peer_gather_bytes(n, "fp8") == 10 * 2304
-    assert L.lpar_peer_flag_bytes(3, n) == 2 * 3 * 4 * 4                  # P = ceil(10 / 3) chunks per shard
+    # P = min(ceil(ceil(T / N) / 16), 1024) chunks per shard (chunks of at least 16 tiles)
+    assert L.lpar_peer_flag_bytes(3, n) == 2 * 3 * 1 * 4
     assert L.lpar_peer_flag_bytes(8, 2048 << 20) == 2 * 8 * 1024 * 4      # P capped at 1024
-    assert L.lpar_peer_flag_bytes(8, 2048 * 8 * 1024) == 2 * 8 * 1024 * 4
-    assert L.lpar_peer_flag_bytes(8, 2048 * (8 * 1024 - 8)) == 2 * 8 * 1023 * 4
+    assert L.lpar_peer_flag_bytes(8, 2048 * 8 * 1024) == 2 * 8 * 64 * 4
+    assert L.lpar_peer_flag_bytes(8, 2048 * (8 * 16 * 1000 + 1)) == 2 * 8 * 1001 * 4
+    assert L.lpar_peer_flag_bytes(2, 2048 * 33) == 2 * 2 * 2 * 4
     for bad in (L.lpar_peer_mailbox_bytes(0, n, "int4"), L.lpar_peer_mailbox_bytes(9, n, "int4"),
                 L.lpar_peer_mailbox_bytes(2, n + 1, "int4"), L.lpar_peer_mailbox_bytes(2, n, 7),
                 L.lpar_peer_gather_bytes(n + 2, "int4"), L.lpar_peer_gather_bytes(n, 9),
@@ -293,11 +295,10 @@ def test_argument_errors_allreduce_peer(L):
     n = 2048 * 4
 
     def call(inputs=(A, A), outputs=(A, A), mailboxes=(A, A), gathered=(A, A), flags=(A, A), n=n, codec="int4",
-             epoch=1, timeout_ns=10 ** 6, status=A, rank0=0, ranks=None):
+             timeout_ns=10 ** 6, status=A, rank0=0, ranks=None):
         return status_of(L.lpar_allreduce_peer, list(inputs), list(outputs), list(mailboxes), list(gathered),
-                         list(flags), n, codec, epoch, timeout_ns, status, rank0=rank0, ranks=ranks, stream=0)
+                         list(flags), n, codec, timeout_ns, status, rank0=rank0, ranks=ranks, stream=0)
 
-    assert call(epoch=0) == 1
     assert call(timeout_ns=0) == 1
     assert call(status=0) == 1
     assert call(status=M) == 2
@@ -315,7 +316,7 @@ def test_argument_errors_allreduce_peer(L):
     assert call(n=0) == 0                                # a no-op, nothing launched
     assert call(inputs=(A, None), outputs=(A, None), ranks=1, n=0) == 0   # rank 1 outside: no input needed
     lib = L.library()
-    assert lib.lpar_allreduce_peer(None, None, None, None, None, 2, 0, 2, n, 2, 1, 10, A, None) == 1
+    assert lib.lpar_allreduce_peer(None, None, None, None, None, 2, 0, 2, n, 2, 10, A, None) == 1
 
 
 def test_peer_ipc_argument_errors(L):

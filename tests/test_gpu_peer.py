@@ -46,16 +46,16 @@ class Bufs:
         self.mbox = [Guarded(L.lpar_peer_mailbox_bytes(N, n, codec), fill=0) for _ in range(N)]
         self.gath = [Guarded(L.lpar_peer_gather_bytes(n, codec), fill=0) for _ in range(N)]
         self.flags = [Guarded(L.lpar_peer_flag_bytes(N, n), fill=0) for _ in range(N)]
-        self.status = torch.zeros(4, dtype=torch.int32, device="cuda")
+        self.status = torch.zeros(8, dtype=torch.int32, device="cuda")
         self.epoch = 0
 
     def call(self, L, ins, outs):
         self.epoch += 1
         L.lpar_allreduce_peer([g.ptr() for g in ins], [g.ptr() for g in outs], [g.ptr() for g in self.mbox],
                               [g.ptr() for g in self.gath], [g.ptr() for g in self.flags], self.n, self.codec,
-                              self.epoch, TIMEOUT_NS, self.status)
+                              TIMEOUT_NS, self.status)
         torch.cuda.synchronize()
-        assert self.status.tolist() == [0, 0, 0, 0]
+        assert self.status.tolist() == [0, 0, 0, 0, self.epoch, 0, 0, 0]   # the launch advanced the epoch
         for g in self.mbox + self.gath + self.flags:
             g.check()
         flags = [g.host().view(np.uint32) for g in self.flags]
@@ -124,24 +124,61 @@ def test_peer_repeated_calls_reuse_the_buffers_and_in_place(L, codec):
             assert np.array_equal(host_u16(o), ref[0]), (codec, k)
 
 
+@pytest.mark.parametrize("codec", ["int4", "fp8", "bf16"])
+def test_peer_calls_replayed_from_a_cuda_graph(L, codec):
+    """The epoch lives in the status words, so one captured launch replayed
+    five times (new inputs copied in before each replay) gives the oracle's
+    result every time and advances the epoch by one per replay."""
+    N, tiles = 4, 13
+    n = tiles * 2048
+    ins = [torch.zeros(n, dtype=torch.bfloat16, device="cuda") for _ in range(N)]
+    outs = [torch.zeros(n, dtype=torch.bfloat16, device="cuda") for _ in range(N)]
+    buf = L.PeerBuffers(N, n, codec)
+    buf.allreduce(ins, outs)                              # warm-up outside the capture (epoch 1)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            buf.allreduce(ins, outs)
+    torch.cuda.synchronize()
+    for k in range(5):
+        xs = inputs(N, n, 8900 + 10 * k)
+        for d, x in zip(ins, xs):
+            d.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        buf.check()
+        assert buf.epoch() == 2 + k
+        ref, _ = O.allreduce(xs, codec)
+        for o in outs:
+            assert np.array_equal(o.view(torch.int16).cpu().numpy().view(np.uint16), ref[0]), (codec, k)
+    del graph
+
+
+def chunks_per_shard(N, T):
+    """min(ceil(ceil(T / N) / 16), 1024): chunks of at least 16 tiles."""
+    return min(max(-(-(-(-T // N)) // 16), 1), 1024)
+
+
 def sampled(xs_dev, tiles):
     idx = torch.from_numpy((tiles[:, None] * 2048 + np.arange(2048)[None, :]).reshape(-1)).cuda()
     return idx, [x[idx].view(torch.int16).cpu().numpy().view(np.uint16) for x in xs_dev]
 
 
 @pytest.mark.parametrize("codec", ["int4", "int3", "fp8", "mxfp4", "bf16"])
-@pytest.mark.parametrize("N,T", [(2, 4099), (5, 5 * 3 * 1024 + 7), (8, 1024 * 8 + 2)])
+@pytest.mark.parametrize("N,T", [(2, 4099), (5, 5 * 3 * 1024 + 7), (8, 1024 * 8 + 2), (2, 2 * 16 * 1024 + 6)])
 def test_peer_many_tile_chunks(L, codec, N, T):
-    """Shards of more than 1024 tiles (the chunk count's cap), so chunks hold
-    several tiles and are ragged; every chunk boundary of shard 0 and 1 and 256
-    random tiles compared with the oracle, and the whole of rank 0's output with
-    lpar_allreduce's."""
+    """Shards cut into many chunks of 16 or more tiles, ragged (the last case
+    at the cap of 1024 chunks per shard); every chunk boundary of shard 0 and 1
+    and 256 random tiles compared with the oracle, and the whole of rank 0's
+    output with lpar_allreduce's."""
     n = T * 2048
     xs = [to_device(x) for x in inputs(N, n, 8400 + N)]
     outs = [Guarded(2 * n, fill=0) for _ in range(N)]
     b = Bufs(L, N, n, codec)
     b.call(L, xs, outs)
-    P = min(-(-T // N), 1024)
+    P = chunks_per_shard(N, T)
     bounds = []
     for j in (0, 1):
         base, S = j * T // N, (j + 1) * T // N - j * T // N
@@ -199,18 +236,19 @@ def test_peer_wait_gives_up_on_a_rank_that_never_runs(L):
     host = [torch.zeros(max(k, 16), dtype=torch.uint8, pin_memory=True)
             for k in (L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
                       L.lpar_peer_flag_bytes(N, n))]
-    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    status = torch.zeros(8, dtype=torch.int32, device="cuda")
     timeout = 50_000_000                                  # 50 ms
     t0 = time.perf_counter()
     L.lpar_allreduce_peer([x0.ptr(), None], [out0.ptr(), None], [mb0.ptr(), host[0].data_ptr()],
-                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, 1, timeout,
+                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, timeout,
                           status, rank0=0, ranks=1)
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
     w = status.tolist()
-    P = min(-(-tiles // N), 1024)
+    P = chunks_per_shard(N, tiles)
     assert w[0] == 1 and w[1] == 1 and w[2] == 0, w       # phase 1 (mailbox), waiting rank 0
     assert P <= w[3] < 2 * P, w                            # a flag of source 1
+    assert w[4:] == [1, 0, 0, 0], w                        # epoch 1 done, every CTA accounted for
     assert elapsed < 5.0, elapsed
     for g in (out0, mb0, ga0, fl0):
         g.check()
@@ -222,10 +260,11 @@ def test_peer_wait_gives_up_on_a_rank_that_never_runs(L):
     # a launch that finds the status set does nothing
     out1 = Guarded(2 * n, fill=0x33)
     L.lpar_allreduce_peer([x0.ptr(), None], [out1.ptr(), None], [mb0.ptr(), host[0].data_ptr()],
-                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, 2, timeout,
+                          [ga0.ptr(), host[1].data_ptr()], [fl0.ptr(), host[2].data_ptr()], n, codec, timeout,
                           status, rank0=0, ranks=1)
     torch.cuda.synchronize()
     assert np.all(out1.host() == 0x33)
+    assert status.tolist()[:5] == w[:4] + [2]
     # the context is intact: a normal all-reduce of both ranks
     out = L.allreduce_peer([torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) for x in xs], codec)
     torch.cuda.synchronize()
@@ -243,13 +282,13 @@ def test_peer_refuses_an_absent_rank_on_this_device(L):
             for k in (L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
                       L.lpar_peer_flag_bytes(N, n))] * 2
     x = torch.zeros(n, dtype=torch.bfloat16, device="cuda")
-    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    status = torch.zeros(8, dtype=torch.int32, device="cuda")
     with pytest.raises(L.LparError) as e:
         L.lpar_allreduce_peer([x, None], [x, None], [bufs[0], bufs[3]], [bufs[1], bufs[4]], [bufs[2], bufs[5]], n,
-                              codec, 1, TIMEOUT_NS, status, rank0=0, ranks=1)
+                              codec, TIMEOUT_NS, status, rank0=0, ranks=1)
     assert e.value.status == 1
     torch.cuda.synchronize()
-    assert status.tolist() == [0, 0, 0, 0]
+    assert status.tolist() == [0] * 8
 
 
 # ---------------------------------------------------------------------------
@@ -290,9 +329,9 @@ def _ipc_worker(rank, world, port, n, codec, q):
         dist.all_gather_object(handles, L.lpar_peer_export(region))
         if rank == 0:
             bases = [region] + [L.lpar_peer_import(h) for h in handles[1:]]
-            status = torch.zeros(4, dtype=torch.int32, device="cuda")
+            status = torch.zeros(8, dtype=torch.int32, device="cuda")
             ptr = lambda k: [b + offs[k] for b in bases]
-            L.lpar_allreduce_peer(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), n, codec, 1, TIMEOUT_NS, status)
+            L.lpar_allreduce_peer(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), n, codec, TIMEOUT_NS, status)
             torch.cuda.synchronize()
             st = status.tolist()
             for b in bases[1:]:
@@ -331,7 +370,7 @@ def test_peer_buffers_shared_by_ipc(world, tiles, codec):
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    assert got[0][1] == [0, 0, 0, 0]
+    assert got[0][1] == [0, 0, 0, 0, 1, 0, 0, 0]
     ref, _ = O.allreduce(inputs(world, n, 8800), codec)
     for r in range(world):
         assert np.array_equal(got[r][0].view(np.uint16), ref[0]), r

@@ -80,13 +80,19 @@ class ShmOps:
         flags = self.view(addr)[:8 * 4 * 2].view(np.uint32)
         while int(flags[index]) < epoch:
             if time.monotonic() > deadline:
-                status[:] = torch.tensor([1, phase, rank, index], dtype=torch.int32)
+                status[:4] = torch.tensor([1, phase, rank, index], dtype=torch.int32)
                 return False
             time.sleep(0.0005)
         return True
 
-    def run(self, inputs, outputs, mailboxes, gathered, flags, n, codec, epoch, timeout_ns, status, rank0, ranks):
+    def run(self, inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0, ranks):
         assert ranks == 1 and inputs[rank0] is not None and all(x is None for i, x in enumerate(inputs) if i != rank0)
+        epoch = int(status[4]) + 1
+        if int(status[0]) == 0:
+            self._run(inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0, epoch)
+        status[4] = epoch
+
+    def _run(self, inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0, epoch):
         N, r, T, tb = len(mailboxes), rank0, n // 2048, O.tile_bytes(codec)
         slot = -(-T // N)
         shard = [(j * T // N, (j + 1) * T // N) for j in range(N)]
@@ -130,7 +136,7 @@ def _worker(rank, world, port, codec, q):
             out = ar.allreduce(x, codec)
             ar.check()
             results.append(out.view(torch.int16).numpy().copy())
-        epochs = {key: reg.epoch for key, reg in ar._regions.items()}
+        epochs = ar.epochs()
         ar.release()
         assert not ops.blocks, "every mapping closed and the own regions freed"
         q.put((rank, results, epochs))
@@ -191,9 +197,10 @@ def _absent_worker(rank, world, port, q):
                 ar.check()
             except L.PeerTimeout as e:
                 err = str(e)
+        status = ar.region(n, "int4").status.tolist()
         dist.barrier()
         ar.release()
-        q.put((rank, err, ar.status.tolist()))
+        q.put((rank, err, status))
     finally:
         dist.destroy_process_group()
 
