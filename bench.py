@@ -426,18 +426,31 @@ def nvlink_bytes_sent(world, n, codec, chunks, rank=0):
     return total
 
 
+def peer_bytes_sent(world, n, codec, rank=0):
+    """Wire bytes one rank stores into other ranks' memory in one peer-kernel
+    all-reduce: its wire tiles of the other ranks' shards, and its reduced
+    shard into every other rank's gathered wire (the flags aside)."""
+    from quantized_precision_all_b200 import distributed as D
+    tb = int(round(CODEC_C[codec] * TILE))
+    T = n // TILE
+    a, b = D.shard_tiles(world, T)[rank]
+    return (T - (b - a)) * tb + (world - 1) * (b - a) * tb
+
+
 def run_distributed(args, rank, world, device):
     """The real all-reduce across the `world` processes (one GPU each): rank r
     holds rank r's message of the workload (same size, same seeded recipe);
-    each step runs every codec of the workload through DistributedAllreduce."""
-    from quantized_precision_all_b200.distributed import DistributedAllreduce
+    each step runs every codec of the workload through DistributedAllreduce
+    (--exchange nccl) or PeerAllreduce (--exchange peer)."""
+    from quantized_precision_all_b200.distributed import DistributedAllreduce, PeerAllreduce
     w = W.WORKLOADS[args.workload]
     if w.dtype != "bf16":
         raise SystemExit("the cross-GPU all-reduce takes BF16 messages")
     n = w.n
     x = W.make_rank_input(w, rank, device)
     out = torch.empty_like(x)
-    ar = DistributedAllreduce(chunks=args.chunks)
+    peer = args.exchange == "peer"
+    ar = PeerAllreduce(device=device) if peer else DistributedAllreduce(chunks=args.chunks)
     stream = torch.cuda.current_stream(device)
 
     def step():
@@ -462,12 +475,17 @@ def run_distributed(args, rank, world, device):
     def eff(c):
         return c if c == "bf16" or 2 * n >= w.min_quant_bytes else "bf16"
 
-    sent = sum(nvlink_bytes_sent(world, n, eff(c), args.chunks, rank) for c in w.codecs)
-    launches = 0
-    from quantized_precision_all_b200 import distributed as D
-    for c in w.codecs:
-        for t0, t1 in D.chunk_tiles(n // TILE, args.chunks):
-            launches += 2 + sum(1 for a, b in D.shard_tiles(world, t1 - t0) if b > a)
+    if peer:
+        ar.check()
+        sent = sum(peer_bytes_sent(world, n, eff(c), rank) for c in w.codecs)
+        launches = len(w.codecs)
+    else:
+        sent = sum(nvlink_bytes_sent(world, n, eff(c), args.chunks, rank) for c in w.codecs)
+        launches = 0
+        from quantized_precision_all_b200 import distributed as D
+        for c in w.codecs:
+            for t0, t1 in D.chunk_tiles(n // TILE, args.chunks):
+                launches += 2 + sum(1 for a, b in D.shard_tiles(world, t1 - t0) if b > a)
 
     e2e = None
     if not args.no_e2e:
@@ -495,12 +513,12 @@ def run_distributed(args, rank, world, device):
         per = 2 * n * len(w.codecs)
         e2e = {"value": aggregate_gbs(world, per, e2e_steps, e_ms), "unit": "GB/s", "h2d_bytes_per_step": per,
                "d2h_bytes_per_step": per, "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
-               "api": "DistributedAllreduce.allreduce, each rank's message uploaded from pinned host memory and "
-                      "its result downloaded, per codec"}
+               "api": "%s.allreduce, each rank's message uploaded from pinned host memory and its result "
+                      "downloaded, per codec" % type(ar).__name__}
         del h_in, h_out
     ar.release()
     return {"ms": ms_max, "clocks": clocks.summary(), "sent": sent, "launches_per_step": launches, "e2e": e2e,
-            "w": w}
+            "w": w, "exchange": args.exchange}
 
 
 def oracle_codecs(w):
@@ -905,11 +923,15 @@ def workload_config(w, args, world=1):
            if w.N * w.message_bytes > 126e6 else "inputs fit in L2",
            "parallelism": "the %d ranks simulated in one GPU's HBM (emulated reduce-scatter / all-gather)" % w.N}
     if world > 1:
-        cfg.update({"simulated_ranks": None, "ranks": world,
+        peer = getattr(args, "exchange", "nccl") == "peer"
+        cfg.update({"simulated_ranks": None, "ranks": world, "exchange": "peer" if peer else "nccl",
                     "l2": "message %d MiB per rank > 126 MB L2: no flush between steps" % (w.message_bytes >> 20),
-                    "parallelism": "real all-reduce across %d GPUs, one rank per GPU: the library's stage kernels "
-                                   "with %s all-to-all and all-gather of the wire bytes, %d chunk(s) pipelined"
-                                   % (world, args.backend.upper(), args.chunks)})
+                    "parallelism": ("real all-reduce across %d GPUs, one rank per GPU: one peer-memory kernel per "
+                                    "rank storing wire tiles into the other ranks' memory over CUDA IPC" % world)
+                    if peer else
+                    ("real all-reduce across %d GPUs, one rank per GPU: the library's stage kernels with %s "
+                     "all-to-all and all-gather of the wire bytes, %d chunk(s) pipelined"
+                     % (world, args.backend.upper(), args.chunks))})
     return cfg
 
 
@@ -923,6 +945,9 @@ def main():
     ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_stage", "single_pass"])
     ap.add_argument("--chunks", type=int, default=4,
                     help="with --gpus > 1: tile ranges pipelined through the cross-GPU all-reduce")
+    ap.add_argument("--exchange", choices=["nccl", "peer"], default="nccl",
+                    help="with --gpus > 1: NCCL exchanges between the stage kernels (DistributedAllreduce) or "
+                         "one peer-memory kernel per rank over CUDA IPC (PeerAllreduce; GPUs must be distinct)")
     ap.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
                     help="with --gpus > 1: the process group's backend (gloo moves the wire bytes through host "
                          "copies; for testing the multi-rank path on fewer GPUs than ranks)")
@@ -999,7 +1024,9 @@ def distributed_line(args, world, res):
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, args, world),
-        "roofline": {"bound": "nvlink", "kernel": "whole step (stage kernels and NCCL exchanges)",
+        "roofline": {"bound": "nvlink", "kernel": ("whole step (one peer-memory kernel per codec)"
+                                                   if res["exchange"] == "peer" else
+                                                   "whole step (stage kernels and NCCL exchanges)"),
                      "achieved": achieved, "peak": NVLINK_GBS, "unit": "GB/s", "frac": achieved / NVLINK_GBS,
                      "traffic": None, "algorithmic_bytes_per_step": res["sent"],
                      "peak_source": "measured peer copy per direction per GPU on this pool (not MEASURED_PEAKS.json)"},

@@ -68,6 +68,20 @@ def test_collective_bytes():
     assert bench.collective_bytes("all_gather", "int3", N, m) == pytest.approx(N * m * (2 + c) + 2 * N * N * m)
     assert bench.collective_bytes("all_to_all", "int3", N, m) == pytest.approx(N * N * m * (2 + c) + 2 * N * N * m)
     assert bench.collective_bytes("all_gather", "bf16", N, m) == N * 2 * m + 2 * N * N * m
+    # the peer-memory all-reduce in one GPU: inputs, mailboxes written and read, N gathered
+    # copies written and read, outputs
+    assert bench.collective_bytes("peer_allreduce", "int3", N, m) == pytest.approx(
+        N * 2 * m + N * m * c + N * m * c + N * m * c + N * m * c + N * 2 * m)
+    assert bench.collective_bytes("peer_allreduce", "bf16", N, m) == N * m * 12
+
+
+def test_peer_bytes_sent():
+    """Per rank: its wire tiles of the other shards, and its reduced shard to the N - 1 others."""
+    T, tb = 10, 896
+    n = T * 2048
+    assert bench.peer_bytes_sent(3, n, "int3", 0) == (10 - 3) * tb + 2 * 3 * tb     # shard 0 = tiles [0, 3)
+    assert bench.peer_bytes_sent(3, n, "int3", 2) == (10 - 4) * tb + 2 * 4 * tb     # shard 2 = tiles [6, 10)
+    assert bench.peer_bytes_sent(1, n, "int4", 0) == 0
 
 
 def test_single_pass_labels_follow_the_launcher_rule():
