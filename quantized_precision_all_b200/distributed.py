@@ -275,9 +275,10 @@ class PeerAllreduce:
     process group and mapped in every process.  A call is one launch on this
     rank's GPU that runs this rank only; every rank must make the same calls in
     the same order (the calls on a region are counted by its epoch).  The ranks' GPUs
-    must be distinct: the library refuses peers whose memory is this GPU's.
-    `check()` synchronises and raises when a wait for another rank gave up
-    (after timeout_ns without progress)."""
+    must be distinct: construction (a collective call) compares the ranks'
+    GPU UUIDs and raises ValueError when two ranks share a GPU.  `check()`
+    synchronises and raises when a wait for another rank gave up (after
+    timeout_ns without progress)."""
 
     def __init__(self, group=None, ops: Optional[PeerOps] = None, timeout_ns: int = 2_000_000_000,
                  device=None):
@@ -289,6 +290,13 @@ class PeerAllreduce:
         self.device = device if device is not None else (torch.device("cuda", torch.cuda.current_device())
                                                          if torch.cuda.is_available() else torch.device("cpu"))
         self._regions: Dict[tuple, _PeerRegion] = {}
+        if self.device.type == "cuda":
+            uuids = [None] * self.N
+            dist.all_gather_object(uuids, str(torch.cuda.get_device_properties(self.device).uuid), group=group)
+            for r in range(self.N):
+                if uuids.index(uuids[r]) != r:
+                    raise ValueError("PeerAllreduce needs one GPU per rank: ranks %d and %d share GPU %s"
+                                     % (uuids.index(uuids[r]), r, uuids[r]))
 
     def region(self, n: int, codec: str) -> _PeerRegion:
         key = (n, codec)

@@ -374,3 +374,38 @@ def test_peer_buffers_shared_by_ipc(world, tiles, codec):
     ref, _ = O.allreduce(inputs(world, n, 8800), codec)
     for r in range(world):
         assert np.array_equal(got[r][0].view(np.uint16), ref[0]), r
+
+
+def _shared_gpu_worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        from quantized_precision_all_b200.distributed import PeerAllreduce
+        try:
+            PeerAllreduce()
+            q.put((rank, None))
+        except ValueError as e:
+            q.put((rank, str(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_allreduce_refuses_ranks_that_share_a_gpu():
+    """Two processes on the one GPU: PeerAllreduce's construction sees the same
+    GPU UUID twice and raises on both ranks before anything is allocated."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shared_gpu_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=300) for _ in range(2))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in range(2):
+        assert got[r] is not None and "share GPU" in got[r], got
