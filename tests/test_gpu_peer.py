@@ -156,6 +156,30 @@ def test_peer_calls_replayed_from_a_cuda_graph(L, codec):
     del graph
 
 
+@pytest.mark.parametrize("case", range(24))
+def test_peer_random_cases(L, case):
+    """Seeded random cases over codec, N in 1..8, 1..700 tiles, in place or not,
+    adversarial or scaled Gaussian inputs per rank; two calls on one set of
+    buffers; every output bit for bit against the oracle."""
+    rng = np.random.default_rng(8950 + case)
+    codec = CODECS[rng.integers(len(CODECS))]
+    N = int(rng.integers(1, 9))
+    tiles = int(rng.integers(1, 701))
+    n = tiles * 2048
+    inplace = bool(rng.integers(2))
+    b = Bufs(L, N, n, codec)
+    for k in range(2):
+        xs = [adversarial_bf16(n, int(rng.integers(1 << 30))) if rng.integers(2)
+              else random_bf16(n, int(rng.integers(1 << 30)), float(2.0 ** rng.integers(-8, 9))) for _ in range(N)]
+        ins = [to_device(x) for x in xs]
+        outs = ins if inplace else [Guarded(2 * n, fill=0) for _ in range(N)]
+        b.call(L, ins, outs)
+        ref, _ = O.allreduce(xs, codec)
+        for o in outs:
+            o.check()
+            assert np.array_equal(host_u16(o), ref[0]), (codec, N, tiles, inplace, k)
+
+
 def chunks_per_shard(N, T):
     """min(ceil(ceil(T / N) / 16), 1024): chunks of at least 16 tiles."""
     return min(max(-(-(-(-T // N)) // 16), 1), 1024)
