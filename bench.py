@@ -409,7 +409,21 @@ def run_ours(args, device):
     cpu = None if args.no_cpu_baseline else cpu_baseline(w, xs)
 
     return {"ms": ms_total, "kern": kern, "clocks": clocks.summary(), "launches_per_step": launches_per_step,
-            "e2e": e2e, "cpu": cpu, "w": w, "accuracy": accuracy, "sets": R}
+            "e2e": e2e, "cpu": cpu, "w": w, "accuracy": accuracy, "sets": R, "inputs": input_digests(w, xs)}
+
+
+def input_digests(w, xs):
+    """The seed and the SHA-256 of each rank's input bytes (host copy), so that a
+    result row names the exact inputs it was measured on."""
+    out = []
+    for r, x in enumerate(xs):
+        h = hashlib.sha256()
+        flat = x.reshape(-1).view(torch.uint8)
+        step = 256 << 20
+        for i in range(0, flat.numel(), step):
+            h.update(flat[i:i + step].cpu().numpy().tobytes())
+        out.append({"rank": r, "seed": w.seed * 1009 + r, "sha256": h.hexdigest()})
+    return out
 
 
 def nvlink_bytes_sent(world, n, codec, chunks, rank=0):
@@ -904,8 +918,10 @@ def run_collectives(args, device):
                 torch.cuda.empty_cache()
 
 
-def emulation_config(w, args, sets):
+def emulation_config(w, args, sets, inputs=None):
     cfg = workload_config(w, args)
+    if inputs:
+        cfg["inputs"] = inputs
     if sets > 1:
         cfg["l2"] = ("inputs %d MiB < 4x L2: the steps rotate over %d buffer sets at distinct addresses spanning "
                      ">= %d MiB, so every step reads its inputs from HBM" % (w.N * w.message_bytes >> 20, sets,
@@ -1052,7 +1068,7 @@ def emulation_line(args, res):
     return {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": emulation_config(w, args, res["sets"]),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": emulation_config(w, args, res["sets"], res.get("inputs")),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": d["achieved_gbs"], "peak": peak,
                      "unit": "GB/s", "frac": d["achieved_gbs"] / peak, "traffic": traffic,
                      "frac_dram": None if traffic is None else traffic / sec / 1e9 / peak,

@@ -103,3 +103,16 @@ def test_single_pass_labels_follow_the_launcher_rule():
     tiles_src = open(os.path.join(ROOT, "quantized_precision_all_b200", "csrc", "lpar_tiles.cuh")).read()
     assert "return C == kFP8 ? 512 : 256;" in tiles_src
     assert bench.BULK_MIN_BYTES == 128 * mib and bench.INT3_WARP_MAX_BYTES == 512 * mib
+
+
+def test_input_digests_name_the_exact_bytes():
+    import hashlib
+    import torch
+    import workloads as W
+    w = W.WORKLOADS["small_int4"]
+    xs = W.make_inputs(w, "cpu")
+    d = bench.input_digests(w, xs)
+    for r, x in enumerate(xs):
+        assert d[r]["seed"] == w.seed * 1009 + r
+        assert d[r]["sha256"] == hashlib.sha256(x.view(torch.int16).numpy().tobytes()).hexdigest()
+    assert d[0]["sha256"] != d[1]["sha256"]
