@@ -8,8 +8,10 @@
 // crosses the links is the quantised wire, the sums are formed in FP32.  One
 // launch per rank runs three phases, with the exchange folded into them:
 //   phase A  stage 1 of this rank's message.  Each wire tile is stored straight
-//            into the mailbox of its shard's owner (slot = this rank); when a
-//            chunk of tiles is there, a flag in the owner's memory is raised.
+//            into the mailbox of its shard's owner (slot = this rank; staged in
+//            shared memory first when the owner is on another GPU, so that
+//            the link carries whole 16-B stores); when a chunk of tiles is
+//            there, a flag in the owner's memory is raised.
 //   phase B  stage 2 of this rank's own shard.  Per chunk: wait for the chunk's
 //            flag from every rank, sum the N wires in FP32 in ascending rank
 //            order from +0, requantise, store the reduced tiles into every
@@ -267,10 +269,13 @@ __device__ void peer_phase_a(const PeerPtrs &p, const PeerGeom &g, uint32_t epoc
                     const float a = absmax_bf16x32(x16);
                     Packed<C> q;
                     encode<C, false, false>(x, a, q, NoSink{});
-                    store_block(wst + (t / kBlocksPerTile) * TB, t % kBlocksPerTile, q);
+                    // to another GPU: staged, then whole 16-B stores; in this GPU's memory: direct
+                    // (measured 2-5% faster with every rank in the launch)
+                    if (g.sys) store_block(wst + (t / kBlocksPerTile) * TB, t % kBlocksPerTile, q);
+                    else store_block(dst + (k * kTilesPerCta + t / kBlocksPerTile) * TB, t % kBlocksPerTile, q);
                 }
-                __syncthreads();
-                copy16(dst + k * (kTilesPerCta * TB), wst, (size_t)ntl * TB);
+                __syncthreads();                                 // wst filled; stage[buf] read by all
+                if (g.sys) copy16(dst + k * (kTilesPerCta * TB), wst, (size_t)ntl * TB);
                 buf ^= 1;
             }
         }
