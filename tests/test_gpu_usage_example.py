@@ -1,6 +1,7 @@
 """A short usage example of the Python binding, run on the GPU: the calls a
 user makes first (the all-reduce with and without a caller workspace, the
-reduce-scatter, the all-gather, host-resident messages), with the results
+reduce-scatter, the all-gather, host-resident messages, the peer-memory
+kernel), with the results
 compared bit for bit with the oracle (needs a B200)."""
 import numpy as np
 import pytest
@@ -45,3 +46,9 @@ def test_usage_example():
     assert all(np.array_equal(_bits(a), b) for a, b in zip(ag, ref_ag))
     ref4, _ = O.allreduce(bits, "int4")
     assert all(np.array_equal(h.view(torch.int16).numpy().view(np.uint16), ref4[0]) for h in host)
+
+    # the peer-memory kernel, every rank in one launch; its buffers kept for later calls
+    pb = L.PeerBuffers(N, n, "int4")
+    peer = L.allreduce_peer(xs, "int4", buffers=pb)
+    pb.check()                                               # raises if a wait for a rank gave up
+    assert all(np.array_equal(_bits(o), ref4[0]) for o in peer)
