@@ -297,6 +297,81 @@ def test_peer_wait_gives_up_on_a_rank_that_never_runs(L):
         assert np.array_equal(o.view(torch.int16).cpu().numpy().view(np.uint16), ref[0])
 
 
+@pytest.mark.parametrize("codec", CODECS)
+@pytest.mark.parametrize("N,d,tiles", [(2, 0, 9), (2, 1, 40), (3, 1, 37), (3, 2, 100)])
+def test_peer_one_rank_against_host_played_peers(L, codec, N, d, tiles):
+    """The form one rank per GPU runs (ranks = 1, system-scope flags, wire tiles
+    staged in shared memory and stored into another rank's memory), with the
+    other ranks played by the host: their buffers are pinned host memory, and
+    before the launch the host writes into rank d's buffers everything they
+    would have sent -- their stage-1 tiles of shard d (the oracle's wires), the
+    reduced shards they own (the oracle's reduction) -- and raises the matching
+    flags.  Every wait of the launch is therefore already satisfied (nothing
+    else runs).  Rank d's output, and what its launch stored into the host
+    ranks' mailboxes, gathered wires and flags, must match the oracle."""
+    n = tiles * 2048
+    T, tb = tiles, L.lpar_tile_bytes(codec)
+    xs = inputs(N, n, 8800 + 10 * N + d)
+    P = chunks_per_shard(N, T)
+    slot = -(-T // N)
+    shard = [(j * T // N, (j + 1) * T // N) for j in range(N)]
+    if codec == "bf16":
+        wires = [x.view(np.uint8) for x in xs]
+        ref, _ = O.allreduce(xs, codec)
+        gathered = ref[0].view(np.uint8)
+    else:
+        wires = [O.quantize(x, codec) for x in xs]
+        gathered = O.reduce(wires, 0, T, codec)
+        ref, _ = O.allreduce(xs, codec)
+    mb_bytes, ga_bytes, fl_bytes = (L.lpar_peer_mailbox_bytes(N, n, codec), L.lpar_peer_gather_bytes(n, codec),
+                                    L.lpar_peer_flag_bytes(N, n))
+    assert fl_bytes == 2 * N * P * 4
+    # rank d: device buffers holding what the host-played ranks sent
+    mb = np.zeros(mb_bytes, np.uint8)
+    ga = np.zeros(ga_bytes, np.uint8)
+    fl = np.zeros(2 * N * P, np.uint32)
+    t0, t1 = shard[d]
+    for h in range(N):
+        if h == d:
+            continue
+        mb[h * slot * tb:(h * slot + t1 - t0) * tb] = wires[h][t0 * tb:t1 * tb]
+        fl[h * P:(h + 1) * P] = 1                                  # source h's mailbox chunks of shard d
+        a0, a1 = shard[h]
+        ga[a0 * tb:a1 * tb] = gathered[a0 * tb:a1 * tb]            # shard h, reduced by its owner
+        fl[N * P + h * P:N * P + (h + 1) * P] = 1
+    dev = [Guarded(mb_bytes, fill=0), Guarded(ga_bytes, fill=0), Guarded(fl_bytes, fill=0)]
+    for g, arr in zip(dev, (mb, ga, fl.view(np.uint8))):
+        g.t.copy_(torch.from_numpy(arr))
+    host = {h: [torch.zeros(k, dtype=torch.uint8, pin_memory=True) for k in (mb_bytes, ga_bytes, fl_bytes)]
+            for h in range(N) if h != d}
+    x_d = to_device(xs[d])
+    out_d = Guarded(2 * n, fill=0)
+    status = torch.zeros(8, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    ptrs = lambda k: [dev[k].ptr() if r == d else host[r][k].data_ptr() for r in range(N)]
+    L.lpar_allreduce_peer([x_d.ptr() if r == d else None for r in range(N)],
+                          [out_d.ptr() if r == d else None for r in range(N)], ptrs(0), ptrs(1), ptrs(2), n, codec,
+                          TIMEOUT_NS, status, rank0=d, ranks=1)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0, 0, 0, 1, 0, 0, 0]
+    for g in dev + [out_d, x_d]:
+        g.check()
+    assert np.array_equal(host_u16(out_d), ref[0]), (codec, N, d)
+    for h, (hmb, hga, hfl) in host.items():
+        a0, a1 = shard[h]
+        assert np.array_equal(hmb.numpy()[d * slot * tb:(d * slot + a1 - a0) * tb], wires[d][a0 * tb:a1 * tb])
+        assert np.array_equal(hga.numpy()[t0 * tb:t1 * tb], gathered[t0 * tb:t1 * tb])   # rank d's reduced shard
+        f = hfl.numpy().view(np.uint32)
+        for c in range(P):
+            lo_h, hi_h = a0 + c * (a1 - a0) // P, a0 + (c + 1) * (a1 - a0) // P
+            assert f[d * P + c] == (1 if hi_h > lo_h else 0), ("mailbox flag", h, c)
+            lo_d, hi_d = t0 + c * (t1 - t0) // P, t0 + (c + 1) * (t1 - t0) // P
+            assert f[N * P + d * P + c] == (1 if hi_d > lo_d else 0), ("gathered flag", h, c)
+        untouched = np.ones(mb_bytes, bool)
+        untouched[d * slot * tb:(d * slot + a1 - a0) * tb] = False
+        assert not hmb.numpy()[untouched].any()                      # nothing outside rank d's slot
+
+
 def test_peer_refuses_an_absent_rank_on_this_device(L):
     """A rank outside the launch whose buffers are this GPU's memory would have
     to be a second launch on the same GPU waiting on this one: refused before
