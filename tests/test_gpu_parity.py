@@ -691,7 +691,9 @@ def test_bulk_output_path_ragged_tail(L, codec, N):
 # (nu = 3).  Each point runs at full size on the GPU.  Up to 64 MiB per rank the
 # whole message is compared with the oracle (run over tile ranges on every host
 # core); above, the first and last tile plus 1024 seeded random tiles (a tile's
-# result depends only on that tile of every rank).
+# result depends only on that tile of every rank).  At every point the stage-1
+# wires and the gathered wire (codes and scales) are compared byte for byte at
+# the first and last tile and 1024 random ones (every tile of smaller messages).
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("N", list(W.SWEEP_RANKS))
 def test_sweep_sampled_tiles(L, N):
@@ -714,7 +716,21 @@ def test_sweep_sampled_tiles(L, N):
         outs = [torch.empty_like(x) for x in xs]
         ws = torch.empty(max(L.lpar_workspace_bytes(N, w.n, c) for c in W.SWEEP_CODECS), dtype=torch.uint8,
                          device="cuda")
+        # the stage-1 wires and the gathered wire (codes and scales) at the checked tiles: every
+        # tile up to 1026 tiles, else the sampled ones
+        wt = np.arange(T) if T <= 1026 else (
+            tiles if not full else np.unique(np.concatenate([[0, T - 1], rng.choice(T, 1024, replace=False)])))
+        if full:
+            wsample = [h.reshape(T, 2048)[wt].reshape(-1) for h in host_in]
+        else:
+            pos = np.searchsorted(tiles, wt)
+            wsample = [h.reshape(-1, 2048)[pos].reshape(-1) for h in sample_in]
         for codec in W.SWEEP_CODECS:
+            if codec != "bf16":
+                tb = L.lpar_tile_bytes(codec)
+                wires = [O.quantize(x, codec) for x in wsample]
+                gathered = O.reduce(wires, 0, len(wt), codec)
+                byte_idx = torch.from_numpy((wt[:, None] * tb + np.arange(tb)[None, :]).reshape(-1)).cuda()
             for schedule in ("fused", "single_pass"):
                 L.lpar_allreduce(xs, w.n, codec, outs, ws, ws.numel(), schedule=schedule)
                 torch.cuda.synchronize()
@@ -722,6 +738,11 @@ def test_sweep_sampled_tiles(L, N):
                     g = o if idx is None else o[idx]
                     assert np.array_equal(g.view(torch.int16).cpu().numpy().view(np.uint16), refs[codec]), \
                         (N, mb, codec, schedule)
+                if codec != "bf16":
+                    wb = T * tb
+                    for r in range(N + 1):                       # rank r's wire, then the gathered wire
+                        got = ws[r * wb + byte_idx].cpu().numpy()
+                        assert np.array_equal(got, wires[r] if r < N else gathered), (N, mb, codec, schedule, r)
         del xs, outs, ws
         torch.cuda.empty_cache()
 
