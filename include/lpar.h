@@ -351,7 +351,8 @@ lpar_status_t lpar_allreduce_f32_host(const void *const *host_inputs, int N, siz
  * GPUs (their buffers are memory of another device, or mapped host memory);
  * a rank outside the launch whose buffers are memory of the current device is
  * refused with LPAR_ERR_INVALID_ARG, because two launches on one GPU that
- * wait on each other are not guaranteed to run at the same time.
+ * wait on each other are not guaranteed to run at the same time, and so is
+ * one whose buffers are host memory the GPU cannot reach (not page-locked).
  *
  * timeout_ns (> 0): a wait for another rank's tiles gives up when it has seen
  * no arrival for this long (or after timeout_ns / 128 polls).

@@ -433,15 +433,19 @@ lpar_status_t launch_peer_c(int N, const PeerPtrs &p, const PeerGeom &g, uint32_
     }
 }
 
-// True when `ptr` is memory of the current device (its kernels and this
-// launch's would share the GPU).
-bool on_this_device(const void *ptr, int dev) {
+// A buffer of a rank outside the launch must be memory this GPU can reach and
+// that another launch (on another GPU) or the host can own: another device's
+// memory (peer or IPC-mapped) or mapped host memory.  Memory of the current
+// device would mean a second launch on this GPU waiting on this one;
+// unregistered host memory is not reachable from the kernel.
+bool reachable_elsewhere(const void *ptr, int dev) {
     cudaPointerAttributes a{};
     if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+    if (a.type == cudaMemoryTypeHost) return true;
+    return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device != dev;
 }
 
 size_t tiles_of(size_t n) { return n / kTileElems; }
@@ -498,7 +502,8 @@ LPAR_API lpar_status_t lpar_allreduce_peer(
     if (ranks < N) {
         for (int r = 0; r < N; ++r) {
             if (r >= rank0 && r < rank0 + ranks) continue;
-            if (on_this_device(mailboxes[r], dev) || on_this_device(gathered[r], dev) || on_this_device(flags[r], dev))
+            if (!reachable_elsewhere(mailboxes[r], dev) || !reachable_elsewhere(gathered[r], dev) ||
+                !reachable_elsewhere(flags[r], dev))
                 return LPAR_ERR_INVALID_ARG;
         }
     }

@@ -388,6 +388,17 @@ def test_peer_refuses_an_absent_rank_on_this_device(L):
     assert e.value.status == 1
     torch.cuda.synchronize()
     assert status.tolist() == [0] * 8
+    # host memory the GPU cannot reach (pageable) is refused the same way
+    pageable = [np.zeros(max(k, 16), np.uint8) for k in (L.lpar_peer_mailbox_bytes(N, n, codec),
+                                                          L.lpar_peer_gather_bytes(n, codec),
+                                                          L.lpar_peer_flag_bytes(N, n))]
+    with pytest.raises(L.LparError) as e:
+        L.lpar_allreduce_peer([x, None], [x, None], [bufs[0], pageable[0].ctypes.data],
+                              [bufs[1], pageable[1].ctypes.data], [bufs[2], pageable[2].ctypes.data], n, codec,
+                              TIMEOUT_NS, status, rank0=0, ranks=1)
+    assert e.value.status == 1
+    torch.cuda.synchronize()
+    assert status.tolist() == [0] * 8
 
 
 # ---------------------------------------------------------------------------
