@@ -413,10 +413,11 @@ lpar_status_t launch_peer_cn(const PeerPtrs &p, const PeerGeom &g, uint32_t *sta
     const size_t items = (size_t)g.P * N * g.R;
     const unsigned grid = (unsigned)std::min<size_t>(res, items);
     void *args[] = {const_cast<PeerPtrs *>(&p), const_cast<PeerGeom *>(&g), &status};
-    return cudaLaunchCooperativeKernel((const void *)k_allreduce_peer<C, N>, dim3(grid), dim3(kThreads), args, 0,
-                                       st) == cudaSuccess
-               ? LPAR_OK
-               : LPAR_ERR_CUDA;
+    if (cudaLaunchCooperativeKernel((const void *)k_allreduce_peer<C, N>, dim3(grid), dim3(kThreads), args, 0, st) ==
+        cudaSuccess)
+        return LPAR_OK;
+    cudaGetLastError();                    // a refused launch leaves no error for later calls to find
+    return LPAR_ERR_CUDA;
 }
 
 template <int C>
