@@ -24,24 +24,25 @@
 //
 // Geometry.  T tiles per rank; shard j = tiles [jT/N, (j+1)T/N); every shard
 // is cut into P chunks (chunk c of shard j = its tiles [cS/P, (c+1)S/P), S the
-// shard's size), P = min(ceil(T/N), 1024), so every rank derives the same
-// chunks from (N, T) alone.  Rank j's mailbox holds N slots of ceil(T/N) tiles
-// (slot s = source rank s); rank r's gathered wire holds all T tiles; rank r's
-// flags are N*P words for its mailbox (index s*P + c: source s, chunk c) then
-// N*P words for its gathered wire (index N*P + j*P + c: owner j, chunk c).
+// shard's size), P = min(ceil(ceil(T/N) / 16), 1024), so every rank derives
+// the same chunks from (N, T) alone.  Rank j's mailbox holds N slots of
+// ceil(T/N) tiles (slot s = source rank s); rank r's gathered wire holds all T
+// tiles; rank r's flags are N*P words for its mailbox (index s*P + c: source
+// s, chunk c) then N*P words for its gathered wire (index N*P + j*P + c: owner
+// j, chunk c).
 //
 // Ordering.  A writer's CTA finishes its stores, meets a CTA barrier, and one
-// thread issues a system-scope fence and a release store of the call's epoch
-// into the flag; a waiter polls the flag with system-scope acquire loads until
-// it reaches the epoch, then meets a CTA barrier before any thread reads the
-// data.  The epoch lives in the launching rank's status words: every CTA reads
-// the previous call's epoch when it starts and the last CTA to finish stores
-// the new one, so a call captured in a CUDA graph advances it on every replay.
-// Epochs grow by one per call, so no flag needs resetting; a buffer is
-// never rewritten before every reader of the previous call is done with it
-// (a rank enters call k+1 only after it has decoded every shard of call k,
-// and every shard of call k was reduced only after its mailbox chunks had been
-// read).
+// thread issues a fence and a release store of the call's epoch into the flag;
+// a waiter polls the flag with acquire loads until it reaches the epoch, then
+// meets a CTA barrier before any thread reads the data (system scope when
+// other ranks run on other GPUs, GPU scope when every rank is in the launch).
+// The epoch lives in the launching rank's status words: every CTA reads the
+// previous call's epoch when it starts and the last CTA to finish stores the
+// new one, so a call captured in a CUDA graph advances it on every replay.
+// Epochs grow by one per call, so no flag needs resetting; a buffer is never
+// rewritten before every reader of the previous call is done with it (a rank
+// enters call k+1 only after it has decoded every shard of call k, and every
+// shard of call k was reduced only after its mailbox chunks had been read).
 //
 // Waits are bounded: a wait that sees no progress for timeout_ns (or after
 // timeout_ns / 128 polls) records the failure in the caller's status words
