@@ -136,6 +136,12 @@ def _worker(rank, world, port, codec, q):
             out = ar.allreduce(x, codec)
             ar.check()
             results.append(out.view(torch.int16).numpy().copy())
+        # below the threshold the message goes through the BF16 passthrough, in its own region
+        n = 5 * 2048
+        x = inputs(world, n, 400)[rank]
+        out = ar.allreduce(x, codec, min_quant_bytes=2 * n + 2)
+        ar.check()
+        results.append(out.view(torch.int16).numpy().copy())
         epochs = ar.epochs()
         ar.release()
         assert not ops.blocks, "every mapping closed and the own regions freed"
@@ -176,8 +182,14 @@ def test_peer_allreduce_host_side(world, codec):
                              codec)
         for r in range(world):
             assert np.array_equal(got[r][0][k].view(np.uint16), ref[0]), (codec, k, r)
+    ref, used = O.allreduce([x.view(torch.int16).numpy().view(np.uint16) for x in inputs(world, 5 * 2048, 400)],
+                            codec, 2 * 5 * 2048 + 2)
+    assert used == "bf16"
     for r in range(world):
-        assert got[r][1] == {(5 * 2048, codec): 3, (12 * 2048, codec): 1}
+        assert np.array_equal(got[r][0][4].view(np.uint16), ref[0]), (codec, "threshold", r)
+        want = {(5 * 2048, codec): 3, (12 * 2048, codec): 1}
+        want[(5 * 2048, "bf16")] = want.get((5 * 2048, "bf16"), 0) + 1
+        assert got[r][1] == want
 
 
 def _absent_worker(rank, world, port, q):
