@@ -328,3 +328,33 @@ def test_peer_ipc_argument_errors(L):
     assert lib.lpar_peer_close(None) == 1
     with pytest.raises(ValueError):
         L.lpar_peer_import(b"\0" * 10)
+
+
+def test_peer_sizes_fit_the_chunk_geometry(L):
+    """For many (N, T): the library's flag count gives P chunks per shard of at
+    least 16 tiles (or one tile when shards are smaller) and at most 1024; the
+    chunks [cS/P, (c+1)S/P) tile every shard exactly; a mailbox slot holds the
+    largest shard; the gathered wire holds every tile."""
+    for N in range(1, 9):
+        for T in list(range(1, 70)) + [127, 128, 129, 1023, 1025, 4099, 16 * 1024 * 8 + 5, 1 << 20]:
+            n = T * 2048
+            P = L.lpar_peer_flag_bytes(N, n) // (2 * N * 4)
+            smax = -(-T // N)
+            assert 1 <= P <= 1024 and P == min(max(-(-smax // 16), 1), 1024), (N, T, P)
+            tb = L.lpar_tile_bytes("int4")
+            assert L.lpar_peer_mailbox_bytes(N, n, "int4") == N * smax * tb
+            assert L.lpar_peer_gather_bytes(n, "int4") == T * tb
+            if T > 5000:
+                continue                                   # the partition check below is O(N P)
+            covered = 0
+            for j in range(N):
+                base, S = j * T // N, (j + 1) * T // N - j * T // N
+                assert S <= smax
+                prev = base
+                for c in range(P):
+                    lo, hi = base + c * S // P, base + (c + 1) * S // P
+                    assert lo == prev and lo <= hi
+                    prev = hi
+                    covered += hi - lo
+                assert prev == base + S
+            assert covered == T
