@@ -24,8 +24,9 @@
 //
 // Geometry.  T tiles per rank; shard j = tiles [jT/N, (j+1)T/N); every shard
 // is cut into P chunks (chunk c of shard j = its tiles [cS/P, (c+1)S/P), S the
-// shard's size), P = min(ceil(ceil(T/N) / 16), 1024), so every rank derives
-// the same chunks from (N, T) alone.  Rank j's mailbox holds N slots of
+// shard's size), P = min(ceil(ceil(T/N) / chunk), 1024) for the chunk size of
+// peer_chunks (1 to 16 tiles by the message size), so every rank derives the
+// same chunks from (N, T) alone.  Rank j's mailbox holds N slots of
 // ceil(T/N) tiles (slot s = source rank s); rank r's gathered wire holds all T
 // tiles; rank r's flags are N*P words for its mailbox (index s*P + c: source
 // s, chunk c) then N*P words for its gathered wire (index N*P + j*P + c: owner
@@ -90,16 +91,23 @@ struct PeerGeom {
 // Status words (LPAR_PEER_STATUS_WORDS, in the launching GPU's memory).
 constexpr int kStFail = 0, kStPhase = 1, kStRank = 2, kStIndex = 3, kStEpoch = 4, kStDone = 5;
 
-// Chunks per shard: shards of up to ceil(T/N) tiles cut into chunks of at
-// least kPeerChunkTiles tiles, at most kPeerMaxChunks chunks.  Every flag costs
-// a CTA barrier, a fence and a wait, so a chunk should carry several tiles;
-// the ranks' shards should still give every CTA work.
+// Chunks per shard.  Every flag costs a CTA barrier, a fence and a wait, so a
+// chunk should carry several tiles; a small message should still give every
+// CTA work.  Chunk size: about N*T/592 tiles (with every rank in one launch
+// that makes about 592 phase-A items, four CTAs on each of 148 SMs), at least
+// one and at most kPeerChunkTiles, a whole number of 4-tile groups above four;
+// at most kPeerMaxChunks chunks per shard.  Measured on B200 with every rank
+// in one launch: 20-30% faster than 16-tile chunks at 1 MiB per rank, the
+// same from 16 MiB.  It depends on (N, T) alone, so every rank derives the
+// same chunks.
 constexpr unsigned kPeerMaxChunks = 1024;
 constexpr unsigned kPeerChunkTiles = 16;
 
 inline unsigned peer_chunks(int N, size_t T) {
     const size_t s = (T + (size_t)N - 1) / (size_t)N;
-    const size_t c = (s + kPeerChunkTiles - 1) / kPeerChunkTiles;
+    size_t ct = std::min<size_t>(std::max<size_t>(((size_t)N * T + 591) / 592, 1), kPeerChunkTiles);
+    if (ct > 4) ct = (ct + 3) / 4 * 4;
+    const size_t c = (s + ct - 1) / ct;
     return (unsigned)std::min<size_t>(std::max<size_t>(c, 1), kPeerMaxChunks);
 }
 

@@ -278,12 +278,14 @@ def test_peer_buffer_bytes(L):
     assert L.lpar_peer_mailbox_bytes(1, n, "mxfp4") == 10 * 1088
     assert L.lpar_peer_gather_bytes(n, "int3") == 10 * 896
     assert L.lpar_peer_gather_bytes(n, "fp8") == 10 * 2304
-    # P = min(ceil(ceil(T / N) / 16), 1024) chunks per shard (chunks of at least 16 tiles)
-    assert L.lpar_peer_flag_bytes(3, n) == 2 * 3 * 1 * 4
+    # chunks of about N T / 592 tiles (1 to 16, a multiple of 4 above 4), at most 1024 per shard
+    assert L.lpar_peer_flag_bytes(3, n) == 2 * 3 * 4 * 4                  # 1-tile chunks: P = ceil(10 / 3)
     assert L.lpar_peer_flag_bytes(8, 2048 << 20) == 2 * 8 * 1024 * 4      # P capped at 1024
-    assert L.lpar_peer_flag_bytes(8, 2048 * 8 * 1024) == 2 * 8 * 64 * 4
+    assert L.lpar_peer_flag_bytes(8, 2048 * 8 * 1024) == 2 * 8 * 64 * 4  # 16-tile chunks
     assert L.lpar_peer_flag_bytes(8, 2048 * (8 * 16 * 1000 + 1)) == 2 * 8 * 1001 * 4
-    assert L.lpar_peer_flag_bytes(2, 2048 * 33) == 2 * 2 * 2 * 4
+    assert L.lpar_peer_flag_bytes(2, 2048 * 256) == 2 * 2 * 128 * 4       # 1 MiB per rank: 1-tile chunks
+    assert L.lpar_peer_flag_bytes(8, 2048 * 256) == 2 * 8 * 8 * 4         # N T / 592 = 3.5: 4-tile chunks
+    assert L.lpar_peer_flag_bytes(2, 2048 * 4096) == 2 * 2 * 128 * 4      # 13.8 rounds to 16-tile chunks
     for bad in (L.lpar_peer_mailbox_bytes(0, n, "int4"), L.lpar_peer_mailbox_bytes(9, n, "int4"),
                 L.lpar_peer_mailbox_bytes(2, n + 1, "int4"), L.lpar_peer_mailbox_bytes(2, n, 7),
                 L.lpar_peer_gather_bytes(n + 2, "int4"), L.lpar_peer_gather_bytes(n, 9),
@@ -331,8 +333,8 @@ def test_peer_ipc_argument_errors(L):
 
 
 def test_peer_sizes_fit_the_chunk_geometry(L):
-    """For many (N, T): the library's flag count gives P chunks per shard of at
-    least 16 tiles (or one tile when shards are smaller) and at most 1024; the
+    """For many (N, T): the library's flag count gives P chunks per shard, of
+    1 to 16 tiles by the message size, at most 1024; the
     chunks [cS/P, (c+1)S/P) tile every shard exactly; a mailbox slot holds the
     largest shard; the gathered wire holds every tile."""
     for N in range(1, 9):
@@ -340,7 +342,9 @@ def test_peer_sizes_fit_the_chunk_geometry(L):
             n = T * 2048
             P = L.lpar_peer_flag_bytes(N, n) // (2 * N * 4)
             smax = -(-T // N)
-            assert 1 <= P <= 1024 and P == min(max(-(-smax // 16), 1), 1024), (N, T, P)
+            ct = min(max(-(-(N * T) // 592), 1), 16)
+            ct = -(-ct // 4) * 4 if ct > 4 else ct
+            assert 1 <= P <= 1024 and P == min(max(-(-smax // ct), 1), 1024), (N, T, P)
             tb = L.lpar_tile_bytes("int4")
             assert L.lpar_peer_mailbox_bytes(N, n, "int4") == N * smax * tb
             assert L.lpar_peer_gather_bytes(n, "int4") == T * tb

@@ -7,7 +7,7 @@ when fewer than two GPUs are visible).
   several calls and codecs.
 - A rank that never makes its call (it leaves between steps, with nothing in
   flight): the other rank's waits give up after the timeout, `check()` raises
-  PeerTimeout naming phase 1, and the process carries on.
+  PeerTimeout naming the phase that gave up first, and the process carries on.
 
 Children run with NCCL's NVLink SHARP off (NCCL_NVLS_ENABLE=0) and a short
 process-group timeout."""
@@ -127,5 +127,5 @@ def test_cross_gpu_allreduce_matches_the_oracle(kind):
 
 def test_peer_allreduce_reports_a_rank_that_never_calls():
     got = _spawn(_absent_worker, 2)
-    assert got[0] is not None and "phase 1" in got[0], got
+    assert got[0] is not None and ("phase 1" in got[0] or "phase 2" in got[0]), got
     assert got[1] is None
