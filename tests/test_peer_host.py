@@ -1,13 +1,15 @@
 """PeerAllreduce's host side on CPU with gloo, world sizes 2 to 4.
 
-The library is replaced by a stand-in whose memory is POSIX shared memory (so
-an address in one process maps another process's buffer after the handle
-exchange, as CUDA IPC does) and whose "kernel" runs the peer protocol in
-Python, each process its own rank, concurrently: phase A stores the oracle's
-stage-1 tiles of every shard into the owner's mailbox slot and raises the
-owner's flag; phase B waits for every rank's flag of its own shard, reduces
-with the oracle and stores the result into every rank's gathered wire with a
-flag; phase C waits for every shard's flag and decodes with the oracle.  This
+The library's calls are replaced by a stand-in whose memory is POSIX shared
+memory (so an address in one process maps another process's buffer after the
+handle exchange, as CUDA IPC does) and whose "kernel" runs the peer protocol in
+Python, with the library's buffer sizes and the kernel's chunk geometry and
+flag indices, each process its own rank, concurrently: phase A stores the
+oracle's stage-1 tiles of every chunk into the owner's mailbox slot and raises
+the owner's flag for that chunk; phase B waits for every rank's flag of each
+chunk of its own shard, reduces it with the oracle and stores the result into
+every rank's gathered wire with a flag; phase C waits for every chunk's flag
+and decodes with the oracle.  This
 checks the regions, the handle exchange, the pointer arrays, the epochs over
 repeated calls and sizes, and the timeout report when a rank never runs.
 Every rank's result must equal the oracle's all-reduce bit for bit."""
@@ -63,21 +65,27 @@ class ShmOps:
         shm.close()
         shm.unlink()
 
+    # the library's buffer sizes (host functions, no GPU needed): the stand-in lays its
+    # buffers out as the kernel does
     @staticmethod
     def mailbox_bytes(N, n, codec):
-        T = n // 2048
-        return N * -(-T // N) * O.tile_bytes(codec)
+        from quantized_precision_all_b200 import lpar as L
+        return L.lpar_peer_mailbox_bytes(N, n, codec)
 
     @staticmethod
     def gather_bytes(n, codec):
-        return n // 2048 * O.tile_bytes(codec)
+        from quantized_precision_all_b200 import lpar as L
+        return L.lpar_peer_gather_bytes(n, codec)
 
     @staticmethod
     def flag_bytes(N, n):
-        return 2 * N * 4                                   # one chunk per shard
+        from quantized_precision_all_b200 import lpar as L
+        return L.lpar_peer_flag_bytes(N, n)
 
-    def _wait(self, addr, index, epoch, deadline, status, phase, rank):
-        flags = self.view(addr)[:8 * 4 * 2].view(np.uint32)
+    def _flags(self, addr, words):
+        return self.view(addr)[:4 * words].view(np.uint32)
+
+    def _wait(self, flags, index, epoch, deadline, status, phase, rank):
         while int(flags[index]) < epoch:
             if time.monotonic() > deadline:
                 status[:4] = torch.tensor([1, phase, rank, index], dtype=torch.int32)
@@ -92,29 +100,53 @@ class ShmOps:
             self._run(inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0, epoch)
         status[4] = epoch
 
-    def _run(self, inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, rank0, epoch):
-        N, r, T, tb = len(mailboxes), rank0, n // 2048, O.tile_bytes(codec)
+    def _run(self, inputs, outputs, mailboxes, gathered, flags, n, codec, timeout_ns, status, me, epoch):
+        """The kernel's protocol, chunk by chunk, with its geometry and flag indices:
+        shard j = tiles [jT/N, (j+1)T/N), cut into P chunks [cS/P, (c+1)S/P); rank r's
+        flags: s*P + c for source s's mailbox chunk c, N*P + j*P + c for owner j's
+        gathered chunk c."""
+        N, T, tb = len(mailboxes), n // 2048, O.tile_bytes(codec)
+        P = self.flag_bytes(N, n) // (2 * N * 4)
         slot = -(-T // N)
         shard = [(j * T // N, (j + 1) * T // N) for j in range(N)]
-        wire = O.quantize(inputs[r].view(torch.int16).numpy().view(np.uint16), codec)
-        for j, (t0, t1) in enumerate(shard):                       # phase A
-            self.view(mailboxes[j])[r * slot * tb:(r * slot + t1 - t0) * tb] = wire[t0 * tb:t1 * tb]
-            self.view(flags[j])[:8 * N].view(np.uint32)[r] = epoch
+
+        def chunk(j, c):
+            b, e = shard[j]
+            return b + c * (e - b) // P, b + (c + 1) * (e - b) // P
+
+        wire = O.quantize(inputs[me].view(torch.int16).numpy().view(np.uint16), codec)
+        for c in range(P):                                         # phase A, chunk-major
+            for j in range(N):
+                lo, hi = chunk(j, c)
+                if lo == hi:
+                    continue
+                base = shard[j][0]
+                self.view(mailboxes[j])[(me * slot + lo - base) * tb:(me * slot + hi - base) * tb] = \
+                    wire[lo * tb:hi * tb]
+                self._flags(flags[j], 2 * N * P)[me * P + c] = epoch
         deadline = time.monotonic() + timeout_ns * 1e-9
-        for s in range(N):                                         # phase B
-            if not self._wait(flags[r], s, epoch, deadline, status, 1, r):
-                return
-        t0, t1 = shard[r]
-        mine = self.view(mailboxes[r])
-        red = O.reduce([mine[s * slot * tb:(s * slot + t1 - t0) * tb] for s in range(N)], 0, t1 - t0, codec)
-        for q in range(N):
-            self.view(gathered[q])[t0 * tb:t1 * tb] = red[:(t1 - t0) * tb]
-            self.view(flags[q])[:8 * N].view(np.uint32)[N + r] = epoch
-        for j in range(N):                                         # phase C
-            if not self._wait(flags[r], N + j, epoch, deadline, status, 2, r):
-                return
-        dec = O.decode(self.view(gathered[r])[:T * tb].copy(), n, codec)
-        outputs[r].copy_(torch.from_numpy(dec.view(np.int16).copy()).view(torch.bfloat16))
+        mine = self._flags(flags[me], 2 * N * P)
+        base = shard[me][0]
+        box = self.view(mailboxes[me])
+        for c in range(P):                                         # phase B: my shard
+            lo, hi = chunk(me, c)
+            if lo == hi:
+                continue
+            for s in range(N):
+                if not self._wait(mine, s * P + c, epoch, deadline, status, 1, me):
+                    return
+            wires = [box[(s * slot + lo - base) * tb:(s * slot + hi - base) * tb] for s in range(N)]
+            red = O.reduce(wires, 0, hi - lo, codec)[:(hi - lo) * tb]
+            for q in range(N):
+                self.view(gathered[q])[lo * tb:hi * tb] = red
+                self._flags(flags[q], 2 * N * P)[N * P + me * P + c] = epoch
+        for c in range(P):                                         # phase C: every shard
+            for j in range(N):
+                lo, hi = chunk(j, c)
+                if lo < hi and not self._wait(mine, N * P + j * P + c, epoch, deadline, status, 2, me):
+                    return
+        dec = O.decode(self.view(gathered[me])[:T * tb].copy(), n, codec)
+        outputs[me].copy_(torch.from_numpy(dec.view(np.int16).copy()).view(torch.bfloat16))
 
 
 def inputs(N, n, seed):
@@ -221,5 +253,7 @@ def test_peer_allreduce_reports_a_rank_that_never_runs():
     got = spawn(_absent_worker, 2)
     err, status = got[0]
     assert err is not None and "phase 1" in err, err
-    assert status[:3] == [1, 1, 0] and status[3] == 1              # waiting for source 1's mailbox flag
+    from quantized_precision_all_b200 import lpar as L
+    P = L.lpar_peer_flag_bytes(2, 4 * 2048) // (2 * 2 * 4)
+    assert status[:3] == [1, 1, 0] and status[3] == P              # source 1's mailbox flag of chunk 0
     assert got[1][0] is None
