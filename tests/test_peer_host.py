@@ -28,11 +28,17 @@ from oracle import oracle as O
 
 
 class ShmOps:
-    """A stand-in for the library's peer calls over shared memory."""
+    """A stand-in for the library's peer calls over shared memory; `jitter`
+    seeds random pauses between chunks (to vary the interleavings)."""
 
-    def __init__(self):
+    def __init__(self, jitter=None):
         self.blocks = {}
         self.next = 1 << 40
+        self.rng = np.random.default_rng(jitter) if jitter is not None else None
+
+    def _pause(self):
+        if self.rng is not None and self.rng.random() < 0.3:
+            time.sleep(float(self.rng.random()) * 0.003)
 
     def _add(self, shm):
         base = self.next
@@ -124,6 +130,7 @@ class ShmOps:
                 self.view(mailboxes[j])[(me * slot + lo - base) * tb:(me * slot + hi - base) * tb] = \
                     wire[lo * tb:hi * tb]
                 self._flags(flags[j], 2 * N * P)[me * P + c] = epoch
+                self._pause()
         deadline = time.monotonic() + timeout_ns * 1e-9
         mine = self._flags(flags[me], 2 * N * P)
         base = shard[me][0]
@@ -140,6 +147,7 @@ class ShmOps:
             for q in range(N):
                 self.view(gathered[q])[lo * tb:hi * tb] = red
                 self._flags(flags[q], 2 * N * P)[N * P + me * P + c] = epoch
+            self._pause()
         for c in range(P):                                         # phase C: every shard
             for j in range(N):
                 lo, hi = chunk(j, c)
@@ -257,3 +265,37 @@ def test_peer_allreduce_reports_a_rank_that_never_runs():
     P = L.lpar_peer_flag_bytes(2, 4 * 2048) // (2 * 2 * 4)
     assert status[:3] == [1, 1, 0] and status[3] == P              # source 1's mailbox flag of chunk 0
     assert got[1][0] is None
+
+
+def _stress_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from quantized_precision_all_b200.distributed import PeerAllreduce
+        ar = PeerAllreduce(ops=ShmOps(jitter=1000 + rank), timeout_ns=60_000_000_000, device=torch.device("cpu"))
+        results = []
+        for k in range(8):                                     # epochs 1..4 on each of two regions
+            codec = ("int4", "fp8")[k % 2]
+            x = inputs(world, 40 * 2048, 700 + k)[rank]
+            results.append(ar.allreduce(x, codec).view(torch.int16).numpy().copy())
+            ar.check()
+        epochs = ar.epochs()
+        ar.release()
+        q.put((rank, results, epochs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_protocol_under_random_interleavings():
+    """Three ranks pausing at random between chunks (each its own seed), eight calls
+    over two regions: every result equals the oracle's, the epochs count the calls."""
+    world = 3
+    got = spawn(_stress_worker, world)
+    for k in range(8):
+        codec = ("int4", "fp8")[k % 2]
+        ref, _ = O.allreduce([x.view(torch.int16).numpy().view(np.uint16) for x in inputs(world, 40 * 2048, 700 + k)],
+                             codec)
+        for r in range(world):
+            assert np.array_equal(got[r][0][k].view(np.uint16), ref[0]), (k, r)
+    for r in range(world):
+        assert got[r][1] == {(40 * 2048, "int4"): 4, (40 * 2048, "fp8"): 4}
