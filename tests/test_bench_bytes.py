@@ -116,3 +116,29 @@ def test_input_digests_name_the_exact_bytes():
         assert d[r]["seed"] == w.seed * 1009 + r
         assert d[r]["sha256"] == hashlib.sha256(x.view(torch.int16).numpy().tobytes()).hexdigest()
     assert d[0]["sha256"] != d[1]["sha256"]
+
+
+def test_buffer_sets_span_four_l2_at_distinct_addresses():
+    """The rotated buffer sets of back-to-back timing: at least 512 MiB in all (4x the
+    126 MB L2), every set's inputs equal to the originals, no two buffers sharing
+    bytes; a workload already larger than that gets one set (its own buffers)."""
+    import torch
+    N, n = 2, 2048 * 64                                    # 256 KiB of BF16 per rank
+    xs = [torch.full((n,), float(r + 1), dtype=torch.bfloat16) for r in range(N)]
+    sets = bench.BufferSets(xs, n, 4096, torch.device("cpu"), rotate=8 << 20)
+    set_bytes = N * n * 2 + N * n * 2 + 4096
+    assert sets.R == -(-(8 << 20) // set_bytes) and sets.R * set_bytes >= 8 << 20
+    spans = []
+    for i in range(sets.R):
+        for r in range(N):
+            assert torch.equal(sets.inputs[i][r], xs[r])
+            t = sets.inputs[i][r]
+            spans.append((t.data_ptr(), t.data_ptr() + t.numel() * 2))
+            o = sets.outputs[i][r]
+            spans.append((o.data_ptr(), o.data_ptr() + o.numel() * 2))
+        spans.append((sets.ws[i].data_ptr(), sets.ws[i].data_ptr() + sets.ws_bytes))
+    spans.sort()
+    assert all(a1 <= b0 for (a0, a1), (b0, b1) in zip(spans, spans[1:]))
+    assert bench.ROTATE_BYTES == 512 << 20
+    big = bench.BufferSets(xs, n, 4096, torch.device("cpu"), rotate=1024)
+    assert big.R == 1 and big.inputs[0][0] is xs[0]
