@@ -142,3 +142,46 @@ def test_buffer_sets_span_four_l2_at_distinct_addresses():
     assert bench.ROTATE_BYTES == 512 << 20
     big = bench.BufferSets(xs, n, 4096, torch.device("cpu"), rotate=1024)
     assert big.R == 1 and big.inputs[0][0] is xs[0]
+
+
+def test_min_dram_bytes():
+    """Inputs read once, the N stage-1 wires and the gathered wire written once, the N
+    outputs written (the wires' read-back may come from L2); BF16 has no stage-1 wire."""
+    n = 2048 * 10
+    assert bench.min_dram_bytes("int4", 2, n) == 2 * 2 * n + 2 * 10 * 1152 + 10 * 1152 + 2 * 2 * n
+    assert bench.min_dram_bytes("fp8", 8, n) == 8 * 2 * n + 8 * 10 * 2304 + 10 * 2304 + 8 * 2 * n
+    assert bench.min_dram_bytes("bf16", 4, n) == 4 * 2 * n + 2 * n + 4 * 2 * n
+
+
+def test_nvlink_bytes_sent():
+    """Per rank and chunk: its wire minus its own shard (the all-to-all), then its
+    padded shard to each of the other ranks (the all-gather)."""
+    tb = 1152
+    n = 2048 * 10
+    # one chunk, 2 ranks: shards [0, 5), [5, 10)
+    assert bench.nvlink_bytes_sent(2, n, "int4", 1, 0) == 10 * tb - 5 * tb + 1 * 5 * tb
+    # 3 ranks: shards [0, 3), [3, 6), [6, 10); slots padded to 4 tiles
+    assert bench.nvlink_bytes_sent(3, n, "int4", 1, 0) == 10 * tb - 3 * tb + 2 * 4 * tb
+    assert bench.nvlink_bytes_sent(3, n, "int4", 1, 2) == 10 * tb - 4 * tb + 2 * 4 * tb
+    # two chunks of 5 tiles, 2 ranks: shards [0, 2), [2, 5) in each, slots of 3 tiles
+    assert bench.nvlink_bytes_sent(2, n, "int4", 2, 0) == 2 * (5 * tb - 2 * tb + 3 * tb)
+
+
+def test_distributed_line_carries_the_contract_keys():
+    """The multi-GPU JSON line: the contract's keys, the whole-job value, an NVLink roofline."""
+    import argparse
+    import workloads as W
+    w = W.WORKLOADS["large_int3_int4"]
+    args = argparse.Namespace(steps=10, warmup=3, schedule="auto", backend="nccl", chunks=4, exchange="peer")
+    res = {"w": w, "ms": 50.0, "sent": 10 ** 9, "launches_per_step": 2, "clocks": {"sm_mhz": 1965.0},
+           "e2e": None, "exchange": "peer"}
+    line = bench.distributed_line(args, 4, res)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "gpu_launches", "clocks", "e2e"):
+        assert k in line, k
+    assert line["n_gpus"] == 4 and line["scaling"] == "weak" and line["gpu_launches"] == 20
+    assert line["value"] == pytest.approx(4 * w.message_bytes * len(w.codecs) * 10 / 50e-3 / 1e9)
+    rf = line["roofline"]
+    assert rf["bound"] == "nvlink" and rf["peak"] == bench.NVLINK_GBS
+    assert rf["achieved"] == pytest.approx(10 ** 9 / 5e-3 / 1e9) and rf["frac"] == pytest.approx(rf["achieved"] / 770.0)
+    assert line["config"]["exchange"] == "peer" and line["config"]["ranks"] == 4
