@@ -185,3 +185,20 @@ def test_distributed_line_carries_the_contract_keys():
     assert rf["bound"] == "nvlink" and rf["peak"] == bench.NVLINK_GBS
     assert rf["achieved"] == pytest.approx(10 ** 9 / 5e-3 / 1e9) and rf["frac"] == pytest.approx(rf["achieved"] / 770.0)
     assert line["config"]["exchange"] == "peer" and line["config"]["ranks"] == 4
+
+
+def test_clock_summary_from_samples():
+    """The clock record: median SM clock, the highest max clock, every throttle reason
+    seen Active, malformed lines skipped; no samples gives an empty record."""
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.lines = ["1965, 1965, 812.4, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+                "1710, 1965, 999.8, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+                "1800, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+                "garbage line",
+                "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    s = cs.summary()
+    assert s == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    cs.lines = ["1500, 1965, 700, 0x8, Active, Not Active, Active, Not Active"]
+    assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    cs.lines = []
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
