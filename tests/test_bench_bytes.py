@@ -202,3 +202,34 @@ def test_clock_summary_from_samples():
     assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     cs.lines = []
     assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_emulation_line_carries_the_contract_keys():
+    """The one-GPU JSON line: the contract's keys, the whole-job value, and the roofline of
+    the dominant kernel from its live launch time and the committed ncu traffic."""
+    import argparse
+    import workloads as W
+    w = W.WORKLOADS["large_int3_int4"]
+    args = argparse.Namespace(steps=20, warmup=3, schedule="auto", eager=False)
+    n = w.n
+    kern = {}
+    for k, ms in (("k_allreduce_single_warp<int3,N=2>", 0.86), ("k_allreduce_single<int4,N=2>", 0.88)):
+        codec = "int3" if "int3" in k else "int4"
+        alg = bench.algorithmic_bytes(k, codec, 2, n)
+        kern[k] = {"ms_total": ms * 20, "launches": 20, "ms_per_launch": ms, "algorithmic_bytes": alg,
+                   "min_dram_bytes": bench.min_dram_bytes(codec, 2, n), "achieved_gbs": alg / (ms * 1e-3) / 1e9}
+    res = {"w": w, "ms": 1.74 * 20, "kern": kern, "clocks": {"sm_mhz": 1965.0, "reasons": []},
+           "launches_per_step": 2, "e2e": {"value": 45.0}, "cpu": {"value": 0.6}, "accuracy": None, "sets": 1,
+           "inputs": [{"rank": 0, "seed": 4036, "sha256": "x"}]}
+    line = bench.emulation_line(args, res)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "gpu_launches", "clocks", "e2e", "cpu_baseline"):
+        assert k in line, k
+    assert line["n_gpus"] == 1 and line["gpu_launches"] == 40
+    assert line["value"] == pytest.approx(2 * w.message_bytes * 2 / 1.74e-3 / 1e9)
+    rf = line["roofline"]
+    assert rf["kernel"] == "k_allreduce_single<int4,N=2>" and rf["bound"] == "hbm"
+    assert rf["frac"] == pytest.approx(rf["achieved"] / rf["peak"])
+    for k in ("achieved", "peak", "unit", "frac", "traffic"):
+        assert k in rf
+    assert line["config"]["inputs"][0]["seed"] == 4036
