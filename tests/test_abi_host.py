@@ -362,3 +362,18 @@ def test_peer_sizes_fit_the_chunk_geometry(L):
                     covered += hi - lo
                 assert prev == base + S
             assert covered == T
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the Python package without liblpar.so: importing the binding (or the
+    cross-process module built on it) raises OSError -- there is no fallback path."""
+    import shutil
+    import sys
+    pkg = tmp_path / "quantized_precision_all_b200"
+    pkg.mkdir()
+    for f in ("__init__.py", "lpar.py", "distributed.py"):
+        shutil.copy(os.path.join(ROOT, "quantized_precision_all_b200", f), pkg / f)
+    for mod in ("quantized_precision_all_b200.lpar", "quantized_precision_all_b200.distributed"):
+        r = subprocess.run([sys.executable, "-c", "import %s" % mod], cwd=tmp_path, capture_output=True, text=True,
+                           env={**os.environ, "PYTHONPATH": str(tmp_path)})
+        assert r.returncode != 0 and "OSError" in r.stderr, (mod, r.stderr[-500:])
