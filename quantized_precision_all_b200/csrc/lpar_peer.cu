@@ -97,9 +97,9 @@ constexpr int kStFail = 0, kStPhase = 1, kStRank = 2, kStIndex = 3, kStEpoch = 4
 // that makes about 592 phase-A items, four CTAs on each of 148 SMs), at least
 // one and at most kPeerChunkTiles, a whole number of 4-tile groups above four;
 // at most kPeerMaxChunks chunks per shard.  Measured on B200 with every rank
-// in one launch: 20-30% faster than 16-tile chunks at 1 MiB per rank, the
-// same from 16 MiB.  It depends on (N, T) alone, so every rank derives the
-// same chunks.
+// in one launch: 20-30% faster than 16-tile chunks at 1 MiB per rank; from
+// 16 MiB it gives 16-tile chunks.  It depends on (N, T) alone, so every rank
+// derives the same chunks.
 constexpr unsigned kPeerMaxChunks = 1024;
 constexpr unsigned kPeerChunkTiles = 16;
 
